@@ -1,0 +1,420 @@
+"""Benchmark of the paged decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one pass of the whole decode path over one batch: copy-on-write block
+copies (when the step has any), the slot-mapped append of every sequence's new
+token, and paged decode attention over the block tables.  Inputs sit in HBM when
+the timed region starts; the KV bytes a step reads (about 1.2 GB for the default
+workload) are far larger than the 126 MB L2, so no flush is needed between steps.
+
+The metric is throughput in GB/s of algorithmic bytes: the K and V rows of every
+context token, q and the output, block tables and lengths, plus the appended rows.
+Whole-block over-reads and the context-split workspace traffic are not counted.
+Sequences/s is reported beside it.
+
+Under torchrun each rank runs its own batch (seed + rank) on its own GPU: the path
+shards by sequence with no data exchange (weak scaling).  Timing is by CUDA events,
+max over ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (rank 0
+only), on a bounded sample of sequences of the same workload per step.
+"""
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from paged_kv_cache_363_b200 import workloads as W  # noqa: E402
+
+METRIC = "paged decode attention KV HBM GB/s (% of B200 peak) and sequences/sec"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2 ** 20
+
+
+# ------------------------------------------------------------------ helpers shared with the tests
+
+def rank_seed(seed, rank):
+    """Each rank draws its own batch: same shapes and distributions, other values."""
+    return int(seed) + 1000 * int(rank)
+
+
+def reduce_max(x, device=None):
+    """Max of a scalar over the ranks of the default process group (x itself if none)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profile_traffic(kernel, workload):
+    """dram bytes per launch from the committed ncu summary for this kernel and workload,
+    if its recorded source hash still matches the kernel source; else None."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "%s_%s.md" % (kernel, workload))
+    src = os.path.join(ROOT, "paged_kv_cache_363_b200", "csrc", "pa_decode.cu")
+    try:
+        with open(src, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()[:16]
+        fields = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and line.startswith("- "):
+                    k, v = line[2:].split(":", 1)
+                    fields[k.strip()] = v.strip().strip("`")
+        if fields.get("source_sha256_16") != h:
+            return None
+        return float(fields["traffic_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while the timed region runs."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index, interval=0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.interval = interval
+        self._stop = threading.Event()
+        self._thread = None
+        self.h = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = int(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self.h = None
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(int(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)))
+        try:
+            bits = int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+        except Exception:
+            bits = int(nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h))
+        for b, name in self.REASONS.items():
+            if bits & b:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                return
+            time.sleep(self.interval)
+
+    def __enter__(self):
+        if self.h is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+def workload_config(wl, partition, batch=None):
+    cfg = {"workload": wl.name, "num_heads": wl.num_heads, "num_kv_heads": wl.num_kv_heads,
+           "head_dim": wl.head_dim, "block_size": wl.block_size, "num_blocks": wl.num_blocks,
+           "partition_size": partition, "seed": wl.seed}
+    if isinstance(wl, W.CowWorkload):
+        cfg.update(num_seqs=wl.num_seqs, prompts=wl.num_prompts, streams_per_prompt=wl.streams_per_prompt)
+    else:
+        cfg.update(num_seqs=wl.num_seqs, context_tokens=int(np.sum(wl.context_lens)),
+                   max_context_len=int(np.max(wl.context_lens)))
+    return cfg
+
+
+# ------------------------------------------------------------------ the oracle on the host cores
+
+def _oracle_sample_inputs(wl, seqs, values):
+    q, keys, vals, off = values
+    ks = [keys[off[s]:off[s + 1]].float().cpu().numpy() for s in seqs]
+    vs = [vals[off[s]:off[s + 1]].float().cpu().numpy() for s in seqs]
+    B, Hkv, D = wl.block_size, wl.num_kv_heads, wl.head_dim
+    nblk = [max(1, -(-len(k) // B)) for k in ks]
+    kp = np.zeros((sum(nblk), Hkv, B, D), np.float32)
+    vp = np.zeros_like(kp)
+    tables = np.full((len(seqs), max(nblk)), -1, np.int32)
+    base = 0
+    for i in range(len(seqs)):
+        L = len(ks[i])
+        pad = nblk[i] * B - L
+        kk = np.concatenate([ks[i], np.zeros((pad, Hkv, D), np.float32)])
+        vv = np.concatenate([vs[i], np.zeros((pad, Hkv, D), np.float32)])
+        kp[base:base + nblk[i]] = kk.reshape(nblk[i], B, Hkv, D).transpose(0, 2, 1, 3)
+        vp[base:base + nblk[i]] = vv.reshape(nblk[i], B, Hkv, D).transpose(0, 2, 1, 3)
+        tables[i, :nblk[i]] = np.arange(base, base + nblk[i])
+        base += nblk[i]
+    lens = np.array([len(k) for k in ks], np.int32)
+    return q[list(seqs)].float().cpu().numpy(), kp, vp, tables, lens
+
+
+def _seq_bytes(wl, seqs):
+    elt = 4 if wl.dtype == "f32" else 2
+    tok = int(sum(int(wl.context_lens[s]) for s in seqs))
+    nblk = int(sum(-(-int(wl.context_lens[s]) // wl.block_size) for s in seqs))
+    return tok * 2 * wl.num_kv_heads * wl.head_dim * elt + 2 * len(seqs) * wl.num_heads * wl.head_dim * elt + \
+        4 * (nblk + len(seqs)) + len(seqs) * (4 * wl.num_kv_heads * wl.head_dim * elt + 8)
+
+
+def oracle_leg(wl, budget_s, values, steps=1):
+    """Times the fp64 oracle on the host cores over a sample of sequences per step.
+    `values` are the generator's tensors (any device; the sample is copied to host).
+    Returns (GB/s of the sample's algorithmic bytes, seqs/s, cores, sample text, seconds)."""
+    from oracle import oracle
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    order = list(range(wl.num_seqs))
+    # calibrate on one sequence, then size the per-step sample to the budget
+    qs, kp, vp, tb, ln = _oracle_sample_inputs(wl, order[:1], values)
+    t0 = time.perf_counter()
+    oracle.decode(qs, kp, vp, tb, ln, wl.scale, nthreads=cores)
+    per_seq = max(1e-4, time.perf_counter() - t0)
+    n = int(max(1, min(wl.num_seqs, budget_s / per_seq)))
+    seqs = order[:n]
+    inputs = _oracle_sample_inputs(wl, seqs, values)
+    t_total = 0.0
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        oracle.decode(*inputs, wl.scale, nthreads=cores)
+        t_total += time.perf_counter() - t0
+    nbytes = _seq_bytes(wl, seqs) * steps
+    sample = "first %d of %d sequences of %s (%d context tokens) per step, fp64, %d threads" % (
+        n, wl.num_seqs, wl.name, int(sum(int(wl.context_lens[s]) for s in seqs)), cores)
+    return nbytes / t_total / 1e9, n * steps / t_total, cores, sample, t_total
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = W.make_workload(W.NAME_TO_ID[args.workload], seed=args.seed)
+    if isinstance(wl, W.CowWorkload):
+        print(json.dumps({"impl": "reference", "unavailable": "oracle leg covers the decode workloads only"}))
+        return 0
+    total = args.steps + args.warmup
+    per_step = min(2.0, 120.0 / max(1, total))
+    try:
+        import torch
+        gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+    except Exception:
+        gen_dev = "cpu"
+    values = W.decode_values(wl, gen_dev)
+    # warm-up steps are untimed passes of the same sample
+    oracle_leg(wl, per_step, values, steps=max(1, min(args.warmup, 3)))
+    gbs, seqs_s, cores, sample, t = oracle_leg(wl, per_step, values, steps=args.steps)
+    line = {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * t / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(wl, wl.partition_size), "seqs_per_s": round(seqs_s, 3),
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------------ the CUDA path
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d" % (args.gpus, world))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    from paged_kv_cache_363_b200 import runner
+
+    wl = W.make_workload(W.NAME_TO_ID[args.workload], seed=rank_seed(args.seed, rank))
+    if args.partition is not None:
+        wl.partition_size = args.partition
+    if isinstance(wl, W.CowWorkload):
+        values = W.cow_values(wl, dev)
+    else:
+        values = W.decode_values(wl, dev)
+    batch = runner.make_batch(wl, dev, values=values)
+    from paged_kv_cache_363_b200 import pa
+    part = pa.pa_decode_partition_size(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size,
+                                       batch.max_context_len, batch.partition_size)
+    n_part = -(-batch.max_context_len // part)
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize(dev)
+    if pa.pa_device_status() != 0:
+        raise SystemExit("device status flagged during set-up")
+
+    dec_bytes = batch.decode_bytes()
+    step_bytes = dec_bytes + batch.append_bytes()
+    cow_launch = 1 if getattr(batch, "cow_pairs", None) is not None and batch.cow_pairs.numel() else 0
+    launches_per_step = 1 + cow_launch + 1 + (1 if n_part > 1 else 0)
+
+    # ---- device-resident timing
+    for _ in range(args.warmup):
+        batch.step(stream)
+    torch.cuda.synchronize(dev)
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for k in range(args.steps):
+            batch.append(stream)
+            ev_s[k].record(stream)
+            batch.decode(stream=stream)
+            ev_e[k].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms = t_start.elapsed_time(t_end)
+    dec_ms = [a.elapsed_time(b) for a, b in zip(ev_s, ev_e)]
+    ms_max = reduce_max(ms, dev)
+    dec_avg = statistics.mean(dec_ms)
+    dec_avg_max = reduce_max(dec_avg, dev)
+    out_ok = bool(torch.isfinite(batch.out.float()).all().item())
+    flags = pa.pa_device_status()
+
+    # ---- end to end through the API, inputs and result in pinned host memory
+    host = {}
+    for name in ("q", "new_k", "new_v", "slot_mapping", "block_tables", "context_lens"):
+        t = getattr(batch, name)
+        host[name] = t.cpu().pin_memory()
+    out_host = torch.empty(batch.out.shape, dtype=batch.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for name, t in host.items():
+            getattr(batch, name).copy_(t, non_blocking=True)
+        batch.step(stream)
+        out_host.copy_(batch.out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e_s = torch.cuda.Event(enable_timing=True)
+    e_e = torch.cuda.Event(enable_timing=True)
+    e_s.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e_e.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = reduce_max(e_s.elapsed_time(e_e), dev)
+    if world > 1:
+        dist.barrier()
+
+    peak, peak_kind = measured_hbm_peak()
+    achieved = dec_bytes / (dec_avg_max * 1e-3) / 1e9
+    value = world * step_bytes * args.steps / (ms_max * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+        "config": dict(workload_config(wl, part), l2="inputs larger than L2: %.0f MB of KV per step vs 126 MB"
+                       % (dec_bytes / 1e6), parallelism="replicas: one batch per GPU (dp%d)" % world),
+        "seqs_per_s": round(world * wl.num_seqs * args.steps / (ms_max * 1e-3), 1),
+        "pct_of_peak": round(100.0 * value / peak, 2),
+        "roofline": {"bound": "hbm", "kernel": "pa_decode (partition kernel + log-sum-exp merge)",
+                     "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4),
+                     "traffic": profile_traffic("decode_partition_kernel", wl.name),
+                     "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_us": round(dec_avg_max * 1e3, 3)},
+        "e2e": {"value": round(world * step_bytes * args.steps / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms / args.steps, 5)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "device_status": flags, "output_finite": out_ok,
+    }
+    if world == 1 and not args.no_cpu_baseline and not isinstance(wl, W.CowWorkload):
+        gbs, seqs_s, cores, sample, _ = oracle_leg(wl, args.cpu_budget, values)
+        line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default="decode-mha-bf16", choices=sorted(W.NAME_TO_ID))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--partition", type=int, default=None, help="context partition tokens (0 = automatic)")
+    ap.add_argument("--cpu-budget", type=float, default=8.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,245 @@
+/*
+ * pa.h - C ABI of libpa.so, a B200 (sm_100a) implementation of the PagedAttention
+ * decode path: paged decode attention, the slot-mapped KV append, the
+ * copy-on-write block copy, and the host block allocator that feeds them.
+ *
+ * Sources, by page title and section:
+ *  [FSAH] "PagedAttention Paper Breakdown: Virtual Memory Allocation for LLM KV
+ *         Cache Serving" (fullstackaihub.com).  Section 2 "Virtual Memory Paging &
+ *         Block Table Architecture", Address Translation Formula: for logical token
+ *         i, b = floor(i/B), o = i mod B, PhysicalAddr(K_i) = T[b]*B + o (a token
+ *         slot).  Section 3 "Dynamic Copy-on-Write (CoW) Parallel Sampling".
+ *  [INIT] "PagedAttention and vLLM Architecture: Virtual Memory for LLM Serving"
+ *         (initnode.dev).  Section 1 "Logical vs Physical Blocks" (fixed pool of
+ *         B-token pages allocated at startup, per-request block table kept by the
+ *         engine); "Why Internal Fragmentation is Bounded" (a block is taken only
+ *         when a token overflows the last one); section 2 "PagedAttention Attention
+ *         CUDA Kernel Mechanics" (the kernel takes q and the block table, walks the
+ *         physical blocks in table order, dots q with each key, and fuses an online
+ *         softmax across blocks with the product by the V blocks); section 3
+ *         "Copy-on-Write (CoW) for Parallel Sampling & Beam Search" (shared blocks
+ *         carry a reference count; writing into a shared block copies it to a new
+ *         block from the free pool, drops the old count and repoints one table).
+ *
+ * Conventions for every call:
+ *  - Tensors are dense and row-major.  Device calls take DEVICE pointers to
+ *    caller-owned memory; the library never allocates device memory and keeps no
+ *    pointer after a call returns.  pa_alloc_* calls take HOST pointers.
+ *  - KV pools: k_cache and v_cache are [num_blocks][num_kv_heads][block_size][head_dim]
+ *    of the call's dtype.  Token slot t lives in physical block t / block_size at
+ *    offset t % block_size.
+ *  - Supported: head_dim in {64, 128}; block_size in {16, 32}; num_heads a multiple
+ *    of num_kv_heads with a group of 1, 2, 4 or 8 query heads per kv head;
+ *    dtype fp32 or bf16 (q, out and both pools share it).  Other values return
+ *    PA_ERR_UNSUPPORTED.  Device pointers must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Device calls are
+ *    asynchronous: they validate their host-side arguments, launch, and return.
+ *    Launch failures return PA_ERR_CUDA.  Checks that need device data (block
+ *    indices, context lengths, slots, copy pairs) are made by the kernels, which
+ *    skip the offending access and raise a flag read by pa_device_status().
+ *  - Errors never abort or throw; pa_last_error_string() describes the last one
+ *    on the calling thread.
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+/* Symbols exported from the shared library; everything else stays hidden. */
+#if defined(PA_BUILDING_LIBRARY) && defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID = -1,       /* bad argument (null pointer, bad size, misalignment, unknown id) */
+    PA_ERR_UNSUPPORTED = -2,   /* shape or dtype outside the supported set above */
+    PA_ERR_OOM = -3,           /* allocator: free pool exhausted (allocator state unchanged) */
+    PA_ERR_CUDA = -4,          /* a CUDA runtime call failed */
+    PA_ERR_DEVICE_CHECK = -5   /* a kernel flagged bad device data (see pa_device_status) */
+} pa_status;
+
+typedef enum { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
+
+/* Bits of the device status word (pa_device_status). */
+#define PA_DEV_BAD_BLOCK     1u   /* a block-table entry outside [0, num_blocks) was read */
+#define PA_DEV_BAD_CONTEXT   2u   /* a context length < 0, > max_context_len or > max_blocks_per_seq*B */
+#define PA_DEV_BAD_SLOT      4u   /* a slot_mapping entry >= num_blocks*block_size */
+#define PA_DEV_BAD_PAIR      8u   /* a block_mapping entry outside [0, num_blocks) */
+#define PA_DEV_WAIT_TIMEOUT 16u   /* a pipeline wait inside a kernel gave up (bounded wait) */
+
+/* ------------------------------------------------------------------ decode */
+
+/*
+ * Context-partition length (tokens) that pa_decode uses for these arguments:
+ * `partition_size` itself when > 0 (it must be a multiple of block_size, at most
+ * 4096), else an automatic choice.  A sequence longer than one partition is
+ * split into partitions whose softmax states are merged by log-sum-exp in a
+ * second kernel.  Returns a negative pa_status on invalid arguments.
+ */
+PA_API int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                             int max_context_len, int partition_size);
+
+/*
+ * Bytes of device workspace pa_decode needs for these arguments (0 when no
+ * sequence can span more than one partition).  The workspace holds, per
+ * (sequence, query head, partition), the running max, the softmax sum and the
+ * unnormalised head_dim-vector of the partition.
+ */
+PA_API size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                int max_context_len, int partition_size);
+
+/*
+ * Paged decode attention ([INIT] section 2; translation per [FSAH] section 2).
+ *   out[s][h][:] = sum_i softmax_i(scale * q[s][h] . K_i) V_i
+ * over the logical tokens i < context_lens[s] of sequence s, where K_i and V_i are
+ * read from physical block block_tables[s][i / block_size], offset
+ * i % block_size, kv head h / (num_heads / num_kv_heads).  Accumulation is fp32;
+ * out is written in `dtype`.  context_lens[s] == 0 gives a zero row.
+ *   out           [num_seqs][num_heads][head_dim]            (device, written)
+ *   q             [num_seqs][num_heads][head_dim]            (device)
+ *   k_cache/v_cache pools as above                           (device)
+ *   block_tables  [num_seqs][max_blocks_per_seq] int32       (device); entries past
+ *                 ceil(context_lens[s]/block_size) are never read
+ *   context_lens  [num_seqs] int32                           (device), each in
+ *                 [0, min(max_context_len, max_blocks_per_seq*block_size)]
+ *   max_context_len  host-side upper bound of context_lens (sizes the launch)
+ *   partition_size   0 = automatic, else tokens per context partition
+ *   workspace     device scratch of at least pa_decode_workspace_size() bytes,
+ *                 16-byte aligned (may be NULL when that size is 0); its contents
+ *                 are overwritten.  Calls that share a workspace must be ordered
+ *                 on one stream.
+ */
+PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_heads,
+                    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+                    int max_context_len, float scale, int partition_size, void* workspace,
+                    size_t workspace_bytes, pa_dtype dtype, void* stream);
+
+/* ------------------------------------------------------------------ KV append */
+
+/*
+ * Slot-mapped KV append: for each token t < num_tokens with slot = slot_mapping[t]
+ * >= 0, k_cache[slot / block_size][h][slot % block_size][:] = key[t][h][:] and the
+ * same for value/v_cache, for every kv head h.  slot = T[b]*B + o is the [FSAH]
+ * section 2 address of the token's position.  Negative slots are padding and
+ * are skipped.  The copy is bit-exact.  Slots must be distinct (otherwise the
+ * surviving row is unspecified).
+ *   key, value    [num_tokens][num_kv_heads][head_dim]  (device)
+ *   slot_mapping  [num_tokens] int64                    (device)
+ */
+PA_API pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                               const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                               int block_size, int num_blocks, pa_dtype dtype, void* stream);
+
+/* ------------------------------------------------------------------ CoW copy */
+
+/*
+ * Copy-on-write block copy ([INIT] section 3): for each pair i,
+ * block block_mapping[2i+1] of both pools becomes a bit-exact copy of block
+ * block_mapping[2i] (all kv heads, all block_size slots).  No destination may
+ * also be a source or appear twice in one call (pairs run concurrently); the
+ * allocator's copy-on-write pairs always satisfy this.
+ *   block_mapping [num_pairs][2] int64 (src, dst)   (device)
+ */
+PA_API pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping, int num_pairs,
+                         int num_kv_heads, int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                         void* stream);
+
+/* ------------------------------------------------------------------ device status */
+
+/*
+ * Waits for `stream`, then returns in *flags the PA_DEV_* bits raised by kernels
+ * on the current device since the last call, and clears them.  Returns PA_OK,
+ * or PA_ERR_CUDA if the wait or the read failed.
+ */
+PA_API pa_status pa_device_status(uint32_t* flags, void* stream);
+
+/* ------------------------------------------------------------------ block allocator */
+
+/*
+ * Host block allocator with reference-counted copy-on-write ([INIT] sections 1
+ * and 3, "Why Internal Fragmentation is Bounded"; [FSAH] sections 2 and 3).
+ * It owns only host memory.  The free pool is a FIFO queue initialised from
+ * free_order (a permutation of 0..num_blocks-1; NULL = ascending); blocks freed
+ * later join its tail.  A handle is not thread-safe.  On every error the
+ * allocator state is left unchanged.
+ */
+typedef struct pa_allocator pa_allocator;
+
+typedef struct {
+    int64_t num_blocks;
+    int64_t num_free;
+    int64_t num_seqs;
+    int64_t shared_blocks;     /* blocks with reference count > 1 */
+    int64_t cow_copies;        /* copy-on-write copies made so far */
+    int64_t tokens;            /* sum of the sequences' token counts */
+    int64_t waste_tokens;      /* unused slots in the sequences' last blocks */
+} pa_alloc_stats_t;
+
+/* Returns NULL on bad arguments (see pa_last_error_string). */
+PA_API pa_allocator* pa_alloc_create(int num_blocks, int block_size, const int32_t* free_order);
+PA_API void pa_alloc_destroy(pa_allocator* a);
+
+/* New sequence of num_tokens tokens (a prompt): takes ceil(num_tokens/B) blocks,
+ * each with reference count 1.  slots_out (nullable, num_tokens entries) receives
+ * the slot of every token.  PA_ERR_INVALID if seq_id exists. */
+PA_API pa_status pa_alloc_add_seq(pa_allocator* a, int64_t seq_id, int num_tokens, int64_t* slots_out);
+
+/* child shares every block of parent (each reference count + 1) and its token count. */
+PA_API pa_status pa_alloc_fork(pa_allocator* a, int64_t parent_id, int64_t child_id);
+
+/*
+ * Slot for one new token of seq_id.  A fresh block is taken when the last block is
+ * full or absent.  If the last block is partially filled and shared (reference
+ * count > 1), it is copied on write: a new block dst is taken, the old count is
+ * decremented, the table entry is repointed, and (src, dst) is returned through
+ * cow_src_out / cow_dst_out (each -1 when no copy is needed; both nullable).
+ * The caller must run pa_copy_blocks for the pair before writing the slot.
+ */
+PA_API pa_status pa_alloc_append_slot(pa_allocator* a, int64_t seq_id, int64_t* slot_out, int32_t* cow_src_out,
+                               int32_t* cow_dst_out);
+
+/*
+ * One append per listed sequence, in list order (a decode step).  slots_out[n],
+ * cow_pairs_out[2 * n] (src, dst pairs, packed) and *num_cow_out receive the
+ * results.  All or nothing: on error no append of the batch remains applied.
+ */
+PA_API pa_status pa_alloc_append_slots(pa_allocator* a, const int64_t* seq_ids, int n, int64_t* slots_out,
+                                int64_t* cow_pairs_out, int* num_cow_out);
+
+/* Drops one reference to each block of seq_id; blocks reaching zero rejoin the free pool. */
+PA_API pa_status pa_alloc_free_seq(pa_allocator* a, int64_t seq_id);
+
+/* Copies seq_id's block table into out[capacity]; *n_out = its length.
+ * PA_ERR_INVALID if capacity is too small (nothing is written then). */
+PA_API pa_status pa_alloc_block_table(const pa_allocator* a, int64_t seq_id, int32_t* out, int capacity, int* n_out);
+
+/* Dense [n][max_blocks] table of the listed sequences, rows padded with `fill`;
+ * *context_lens_out (nullable, n entries) receives their token counts. */
+PA_API pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq_ids, int n, int32_t* out,
+                                int max_blocks, int32_t fill, int32_t* context_lens_out);
+
+PA_API int pa_alloc_ref_count(const pa_allocator* a, int32_t block);   /* -1 if out of range */
+PA_API int pa_alloc_num_free(const pa_allocator* a);
+PA_API int pa_alloc_num_tokens(const pa_allocator* a, int64_t seq_id); /* -1 if unknown */
+PA_API pa_status pa_alloc_stats(const pa_allocator* a, pa_alloc_stats_t* out);
+
+/* ------------------------------------------------------------------ diagnostics */
+
+/* Message of the last failed call on this thread ("" if none).  Valid until the
+ * next failing call on the same thread. */
+PA_API const char* pa_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

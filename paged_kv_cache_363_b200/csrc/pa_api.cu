@@ -1,0 +1,297 @@
+// C ABI of libpa.so (declared in include/pa.h): argument validation, dispatch to
+// the kernels, the device status word, and the per-thread error message.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "pa.h"
+#include "pa_internal.h"
+
+namespace pa {
+
+static thread_local std::string g_err;
+
+void set_error(const std::string& msg) { g_err = msg; }
+
+namespace {
+
+// Device status word: kernels OR PA_DEV_* bits into it.  Host code reaches it
+// through its per-device address (the symbol itself is only a host-side handle).
+__device__ unsigned int g_status_word;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+unsigned int* g_status_ptr[kMaxDevices] = {};
+
+pa_status cuda_fail(const char* what, cudaError_t e)
+{
+    set_error(std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")");
+    return PA_ERR_CUDA;
+}
+
+// Address of the status word on the current device (resolved once per device).
+pa_status status_ptr(unsigned int** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    if (dev < 0 || dev >= kMaxDevices) {
+        set_error("device index out of range");
+        return PA_ERR_INVALID;
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_status_word);
+        if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress(status word)", e);
+        g_status_ptr[dev] = static_cast<unsigned int*>(p);
+    }
+    *out = g_status_ptr[dev];
+    return PA_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int elt_bytes(pa_dtype dt) { return dt == PA_DTYPE_F32 ? 4 : 2; }
+
+pa_status check_common(const char* fn, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                       pa_dtype dtype)
+{
+    if (dtype != PA_DTYPE_F32 && dtype != PA_DTYPE_BF16) {
+        set_error(std::string(fn) + ": dtype must be PA_DTYPE_F32 or PA_DTYPE_BF16");
+        return PA_ERR_UNSUPPORTED;
+    }
+    if (head_dim != 64 && head_dim != 128) {
+        set_error(std::string(fn) + ": head_dim must be 64 or 128");
+        return PA_ERR_UNSUPPORTED;
+    }
+    if (block_size != 16 && block_size != 32) {
+        set_error(std::string(fn) + ": block_size must be 16 or 32");
+        return PA_ERR_UNSUPPORTED;
+    }
+    if (num_kv_heads <= 0 || num_kv_heads > 65535 || num_blocks <= 0) {
+        set_error(std::string(fn) + ": num_kv_heads and num_blocks must be > 0 (num_kv_heads <= 65535)");
+        return PA_ERR_INVALID;
+    }
+    return PA_OK;
+}
+
+constexpr int kAutoPartitionTokens = 512;
+
+// Partition tokens for the arguments, or a negative pa_status.
+int resolve_partition(int block_size, int max_context_len, int partition_size)
+{
+    int p = partition_size > 0 ? partition_size : kAutoPartitionTokens;
+    if (p % block_size != 0 || p > kMaxPartitionTokens) {
+        set_error("partition_size must be a multiple of block_size and at most " +
+                  std::to_string(kMaxPartitionTokens));
+        return PA_ERR_INVALID;
+    }
+    const long np = ((long)max_context_len + p - 1) / p;
+    if (np > kMaxPartitions) {
+        set_error("max_context_len / partition_size exceeds " + std::to_string(kMaxPartitions) +
+                  " partitions; use a larger partition_size");
+        return PA_ERR_UNSUPPORTED;
+    }
+    return p;
+}
+
+}  // namespace
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+const char* pa_last_error_string(void) { return g_err.c_str(); }
+
+int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                             int max_context_len, int partition_size)
+{
+    (void)num_seqs;
+    (void)num_heads;
+    (void)num_kv_heads;
+    (void)head_dim;
+    if (block_size != 16 && block_size != 32) {
+        set_error("pa_decode_partition_size: block_size must be 16 or 32");
+        return PA_ERR_UNSUPPORTED;
+    }
+    if (max_context_len < 0 || partition_size < 0) {
+        set_error("pa_decode_partition_size: negative size");
+        return PA_ERR_INVALID;
+    }
+    return resolve_partition(block_size, max_context_len, partition_size);
+}
+
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                int max_context_len, int partition_size)
+{
+    const int p = pa_decode_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                           max_context_len, partition_size);
+    if (p <= 0 || num_seqs <= 0 || num_heads <= 0 || head_dim <= 0) return 0;
+    const size_t np = ((size_t)max_context_len + p - 1) / p;
+    if (np <= 1) return 0;
+    const size_t rows = (size_t)num_seqs * num_heads * np;
+    return rows * (size_t)(head_dim + 2) * sizeof(float);
+}
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_heads,
+                    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+                    int max_context_len, float scale, int partition_size, void* workspace,
+                    size_t workspace_bytes, pa_dtype dtype, void* stream)
+{
+    pa_status st = check_common("pa_decode", num_kv_heads, head_dim, block_size, num_blocks, dtype);
+    if (st != PA_OK) return st;
+    if (num_seqs < 0 || num_seqs > 65535 || num_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 ||
+        partition_size < 0 || !std::isfinite(scale)) {
+        set_error("pa_decode: bad size or scale");
+        return PA_ERR_INVALID;
+    }
+    if (num_heads % num_kv_heads != 0) {
+        set_error("pa_decode: num_heads must be a multiple of num_kv_heads");
+        return PA_ERR_INVALID;
+    }
+    const int group = num_heads / num_kv_heads;
+    if (group != 1 && group != 2 && group != 4 && group != 8) {
+        set_error("pa_decode: num_heads / num_kv_heads must be 1, 2, 4 or 8");
+        return PA_ERR_UNSUPPORTED;
+    }
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) {
+        set_error("pa_decode: null pointer");
+        return PA_ERR_INVALID;
+    }
+    if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_tables, 4) || !aligned(context_lens, 4)) {
+        set_error("pa_decode: misaligned pointer (q, out, caches need 16 bytes)");
+        return PA_ERR_INVALID;
+    }
+    const int p = resolve_partition(block_size, max_context_len, partition_size);
+    if (p < 0) return (pa_status)p;
+    const int np = max_context_len > 0 ? (max_context_len + p - 1) / p : 1;
+    DecodeArgs a{};
+    if (np > 1) {
+        const size_t need = pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
+                                                     max_context_len, partition_size);
+        if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) {
+            set_error("pa_decode: workspace missing, too small (need " + std::to_string(need) +
+                      " bytes) or not 16-byte aligned");
+            return PA_ERR_INVALID;
+        }
+        a.ws_acc = static_cast<float*>(workspace);
+        a.ws_ml = a.ws_acc + (size_t)num_seqs * num_heads * np * head_dim;
+    }
+    unsigned int* status = nullptr;
+    st = status_ptr(&status);
+    if (st != PA_OK) return st;
+    a.out = out;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.status = status;
+    a.num_seqs = num_seqs;
+    a.num_heads = num_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.num_blocks = num_blocks;
+    a.max_context_len = max_context_len;
+    a.partition_blocks = p / block_size;
+    a.num_partitions = np;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    const cudaError_t e =
+        launch_decode(a, dtype, head_dim, block_size, group, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail("pa_decode launch", e);
+    return PA_OK;
+}
+
+pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                               const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                               int block_size, int num_blocks, pa_dtype dtype, void* stream)
+{
+    pa_status st = check_common("pa_reshape_and_cache", num_kv_heads, head_dim, block_size, num_blocks, dtype);
+    if (st != PA_OK) return st;
+    if (num_tokens < 0) {
+        set_error("pa_reshape_and_cache: num_tokens < 0");
+        return PA_ERR_INVALID;
+    }
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping) {
+        set_error("pa_reshape_and_cache: null pointer");
+        return PA_ERR_INVALID;
+    }
+    if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(slot_mapping, 8)) {
+        set_error("pa_reshape_and_cache: misaligned pointer");
+        return PA_ERR_INVALID;
+    }
+    unsigned int* status = nullptr;
+    st = status_ptr(&status);
+    if (st != PA_OK) return st;
+    ReshapeArgs a{key, value, k_cache, v_cache, slot_mapping, status, num_tokens, num_kv_heads, num_blocks};
+    const cudaError_t e =
+        launch_reshape_and_cache(a, elt_bytes(dtype), head_dim, block_size, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail("pa_reshape_and_cache launch", e);
+    return PA_OK;
+}
+
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping, int num_pairs,
+                         int num_kv_heads, int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                         void* stream)
+{
+    pa_status st = check_common("pa_copy_blocks", num_kv_heads, head_dim, block_size, num_blocks, dtype);
+    if (st != PA_OK) return st;
+    if (num_pairs < 0 || num_pairs > 65535) {
+        set_error("pa_copy_blocks: num_pairs must be in [0, 65535]");
+        return PA_ERR_INVALID;
+    }
+    if (num_pairs == 0) return PA_OK;
+    if (!k_cache || !v_cache || !block_mapping) {
+        set_error("pa_copy_blocks: null pointer");
+        return PA_ERR_INVALID;
+    }
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(block_mapping, 8)) {
+        set_error("pa_copy_blocks: misaligned pointer");
+        return PA_ERR_INVALID;
+    }
+    unsigned int* status = nullptr;
+    st = status_ptr(&status);
+    if (st != PA_OK) return st;
+    CopyArgs a{};
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_mapping = block_mapping;
+    a.status = status;
+    a.num_pairs = num_pairs;
+    a.num_blocks = num_blocks;
+    a.block_bytes = (size_t)num_kv_heads * block_size * head_dim * elt_bytes(dtype);
+    const cudaError_t e = launch_copy_blocks(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail("pa_copy_blocks launch", e);
+    return PA_OK;
+}
+
+pa_status pa_device_status(uint32_t* flags, void* stream)
+{
+    if (!flags) return PA_ERR_INVALID;
+    unsigned int* status = nullptr;
+    pa_status st = status_ptr(&status);
+    if (st != PA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, status, sizeof(v), cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_fail("pa_device_status read", e);
+    e = cudaMemsetAsync(status, 0, sizeof(unsigned int), s);
+    if (e != cudaSuccess) return cuda_fail("pa_device_status clear", e);
+    e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail("pa_device_status sync", e);
+    *flags = v;
+    return PA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,224 @@
+"""The C-ABI library loads, exports every symbol include/pa.h declares, validates
+its host-side arguments, and its allocator matches the oracle allocator (CPU only:
+no call here reaches a GPU)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from conftest import ROOT
+from oracle.allocator import OracleAllocator, OutOfBlocks as OracleOOM
+
+pa = pytest.importorskip("paged_kv_cache_363_b200.pa", reason="libpa.so not built")
+
+
+def _declared_symbols():
+    with open(os.path.join(ROOT, "include", "pa.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^PA_API [^(]*?\b(pa_\w+)\(", text, flags=re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _declared_symbols()
+    assert len(declared) >= 19
+    for name in declared:
+        assert hasattr(pa.lib, name), name
+    bound = sorted(n for n, _, _ in pa.SIGNATURES)
+    assert bound == declared
+
+
+def test_exported_symbols_are_exactly_the_header():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", pa.LIB_PATH], capture_output=True, text=True).stdout
+    exported = sorted(l.split()[-1] for l in out.splitlines() if " T " in l)
+    assert exported == _declared_symbols()
+
+
+def test_host_validation_rejects_before_any_device_work():
+    L = pa.lib
+    p = ctypes.c_void_p(0x1000)
+    # unsupported head_dim / block size / dtype / group
+    assert L.pa_decode(p, p, p, p, p, p, 1, 4, 4, 96, 16, 4, 8, 64, 1.0, 0, None, 0, 1, None) == pa.PA_ERR_UNSUPPORTED
+    assert L.pa_decode(p, p, p, p, p, p, 1, 4, 4, 128, 8, 4, 8, 64, 1.0, 0, None, 0, 1, None) == pa.PA_ERR_UNSUPPORTED
+    assert L.pa_decode(p, p, p, p, p, p, 1, 4, 4, 128, 16, 4, 8, 64, 1.0, 0, None, 0, 7, None) == pa.PA_ERR_UNSUPPORTED
+    assert L.pa_decode(p, p, p, p, p, p, 1, 12, 4, 128, 16, 4, 8, 64, 1.0, 0, None, 0, 1, None) == pa.PA_ERR_UNSUPPORTED
+    assert L.pa_decode(p, p, p, p, p, p, 1, 6, 4, 128, 16, 4, 8, 64, 1.0, 0, None, 0, 1, None) == pa.PA_ERR_INVALID
+    # null / misaligned pointers, non-finite scale, bad partition, missing workspace
+    assert L.pa_decode(None, p, p, p, p, p, 1, 4, 4, 128, 16, 4, 8, 64, 1.0, 0, None, 0, 1, None) == pa.PA_ERR_INVALID
+    q = ctypes.c_void_p(0x1008)
+    assert L.pa_decode(p, q, p, p, p, p, 1, 4, 4, 128, 16, 4, 8, 64, 1.0, 0, None, 0, 1, None) == pa.PA_ERR_INVALID
+    assert L.pa_decode(p, p, p, p, p, p, 1, 4, 4, 128, 16, 4, 8, 64, float("inf"), 0, None, 0, 1, None) == pa.PA_ERR_INVALID
+    assert L.pa_decode(p, p, p, p, p, p, 1, 4, 4, 128, 16, 4, 8, 64, 1.0, 24, None, 0, 1, None) == pa.PA_ERR_INVALID
+    assert L.pa_decode(p, p, p, p, p, p, 1, 4, 4, 128, 16, 64, 8, 1024, 1.0, 0, None, 0, 1, None) == pa.PA_ERR_INVALID
+    assert "workspace" in L.pa_last_error_string().decode()
+    # zero sequences is a no-op
+    assert L.pa_decode(None, None, None, None, None, None, 0, 4, 4, 128, 16, 4, 8, 0, 1.0, 0, None, 0, 1, None) == pa.PA_OK
+    # companions
+    assert L.pa_reshape_and_cache(p, p, p, p, p, 4, 4, 100, 16, 8, 1, None) == pa.PA_ERR_UNSUPPORTED
+    assert L.pa_reshape_and_cache(p, p, p, p, None, 4, 4, 128, 16, 8, 1, None) == pa.PA_ERR_INVALID
+    assert L.pa_reshape_and_cache(None, None, None, None, None, 0, 4, 128, 16, 8, 1, None) == pa.PA_OK
+    assert L.pa_copy_blocks(p, p, None, 3, 4, 128, 16, 8, 1, None) == pa.PA_ERR_INVALID
+    assert L.pa_copy_blocks(p, p, p, 70000, 4, 128, 16, 8, 1, None) == pa.PA_ERR_INVALID
+    assert L.pa_copy_blocks(None, None, None, 0, 4, 128, 16, 8, 1, None) == pa.PA_OK
+
+
+def test_partition_and_workspace_sizes():
+    assert pa.pa_decode_partition_size(8, 32, 8, 128, 32, 32768, 512) == 512
+    assert pa.pa_decode_partition_size(8, 32, 8, 128, 32, 32768, 0) % 32 == 0
+    with pytest.raises(pa.PAError):
+        pa.pa_decode_partition_size(8, 32, 8, 128, 32, 32768, 48)
+    with pytest.raises(pa.PAError):
+        pa.pa_decode_partition_size(8, 32, 8, 128, 16, 10 ** 7, 16)      # too many partitions
+    # one partition: no workspace
+    assert pa.pa_decode_workspace_size(4, 4, 4, 64, 16, 100, 512) == 0
+    # S * Hq * NP * (D + 2) floats
+    assert pa.pa_decode_workspace_size(8, 32, 8, 128, 32, 32768, 512) == 8 * 32 * 64 * 130 * 4
+
+
+def _replay(ops, NB, B, order):
+    """Run the same script on the library allocator and the oracle allocator."""
+    lib_a = pa.Allocator(NB, B, order)
+    ora = OracleAllocator(NB, B, order)
+    for op in ops:
+        kind = op[0]
+        if kind == "add":
+            try:
+                want = ora.add_seq(op[1], op[2])
+            except OracleOOM:
+                with pytest.raises(pa.OutOfBlocks):
+                    lib_a.add_seq(op[1], op[2])
+                continue
+            assert lib_a.add_seq(op[1], op[2]).tolist() == want
+        elif kind == "fork":
+            ora.fork(op[1], op[2])
+            lib_a.fork(op[1], op[2])
+        elif kind == "append":
+            try:
+                want = ora.append_slot(op[1])
+            except OracleOOM:
+                with pytest.raises(pa.OutOfBlocks):
+                    lib_a.append_slot(op[1])
+                continue
+            assert lib_a.append_slot(op[1]) == want
+        elif kind == "batch":
+            snap = (list(ora.free), list(ora.ref), {k: list(v) for k, v in ora.tables.items()},
+                    dict(ora.ntokens), ora.cow_count)
+            try:
+                res = [ora.append_slot(s) for s in op[1]]
+            except OracleOOM:
+                # all-or-nothing: restore the oracle and expect the library to refuse the batch
+                ora.free.clear()
+                ora.free.extend(snap[0])
+                ora.ref[:] = snap[1]
+                ora.tables = snap[2]
+                ora.ntokens = snap[3]
+                ora.cow_count = snap[4]
+                with pytest.raises(pa.OutOfBlocks):
+                    lib_a.append_slots(op[1])
+                continue
+            slots, pairs = lib_a.append_slots(op[1])
+            assert slots.tolist() == [r[0] for r in res]
+            assert [tuple(p) for p in pairs.tolist()] == [r[1] for r in res if r[1] is not None]
+        elif kind == "free":
+            ora.free_seq(op[1])
+            lib_a.free_seq(op[1])
+        # full state comparison after every op
+        assert lib_a.num_free() == ora.num_free()
+        for b in range(NB):
+            assert lib_a.ref_count(b) == ora.ref[b]
+        for sid in ora.tables:
+            assert lib_a.block_table(sid) == ora.block_table(sid)
+            assert lib_a.num_tokens(sid) == ora.ntokens[sid]
+    st = lib_a.stats()
+    assert st["cow_copies"] == ora.cow_count
+    assert st["waste_tokens"] == sum(ora.waste_tokens(s) for s in ora.tables)
+    return lib_a, ora
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_allocator_matches_oracle_on_random_scripts(seed):
+    rng = np.random.default_rng(seed)
+    NB, B = int(rng.integers(20, 80)), int(rng.choice([4, 16]))
+    order = rng.permutation(NB)
+    ops, live, nxt = [], [], 0
+    for _ in range(300):
+        r = rng.random()
+        if r < 0.15 or not live:
+            ops.append(("add", nxt, int(rng.integers(0, 3 * B))))
+            live.append(nxt)
+            nxt += 1
+        elif r < 0.3:
+            ops.append(("fork", int(rng.choice(live)), nxt))
+            live.append(nxt)
+            nxt += 1
+        elif r < 0.7:
+            ops.append(("append", int(rng.choice(live))))
+        elif r < 0.85:
+            k = int(rng.integers(1, len(live) + 1))
+            ops.append(("batch", [int(x) for x in rng.choice(live, size=k, replace=False)]))
+        else:
+            sid = int(rng.choice(live))
+            ops.append(("free", sid))
+            live.remove(sid)
+    # failing adds never create the sequence: drop later ops on it by replaying defensively
+    lib_a, ora = None, None
+    clean, known = [], set()
+    sim = OracleAllocator(NB, B, order)
+    for op in ops:
+        if op[0] == "add":
+            try:
+                sim.add_seq(op[1], op[2])
+                known.add(op[1])
+            except OracleOOM:
+                pass
+            clean.append(op)
+        elif op[0] == "fork":
+            if op[1] in known:
+                sim.fork(op[1], op[2])
+                known.add(op[2])
+                clean.append(op)
+        elif op[0] == "append":
+            if op[1] in known:
+                try:
+                    sim.append_slot(op[1])
+                except OracleOOM:
+                    pass
+                clean.append(op)
+        elif op[0] == "batch":
+            ids = [s for s in op[1] if s in known]
+            if ids:
+                snap = (list(sim.free), list(sim.ref), {k: list(v) for k, v in sim.tables.items()},
+                        dict(sim.ntokens), sim.cow_count)
+                try:
+                    for s in ids:
+                        sim.append_slot(s)
+                except OracleOOM:
+                    sim.free.clear()
+                    sim.free.extend(snap[0])
+                    sim.ref[:] = snap[1]
+                    sim.tables, sim.ntokens, sim.cow_count = snap[2], snap[3], snap[4]
+                clean.append(("batch", ids))
+        elif op[0] == "free":
+            if op[1] in known:
+                sim.free_seq(op[1])
+                known.discard(op[1])
+                clean.append(op)
+    _replay(clean, NB, B, order)
+
+
+def test_allocator_argument_errors():
+    with pytest.raises(pa.PAError):
+        pa.Allocator(8, 16, free_order=[0, 1, 2, 3, 4, 5, 6, 6])
+    a = pa.Allocator(8, 16)
+    a.add_seq(1, 5)
+    with pytest.raises(pa.PAError):
+        a.add_seq(1, 5)
+    with pytest.raises(pa.PAError):
+        a.fork(9, 10)
+    with pytest.raises(pa.PAError):
+        a.append_slot(9)
+    with pytest.raises(pa.PAError):
+        a.free_seq(9)
+    assert a.ref_count(-1) == -1 and a.ref_count(8) == -1 and a.num_tokens(9) == -1

@@ -280,7 +280,8 @@ def run_gpu(args):
 
     from paged_kv_cache_363_b200 import runner
 
-    wl = W.make_workload(W.NAME_TO_ID[args.workload], seed=rank_seed(args.seed, rank))
+    overrides = {} if args.pool_blocks is None else {"num_blocks": args.pool_blocks}
+    wl = W.make_workload(W.NAME_TO_ID[args.workload], seed=rank_seed(args.seed, rank), **overrides)
     if args.partition is not None:
         wl.partition_size = args.partition
     if isinstance(wl, W.CowWorkload):
@@ -332,36 +333,40 @@ def run_gpu(args):
     out_ok = bool(torch.isfinite(batch.out.float()).all().item())
     flags = pa.pa_device_status()
 
-    # ---- end to end through the API, inputs and result in pinned host memory
-    host = {}
-    for name in ("q", "new_k", "new_v", "slot_mapping", "block_tables", "context_lens"):
-        t = getattr(batch, name)
-        host[name] = t.cpu().pin_memory()
-    out_host = torch.empty(batch.out.shape, dtype=batch.out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_host.numel() * out_host.element_size()
+    e2e = None
+    if not args.skip_e2e:
+        # ---- end to end through the API, inputs and result in pinned host memory
+        host = {}
+        for name in ("q", "new_k", "new_v", "slot_mapping", "block_tables", "context_lens"):
+            t = getattr(batch, name)
+            host[name] = t.cpu().pin_memory()
+        out_host = torch.empty(batch.out.shape, dtype=batch.out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_host.numel() * out_host.element_size()
 
-    def e2e_step():
-        for name, t in host.items():
-            getattr(batch, name).copy_(t, non_blocking=True)
-        batch.step(stream)
-        out_host.copy_(batch.out, non_blocking=True)
+        def e2e_step():
+            for name, t in host.items():
+                getattr(batch, name).copy_(t, non_blocking=True)
+            batch.step(stream)
+            out_host.copy_(batch.out, non_blocking=True)
 
-    for _ in range(args.warmup):
-        e2e_step()
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    e_s = torch.cuda.Event(enable_timing=True)
-    e_e = torch.cuda.Event(enable_timing=True)
-    e_s.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e_e.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = reduce_max(e_s.elapsed_time(e_e), dev)
-    if world > 1:
-        dist.barrier()
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e_s = torch.cuda.Event(enable_timing=True)
+        e_e = torch.cuda.Event(enable_timing=True)
+        e_s.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e_e.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = reduce_max(e_s.elapsed_time(e_e), dev)
+        if world > 1:
+            dist.barrier()
+        e2e = {"value": round(world * step_bytes * args.steps / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 5)}
 
     peak, peak_kind = measured_hbm_peak()
     achieved = dec_bytes / (dec_avg_max * 1e-3) / 1e9
@@ -379,9 +384,7 @@ def run_gpu(args):
                      "frac": round(achieved / peak, 4),
                      "traffic": profile_traffic("decode_partition_kernel", wl.name),
                      "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_us": round(dec_avg_max * 1e3, 3)},
-        "e2e": {"value": round(world * step_bytes * args.steps / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(e2e_ms / args.steps, 5)},
+        "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
         "device_status": flags, "output_finite": out_ok,
@@ -408,6 +411,9 @@ def main(argv=None):
     ap.add_argument("--partition", type=int, default=None, help="context partition tokens (0 = automatic)")
     ap.add_argument("--cpu-budget", type=float, default=8.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
+    ap.add_argument("--pool-blocks", type=int, default=None,
+                    help="override the pool size (profiling runs on a smaller device footprint)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

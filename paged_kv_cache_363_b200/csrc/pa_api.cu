@@ -2,6 +2,7 @@
 // the kernels, the device status word, and the per-thread error message.
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -170,6 +171,11 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
         !aligned(block_tables, 4) || !aligned(context_lens, 4)) {
         set_error("pa_decode: misaligned pointer (q, out, caches need 16 bytes)");
         return PA_ERR_INVALID;
+    }
+    if (decode_uses_tensor_cores(dtype, head_dim, group) &&
+        (int64_t)num_blocks * num_kv_heads * block_size > (int64_t)INT32_MAX) {
+        set_error("pa_decode: num_blocks * num_kv_heads * block_size must stay below 2^31 (tensor-copy row index)");
+        return PA_ERR_UNSUPPORTED;
     }
     const int p = resolve_partition(block_size, max_context_len, partition_size);
     if (p < 0) return (pa_status)p;

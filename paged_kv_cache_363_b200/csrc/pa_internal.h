@@ -38,6 +38,11 @@ struct DecodeArgs {
 cudaError_t launch_decode(const DecodeArgs& a, pa_dtype dtype, int head_dim, int block_size, int group,
                           cudaStream_t stream);
 
+// bf16 with a group of 2, 4 or 8 query heads per kv head runs on the tensor cores
+// (pa_decode_mma.cu); everything else on the CUDA cores (pa_decode.cu).
+bool decode_uses_tensor_cores(pa_dtype dtype, int head_dim, int group);
+cudaError_t launch_decode_mma(const DecodeArgs& a, int head_dim, int block_size, int group, cudaStream_t stream);
+
 struct ReshapeArgs {
     const void* key;
     const void* value;

@@ -171,6 +171,23 @@ def workload_config(wl, partition, batch=None):
     return cfg
 
 
+def parse_overrides(items):
+    """KEY=VALUE workload overrides; VALUE is an int, a float, or a comma list."""
+    def conv(x):
+        for f in (int, float):
+            try:
+                return f(x)
+            except ValueError:
+                pass
+        return x
+    out = {}
+    for it in items:
+        k, v = it.split("=", 1)
+        parts = [conv(x) for x in v.split(",")]
+        out[k] = tuple(parts) if len(parts) > 1 else parts[0]
+    return out
+
+
 # ------------------------------------------------------------------ the oracle on the host cores
 
 def _oracle_sample_inputs(wl, seqs, values):
@@ -281,6 +298,7 @@ def run_gpu(args):
     from paged_kv_cache_363_b200 import runner
 
     overrides = {} if args.pool_blocks is None else {"num_blocks": args.pool_blocks}
+    overrides.update(parse_overrides(args.set))
     wl = W.make_workload(W.NAME_TO_ID[args.workload], seed=rank_seed(args.seed, rank), **overrides)
     if args.partition is not None:
         wl.partition_size = args.partition
@@ -301,7 +319,7 @@ def run_gpu(args):
     dec_bytes = batch.decode_bytes()
     step_bytes = dec_bytes + batch.append_bytes()
     cow_launch = 1 if getattr(batch, "cow_pairs", None) is not None and batch.cow_pairs.numel() else 0
-    launches_per_step = 1 + cow_launch + 1 + (1 if n_part > 1 else 0)
+    launches_per_step = 1 + cow_launch + 2   # append, [copy], plan + persistent decode
 
     # ---- device-resident timing
     for _ in range(args.warmup):
@@ -379,7 +397,7 @@ def run_gpu(args):
                        % (dec_bytes / 1e6), parallelism="replicas: one batch per GPU (dp%d)" % world),
         "seqs_per_s": round(world * wl.num_seqs * args.steps / (ms_max * 1e-3), 1),
         "pct_of_peak": round(100.0 * value / peak, 2),
-        "roofline": {"bound": "hbm", "kernel": "pa_decode (partition kernel + log-sum-exp merge)",
+        "roofline": {"bound": "hbm", "kernel": "pa_decode (plan kernel + persistent decode kernel)",
                      "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
                      "traffic": profile_traffic("decode_partition_kernel", wl.name),
@@ -414,6 +432,8 @@ def main(argv=None):
     ap.add_argument("--skip-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
     ap.add_argument("--pool-blocks", type=int, default=None,
                     help="override the pool size (profiling runs on a smaller device footprint)")
+    ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
+                    help="override a workload field, e.g. num_kv_heads=32 or lens=uniform,128,2048")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

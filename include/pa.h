@@ -88,10 +88,11 @@ PA_API int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_head
                              int max_context_len, int partition_size);
 
 /*
- * Bytes of device workspace pa_decode needs for these arguments (0 when no
- * sequence can span more than one partition).  The workspace holds, per
- * (sequence, query head, partition), the running max, the softmax sum and the
- * unnormalised head_dim-vector of the partition.
+ * Bytes of device workspace pa_decode needs for these arguments (> 0 whenever
+ * num_seqs > 0).  The workspace holds the call's work plan (the (sequence,
+ * partition) pairs, longest first, and a work counter) and, when a sequence can
+ * span more than one partition, per (sequence, query head, partition) the running
+ * max, the softmax sum and the unnormalised head_dim-vector of the partition.
  */
 PA_API size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
                                 int max_context_len, int partition_size);
@@ -113,9 +114,9 @@ PA_API size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_h
  *   max_context_len  host-side upper bound of context_lens (sizes the launch)
  *   partition_size   0 = automatic, else tokens per context partition
  *   workspace     device scratch of at least pa_decode_workspace_size() bytes,
- *                 16-byte aligned (may be NULL when that size is 0); its contents
- *                 are overwritten.  Calls that share a workspace must be ordered
- *                 on one stream.
+ *                 16-byte aligned; its contents are overwritten (no initial
+ *                 contents are needed).  Calls that share a workspace must be
+ *                 ordered on one stream.
  */
 PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_heads,

@@ -134,10 +134,8 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, i
     const int p = pa_decode_partition_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
                                            max_context_len, partition_size);
     if (p <= 0 || num_seqs <= 0 || num_heads <= 0 || head_dim <= 0) return 0;
-    const size_t np = ((size_t)max_context_len + p - 1) / p;
-    if (np <= 1) return 0;
-    const size_t rows = (size_t)num_seqs * num_heads * np;
-    return rows * (size_t)(head_dim + 2) * sizeof(float);
+    const size_t np = max_context_len > 0 ? ((size_t)max_context_len + p - 1) / p : 1;
+    return decode_workspace((size_t)num_seqs, (size_t)num_heads, (size_t)head_dim, np).total;
 }
 
 pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -180,17 +178,19 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     const int p = resolve_partition(block_size, max_context_len, partition_size);
     if (p < 0) return (pa_status)p;
     const int np = max_context_len > 0 ? (max_context_len + p - 1) / p : 1;
+    const DecodeWorkspace wl = decode_workspace((size_t)num_seqs, (size_t)num_heads, (size_t)head_dim, (size_t)np);
+    if (!workspace || workspace_bytes < wl.total || !aligned(workspace, 16)) {
+        set_error("pa_decode: workspace missing, too small (need " + std::to_string(wl.total) +
+                  " bytes) or not 16-byte aligned");
+        return PA_ERR_INVALID;
+    }
     DecodeArgs a{};
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    a.plan = reinterpret_cast<unsigned int*>(ws + wl.plan);
+    a.plan_list = reinterpret_cast<uint2*>(ws + wl.list);
     if (np > 1) {
-        const size_t need = pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
-                                                     max_context_len, partition_size);
-        if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) {
-            set_error("pa_decode: workspace missing, too small (need " + std::to_string(need) +
-                      " bytes) or not 16-byte aligned");
-            return PA_ERR_INVALID;
-        }
-        a.ws_acc = static_cast<float*>(workspace);
-        a.ws_ml = a.ws_acc + (size_t)num_seqs * num_heads * np * head_dim;
+        a.ws_acc = reinterpret_cast<float*>(ws + wl.acc);
+        a.ws_ml = reinterpret_cast<float*>(ws + wl.ml);
     }
     unsigned int* status = nullptr;
     st = status_ptr(&status);
@@ -209,6 +209,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     a.num_blocks = num_blocks;
     a.max_context_len = max_context_len;
     a.partition_blocks = p / block_size;
+    a.adaptive = partition_size == 0 ? 1 : 0;
     a.num_partitions = np;
     a.scale_log2 = scale * 1.4426950408889634f;
     const cudaError_t e =

@@ -9,33 +9,42 @@
 // ("PagedAttention Paper Breakdown", section 2, Address Translation Formula).
 //
 // B200 design:
-//  * One CTA per (kv head, sequence, context partition).  All query heads of the
-//    kv head's group are packed into the CTA, so each K/V byte leaves HBM once.
-//  * A physical block's K tile (and its V tile) for one kv head is one contiguous run
-//    of B*D elements in the [num_blocks][kv_heads][B][D] pool, so a single producer
-//    thread streams whole tiles with 1-D bulk copies (the TMA engine, no tensor map,
-//    no multicast) into a ring of shared-memory stages guarded by mbarriers.
-//  * Four consumer warps take alternate blocks, each with its own online-softmax
-//    state; the states are merged once per partition.  Inside a warp every lane
-//    reads 16-byte vectors; the B x G logits are summed across the lanes of a row
-//    with a transposing butterfly (each step halves the values a lane holds), and the
-//    softmax weights are shared through a small per-warp shared buffer.
-//  * Sequences longer than one partition leave (max, sum, unnormalised output) per
-//    partition in the workspace; a second kernel merges them by log-sum-exp.  That
-//    kernel is launched with programmatic dependent launch so its launch overlaps the
-//    first kernel's tail.
+//  * Work units are (sequence, context partition, kv head).  All query heads of the
+//    kv head's group are packed into one unit, so each K/V byte leaves HBM once.
+//  * A plan kernel lists the (sequence, partition) pairs longest first; a persistent
+//    kernel (a few CTAs per SM) takes units from that list with an atomic counter, so
+//    the grid holds no empty CTAs and the short units are the ones left at the end.
+//  * In each CTA one warp fetches units ahead of use (block-table slice and q into a
+//    small shared ring), one thread streams the units' K/V tiles into a ring of
+//    shared-memory stages with the TMA engine (1-D bulk copies of whole tiles, or 2-D
+//    tensor boxes with the 128-byte swizzle for the tensor-core consumer; never
+//    multicast) and four consumer warps take alternate blocks.  The stream of tiles
+//    runs across unit boundaries, so the pipeline does not drain between units.
+//  * Consumers: CUDA cores (fp32; bf16 with one query head per kv head) or tensor
+//    cores (bf16 with 2, 4 or 8 query heads per kv head); see the two policy headers.
+//  * At the end of a unit the four warps' softmax states are merged; a sequence
+//    longer than one partition leaves (max, sum, unnormalised output) per partition in
+//    the workspace and a log-sum-exp merge kernel combines them.  Plan, persistent and
+//    merge kernels are chained with programmatic dependent launch.
 //  * Logits are kept in base-2 units (q pre-scaled by scale*log2 e) and exponentials
 //    use exp2f, the reformulation of online softmax by Milakov & Gimelshein (2018).
-//  * Every wait is bounded; bad block indices or context lengths raise a status bit
-//    and are clamped instead of being dereferenced.
+//  * Every wait is bounded: a wait that runs out raises PA_DEV_WAIT_TIMEOUT and the
+//    CTA winds down instead of hanging.  Bad block indices or context lengths raise a
+//    status bit and are clamped instead of being dereferenced.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
-#include <cfloat>
 #include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <type_traits>
 
 #include "pa_decode_common.cuh"
+#include "pa_decode_fma.cuh"
+#include "pa_decode_mma.cuh"
 #include "pa_internal.h"
 #include "pa_ptx.cuh"
 
@@ -43,368 +52,450 @@ namespace pa {
 
 namespace {
 
-template <typename T, int D, int B, int G>
-struct Cfg {
-    static constexpr int kElt = sizeof(T);
-    static constexpr int EPL = 16 / kElt;                 // elements per lane vector
-    static constexpr int LPR = D * kElt / 16;             // lanes covering one token row
-    static constexpr int RPW = 32 / LPR;                  // rows a warp reads per step
-    static constexpr int TPL = B / RPW;                   // row steps per block
-    static constexpr int TPC = cmax(1, cmin(TPL, 32 / G));  // row steps per softmax chunk
-    static constexpr int NCH = TPL / TPC;                 // chunks per block
-    static constexpr int NV = G * TPC;                    // partial logits per lane per chunk
-    static constexpr int NVO = NV >= LPR ? NV / LPR : 1;  // full logits a lane holds after the butterfly
-    static constexpr int DUP = NV >= LPR ? 1 : LPR / NV;  // lanes holding the same logit
-    static constexpr int LPH = LPR / G;                   // lanes of a row group sharing one head
-    static constexpr int TILE = B * D;                    // elements of one K (or V) tile
-    static constexpr int TILE_BYTES = TILE * kElt;
-    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-    static constexpr int NCW = 4;                         // consumer warps
-    // Stage i % NSTAGES holds block i and warp i % NCW consumes it.  With NSTAGES a
-    // multiple of NCW the warp that waits for a stage's n-th fill also consumed its
-    // (n-1)-th, so the one-bit phase parity of the wait can never be stale.
-    static constexpr int NSTAGES = cmax(NCW, cmin(8, 65536 / STAGE_BYTES));
-    static constexpr int THREADS = (NCW + 1) * 32;
-    static constexpr int MAX_PBLK = kMaxPartitionTokens / 16;
-    // shared-memory carve-up (bytes)
-    static constexpr int OFF_BAR = NSTAGES * STAGE_BYTES;
-    static constexpr int OFF_TABLE = OFF_BAR + 2 * NSTAGES * 8;
-    static constexpr int OFF_P = OFF_TABLE + MAX_PBLK * 4;
-    static constexpr int P_FLOATS = NCW * RPW * NV;       // per warp: [RPW][TPC][G]
-    static constexpr int OFF_M = OFF_P + P_FLOATS * 4;
-    static constexpr int OFF_ABORT = OFF_M + NCW * G * 4;
-    static constexpr int SMEM = OFF_ABORT + 16;
-    // merge area (aliases the stages once the pipeline has drained)
-    static constexpr int MERGE_BYTES = NCW * G * (D + 2) * 4;
+constexpr int kEndUnit = 1;    // no more work for this CTA
+constexpr int kSplitUnit = 2;  // the sequence spans several partitions
 
-    static_assert(16 % kElt == 0 && D % EPL == 0, "vector width");
-    static_assert(LPR >= 1 && LPR <= 32 && (32 % LPR) == 0, "row lanes");
-    static_assert(B % RPW == 0 && TPL % TPC == 0, "block split");
-    static_assert(G <= LPR, "group larger than a row's lanes");
-    static_assert(MERGE_BYTES <= OFF_BAR, "merge area must fit in the stage ring");
-    static_assert(TILE_BYTES % 16 == 0, "bulk copy size");
+struct UnitInfo {
+    int s, kvh, part, nb, b0, first, L, flags, np, pad[3];
+};
+
+// Shared-memory budget of one CTA: two CTAs per SM, each with about 96 KB of K/V
+// stages in flight, keep enough bytes moving to cover the HBM latency under load.
+constexpr int kCtaSmemBudget = 110 * 1024;
+
+// Cons: the consumer policy (tiles of Cons::B = 16 tokens); BS: the physical block
+// size.  A stage holds one 16-token tile of K and of V; a block of BS tokens is
+// BS / 16 consecutive tiles.
+template <class Cons, int BS>
+struct Persist {
+    using T = typename Cons::T;
+    static constexpr int D = Cons::D, G = Cons::G;
+    static constexpr int TR = Cons::B;                  // tokens per stage
+    static constexpr int SPB = BS / TR;                 // stages per physical block
+    static constexpr int TILE_BYTES = TR * D * (int)sizeof(T);
+    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;  // K tile, then V tile
+    static constexpr int NCW = 4;                       // consumer warps
+    static constexpr int UR = 2;                        // units held: the current one and the next
+    static constexpr int MAX_PBLK = kMaxPartitionTokens / 16;
+    static constexpr int QBYTES = G * D * (int)sizeof(T);
+    static constexpr int SLOT_BYTES = (QBYTES + MAX_PBLK * 4 + (int)sizeof(UnitInfo) + 127) / 128 * 128;
+    static constexpr int THREADS = (NCW + 2) * 32;      // consumers, tile producer, unit producer
+    static constexpr int MERGE_FLOATS = NCW * G * (D + 2);
+    static constexpr int NBAR_FIXED = 3 * UR + 1;
+    static constexpr int FIXED_BYTES = UR * SLOT_BYTES + MERGE_FLOATS * 4 + NCW * Cons::SCRATCH_FLOATS * 4 +
+                                       NBAR_FIXED * 8 + 16 + 1024;
+    // Stage i of the CTA's stream is consumed by warp i % NCW.  With NSTAGES a multiple
+    // of NCW the warp that waits for a stage's n-th fill also consumed its (n-1)-th, so
+    // a one-bit phase parity is never stale.
+    static constexpr int NSTAGES =
+        cmax(NCW, cmin(24, ((kCtaSmemBudget - FIXED_BYTES - 16 * 24) / STAGE_BYTES) / NCW * NCW));
+    static constexpr int OFF_SLOT = NSTAGES * STAGE_BYTES;
+    static constexpr int OFF_MERGE = OFF_SLOT + UR * SLOT_BYTES;
+    static constexpr int OFF_SCRATCH = OFF_MERGE + MERGE_FLOATS * 4;
+    static constexpr int OFF_BAR = (OFF_SCRATCH + NCW * Cons::SCRATCH_FLOATS * 4 + 7) / 8 * 8;
+    static constexpr int NBAR = 2 * NSTAGES + NBAR_FIXED;
+    static constexpr int OFF_ABORT = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM = OFF_ABORT + 16 + 1024;  // + slack to align the base to 1024 bytes
+
+    static_assert(BS % TR == 0, "block size must be a multiple of the stage tile");
     static_assert(NSTAGES % NCW == 0, "stage ring must be a multiple of the consumer warps");
+    static_assert(TILE_BYTES % 1024 == 0, "tiles keep the 1024-byte alignment of the swizzle atoms");
+    static_assert(QBYTES % 16 == 0, "q rows are bulk-copied");
     static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
-// Sums N per-lane values across the LPR lanes of each row group (xor offsets
-// LPR/2 .. 1), halving the values a lane holds at each step while N >= 2.  Lane c
-// of a group ends with max(1, N/LPR) full sums, value indices starting at c*N/LPR.
-template <int N, int OFF>
-struct Butterfly {
-    static __device__ __forceinline__ void run(float* v, int lane)
-    {
-        if constexpr (OFF >= 1) {
-            if constexpr (N >= 2) {
-                const bool up = (lane & OFF) != 0;
-#pragma unroll
-                for (int i = 0; i < N / 2; ++i) {
-                    const float lo = v[i];
-                    const float hi = v[i + N / 2];
-                    const float send = up ? lo : hi;
-                    const float keep = up ? hi : lo;
-                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, OFF);
-                }
-                Butterfly<N / 2, OFF / 2>::run(v, lane);
-            } else {
-                v[0] += __shfl_xor_sync(0xffffffffu, v[0], OFF);
-                Butterfly<1, OFF / 2>::run(v, lane);
-            }
-        }
-    }
-};
-
-// Max (or sum) over the lanes that share a head: the LPH lanes inside a row group
-// and the same lanes of every row group.
-template <int LPH, int LPR, bool MAX>
-__device__ __forceinline__ float head_allreduce(float x)
+// Moves 16-token tile h of one physical block's K and V into a stage; completion is
+// counted on bar.
+template <class Cons, int BS>
+__device__ __forceinline__ void issue_tile(unsigned char* stage, const DecodeArgs& a, const CUtensorMap* tk,
+                                           const CUtensorMap* tv, int phys, int kvh, int h, uint64_t* bar,
+                                           uint64_t policy)
 {
+    using P = Persist<Cons, BS>;
+    mbar_arrive_expect_tx(bar, 2 * P::TILE_BYTES);
+    if constexpr (Cons::kTensorLoads) {
+        const int row = (phys * a.num_kv_heads + kvh) * BS + h * P::TR;
+        const uint32_t dk = smem_u32(stage);
 #pragma unroll
-    for (int o = 1; o < LPH; o <<= 1) {
-        const float y = __shfl_xor_sync(0xffffffffu, x, o);
-        x = MAX ? fmaxf(x, y) : x + y;
+        for (int hh = 0; hh < Cons::NHALF; ++hh) {
+            tma_load_2d(dk + hh * Cons::HALF_BYTES, tk, hh * 64, row, bar, policy);
+            tma_load_2d(dk + P::TILE_BYTES + hh * Cons::HALF_BYTES, tv, hh * 64, row, bar, policy);
+        }
+    } else {
+        const size_t off = (((size_t)phys * a.num_kv_heads + kvh) * BS + (size_t)h * P::TR) * P::D * sizeof(typename P::T);
+        bulk_g2s_hint(stage, static_cast<const unsigned char*>(a.k_cache) + off, P::TILE_BYTES, bar, policy);
+        bulk_g2s_hint(stage + P::TILE_BYTES, static_cast<const unsigned char*>(a.v_cache) + off, P::TILE_BYTES,
+                      bar, policy);
     }
-#pragma unroll
-    for (int o = LPR; o < 32; o <<= 1) {
-        const float y = __shfl_xor_sync(0xffffffffu, x, o);
-        x = MAX ? fmaxf(x, y) : x + y;
-    }
-    return x;
 }
 
-// Three CTAs per SM (about 200 KB of stages in flight); a group of 8 heads needs
-// more registers per thread and runs two.
-template <typename T, int D, int B, int G>
-__global__ void __launch_bounds__(Cfg<T, D, B, G>::THREADS, (G >= 8 ? 2 : 3))
-    decode_partition_kernel(const DecodeArgs a)
+// Barrier among the consumer warps (an mbarrier, so the wait is bounded).
+__device__ __forceinline__ bool consumer_sync(uint64_t* bar, int n, int lane, volatile int* abort_flag)
 {
-    using C = Cfg<T, D, B, G>;
-    extern __shared__ __align__(128) unsigned char smem[];
-    T* stages = reinterpret_cast<T*>(smem);
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-    uint64_t* empty_bar = full_bar + C::NSTAGES;
-    int* s_table = reinterpret_cast<int*>(smem + C::OFF_TABLE);
-    float* s_p = reinterpret_cast<float*>(smem + C::OFF_P);
-    float* s_m = reinterpret_cast<float*>(smem + C::OFF_M);
-    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_ABORT);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
+    return mbar_wait_bounded(bar, n & 1, abort_flag);
+}
 
-    const int kvh = blockIdx.x;
-    const int s = blockIdx.y;
-    const int part = blockIdx.z;
+template <class Cons, int BS>
+__global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
+    decode_persistent_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
+                             const __grid_constant__ CUtensorMap tmap_v)
+{
+    using P = Persist<Cons, BS>;
+    using T = typename Cons::T;
+    constexpr int D = P::D, B = BS, G = P::G, NCW = P::NCW, NS = P::NSTAGES, UR = P::UR, TR = P::TR,
+                  SPB = P::SPB;
+
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::OFF_BAR);
+    uint64_t* full = bars;            // stage filled (tx bytes)
+    uint64_t* empty = bars + NS;      // stage consumed
+    uint64_t* ufull = bars + 2 * NS;  // unit slot filled (q bytes)
+    uint64_t* uempty = ufull + UR;    // unit slot released (consumers and tile producer)
+    uint64_t* utab = uempty + UR;     // unit slot's block-table slice written (tile producer)
+    uint64_t* group = utab + UR;      // consumer-warp barrier
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + P::OFF_ABORT);
+    float* mg_m = reinterpret_cast<float*>(smem + P::OFF_MERGE);
+    float* mg_l = mg_m + NCW * G;
+    float* mg_acc = mg_l + NCW * G;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Sequences that fit in fewer partitions exit at once; the exit also lets the
-    // merge kernel (programmatic dependent launch) start once every CTA got here.
     pdl_launch_dependents();
-
-    int L = __ldg(a.context_lens + s);
-    const int Lcap = min(a.max_context_len, a.max_blocks_per_seq * B);
-    if (L < 0 || L > Lcap) {
-        if (threadIdx.x == 0 && part == 0 && kvh == 0) atomicOr(a.status, PA_DEV_BAD_CONTEXT);
-        L = L < 0 ? 0 : Lcap;
-    }
-    const int nblk_seq = (L + B - 1) / B;
-    const int pb = a.partition_blocks;
-    const int b0 = part * pb;
-    if (part > 0 && b0 >= nblk_seq) return;
-    const int nblk = max(0, min(pb, nblk_seq - b0));
-    const bool split = nblk_seq > pb;
-
-    for (int i = threadIdx.x; i < nblk; i += C::THREADS)
-        s_table[i] = __ldg(a.block_tables + (size_t)s * a.max_blocks_per_seq + b0 + i);
     if (threadIdx.x == 0) {
-#pragma unroll
-        for (int st = 0; st < C::NSTAGES; ++st) {
-            mbar_init(&full_bar[st], 1);
-            mbar_init(&empty_bar[st], 1);
+        for (int st = 0; st < NS; ++st) {
+            mbar_init(&full[st], 1);
+            mbar_init(&empty[st], 1);
         }
-        *s_abort = 0;
+        for (int u = 0; u < UR; ++u) {
+            mbar_init(&ufull[u], 1);
+            mbar_init(&uempty[u], 2);
+            mbar_init(&utab[u], 1);
+        }
+        mbar_init(group, NCW);
+        *abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
+    pdl_wait_primary();  // the plan kernel's list and counter are visible after this
 
-    const float NEG_INF = -INFINITY;
-    const int c = lane % C::LPR;  // 16-byte column chunk of the row this lane reads
-    const int r = lane / C::LPR;  // row group
-    float m_run[G];               // running max per head (same in every lane)
-    float acc[G][C::EPL];         // unnormalised output, this lane's columns, row group r
-    float l_own = 0.f;            // running sum of this lane's logits (head g_own)
-    float m_own = NEG_INF;        // running max of head g_own
-    const int g_own = (c * G) / C::LPR;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        m_run[g] = NEG_INF;
-#pragma unroll
-        for (int e = 0; e < C::EPL; ++e) acc[g][e] = 0.f;
-    }
+    auto slot = [&](int k) { return smem + P::OFF_SLOT + (k % UR) * P::SLOT_BYTES; };
+    auto slot_table = [&](int k) { return reinterpret_cast<int*>(slot(k) + P::QBYTES); };
+    auto slot_info = [&](int k) { return reinterpret_cast<UnitInfo*>(slot(k) + P::QBYTES + P::MAX_PBLK * 4); };
 
-    if (warp == C::NCW) {
-        // ---------------- producer: one thread streams K/V tiles into the ring
+    if (warp == NCW + 1) {
+        // ---------------- unit producer: takes units from the plan, fills the unit ring
+        unsigned npairs = 0;
+        if (lane == 0) npairs = *reinterpret_cast<volatile unsigned*>(a.plan + 1);
+        npairs = __shfl_sync(0xffffffffu, npairs, 0);
+        const unsigned nunits = npairs * (unsigned)a.num_kv_heads;
+        int first = 0;
+        int k = 0;
+        bool ended = false;
+        for (;; ++k) {
+            if (k >= UR && !mbar_wait_bounded(&uempty[k % UR], ((k / UR) & 1) ^ 1, abort_flag)) {
+                if (lane == 0) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+                *abort_flag = 1;
+                break;
+            }
+            UnitInfo* info = slot_info(k);
+            // the first unit of CTA b is unit b; later ones come from the counter
+            unsigned u = blockIdx.x;
+            if (k > 0) {
+                if (lane == 0) u = gridDim.x + atomicAdd(a.plan, 1u);
+                u = __shfl_sync(0xffffffffu, u, 0);
+            }
+            if (u >= nunits) {
+                if (lane == 0) {
+                    info->flags = kEndUnit;
+                    mbar_arrive(&utab[k % UR]);
+                    mbar_arrive(&ufull[k % UR]);
+                }
+                ended = true;
+                break;
+            }
+            const uint2 e = a.plan_list[u / (unsigned)a.num_kv_heads];
+            const int kvh = (int)(u % (unsigned)a.num_kv_heads);
+            const int s = (int)(e.x >> 11);
+            const int part = (int)(e.x & 2047u);
+            const int L = (int)e.y;
+            const int nblk_seq = (L + B - 1) / B;
+            const int pb = (int)a.plan[2];
+            const int b0 = part * pb;
+            const int nb = max(0, min(pb, nblk_seq - b0));
+            int* tab = slot_table(k);
+            for (int i = lane; i < nb; i += 32)
+                tab[i] = __ldg(a.block_tables + (size_t)s * a.max_blocks_per_seq + b0 + i);
+            if (lane == 0) {
+                info->s = s;
+                info->kvh = kvh;
+                info->part = part;
+                info->nb = nb;
+                info->b0 = b0;
+                info->first = first;
+                info->L = L;
+                info->flags = nblk_seq > pb ? kSplitUnit : 0;
+                info->np = (nblk_seq + pb - 1) / pb;
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&utab[k % UR]);  // the tile producer may start on this unit
+                mbar_arrive_expect_tx(&ufull[k % UR], P::QBYTES);
+                bulk_g2s(slot(k), static_cast<const T*>(a.q) + ((size_t)s * a.num_heads + (size_t)kvh * G) * D,
+                         P::QBYTES, &ufull[k % UR]);
+            }
+            first += nb * SPB;
+        }
+        // No q copy may still be landing in shared memory at exit: wait for the fills of
+        // the last units.  After an end marker, slot k % UR has moved on past unit k - UR
+        // (a parity wait on that older phase would alias), so only units k-UR+1 .. k-1.
         if (lane == 0) {
-            const T* kc = static_cast<const T*>(a.k_cache);
-            const T* vc = static_cast<const T*>(a.v_cache);
+            volatile int never = 0;
+            const int j0 = k - UR + (ended ? 1 : 0);
+            for (int j = j0 < 0 ? 0 : j0; j < k; ++j)
+                if (!mbar_wait_bounded(&ufull[j % UR], (j / UR) & 1, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+        }
+    } else if (warp == NCW) {
+        // ---------------- tile producer: one thread streams K/V tiles into the stages
+        if (lane == 0) {
             const uint64_t policy = policy_evict_first();
-            int issued = 0;
+            int i = 0;  // blocks issued so far (the CTA's stream index)
             bool ok = true;
-            for (int i = 0; i < nblk; ++i) {
-                const int st = i % C::NSTAGES;
-                if (i >= C::NSTAGES &&
-                    !mbar_wait_bounded(&empty_bar[st], ((i / C::NSTAGES) & 1) ^ 1, s_abort)) {
+            for (int k = 0; ok; ++k) {
+                if (!mbar_wait_bounded(&utab[k % UR], (k / UR) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                int phys = s_table[i];
-                if ((unsigned)phys >= (unsigned)a.num_blocks) {
-                    atomicOr(a.status, PA_DEV_BAD_BLOCK);
-                    phys = 0;
+                const UnitInfo* info = slot_info(k);
+                if (info->flags & kEndUnit) break;
+                const int nt = info->nb * SPB;
+                const int kvh = info->kvh;
+                const int* tab = slot_table(k);
+                int phys = 0;
+                for (int j = 0; j < nt; ++j, ++i) {
+                    const int st = i % NS;
+                    if (i >= NS && !mbar_wait_bounded(&empty[st], ((i / NS) & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (j % SPB == 0) {
+                        phys = tab[j / SPB];
+                        if ((unsigned)phys >= (unsigned)a.num_blocks) {
+                            atomicOr(a.status, PA_DEV_BAD_BLOCK);
+                            phys = 0;
+                        }
+                    }
+                    issue_tile<Cons, BS>(smem + st * P::STAGE_BYTES, a, &tmap_k, &tmap_v, phys, kvh, j % SPB,
+                                         &full[st], policy);
                 }
-                const size_t off = ((size_t)phys * a.num_kv_heads + kvh) * C::TILE;
-                T* dk = stages + (size_t)st * 2 * C::TILE;
-                mbar_arrive_expect_tx(&full_bar[st], 2 * C::TILE_BYTES);
-                bulk_g2s_hint(dk, kc + off, C::TILE_BYTES, &full_bar[st], policy);
-                bulk_g2s_hint(dk + C::TILE, vc + off, C::TILE_BYTES, &full_bar[st], policy);
-                ++issued;
+                // done with this unit's table: the slot may be refilled once the consumers are done too
+                if (ok) mbar_arrive(&uempty[k % UR]);
             }
             if (!ok) {
                 atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
-                *s_abort = 1;
+                *abort_flag = 1;
             }
-            // Drain: no bulk copy may still be landing in shared memory at exit.
+            // no tile copy may still be landing in shared memory at exit
             volatile int never = 0;
-            for (int i = max(0, issued - C::NSTAGES); i < issued; ++i)
-                if (!mbar_wait_bounded(&full_bar[i % C::NSTAGES], (i / C::NSTAGES) & 1, &never))
-                    atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+            for (int j = i - NS < 0 ? 0 : i - NS; j < i; ++j)
+                if (!mbar_wait_bounded(&full[j % NS], (j / NS) & 1, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
         }
     } else {
         // ---------------- consumers
-        float qf[G][C::EPL];
-        {
-            const T* qp = static_cast<const T*>(a.q) + ((size_t)s * a.num_heads + (size_t)kvh * G) * D;
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                load16_f32<T>(qp + g * D + c * C::EPL, qf[g]);
-#pragma unroll
-                for (int e = 0; e < C::EPL; ++e) qf[g][e] *= a.scale_log2;
-            }
-        }
-        float* p_w = s_p + warp * (C::RPW * C::NV);  // [RPW][TPC][G]
-        float* m_w = s_m + warp * G;
-        const int idx0 = (c * C::NV) / C::LPR;       // first logit index this lane holds
-
-        for (int i = warp; i < nblk; i += C::NCW) {
-            const int st = i % C::NSTAGES;
-            if (!mbar_wait_bounded(&full_bar[st], (i / C::NSTAGES) & 1, s_abort)) {
-                atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
-                *s_abort = 1;
+        Cons cons;
+        cons.init(reinterpret_cast<float*>(smem + P::OFF_SCRATCH) + warp * Cons::SCRATCH_FLOATS, lane);
+        int nsync = 0;
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+            if (!mbar_wait_bounded(&ufull[k % UR], (k / UR) & 1, abort_flag)) {
+                ok = false;
                 break;
             }
-            const T* kt = stages + (size_t)st * 2 * C::TILE;
-            const T* vt = kt + C::TILE;
-            const int nvalid = min(B, L - (b0 + i) * B);
-
-#pragma unroll
-            for (int ch = 0; ch < C::NCH; ++ch) {
-                // q . K for this chunk's rows: v[g*TPC + t], row j = (ch*TPC + t)*RPW + r
-                float v[C::NV];
-#pragma unroll
-                for (int t = 0; t < C::TPC; ++t) {
-                    const int j = (ch * C::TPC + t) * C::RPW + r;
-                    float kf[C::EPL];
-                    load16_f32<T>(kt + j * D + c * C::EPL, kf);
-#pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        float sum = 0.f;
-#pragma unroll
-                        for (int e = 0; e < C::EPL; ++e) sum = fmaf(qf[g][e], kf[e], sum);
-                        v[g * C::TPC + t] = sum;
-                    }
+            const UnitInfo* info = slot_info(k);
+            if (info->flags & kEndUnit) break;
+            const int first = info->first, nt = info->nb * SPB, L = info->L;
+            const int tok0 = info->b0 * B;  // first token of the unit
+            cons.begin_unit(reinterpret_cast<const T*>(slot(k)), a.scale_log2);
+            for (int i = first + ((warp - first % NCW) + NCW) % NCW; i < first + nt; i += NCW) {
+                const int st = i % NS;
+                if (!mbar_wait_bounded(&full[st], (i / NS) & 1, abort_flag)) {
+                    ok = false;
+                    break;
                 }
-                Butterfly<C::NV, C::LPR / 2>::run(v, lane);
-
-                // This lane now holds logits idx0 .. idx0+NVO-1, all of head g_own.
-                float cmax_ = NEG_INF;
-#pragma unroll
-                for (int k = 0; k < C::NVO; ++k) {
-                    const int t = (idx0 + k) % C::TPC;
-                    const int j = (ch * C::TPC + t) * C::RPW + r;
-                    if (j >= nvalid) v[k] = NEG_INF;
-                    cmax_ = fmaxf(cmax_, v[k]);
-                }
-                cmax_ = head_allreduce<C::LPH, C::LPR, true>(cmax_);
-                const float m_new = fmaxf(m_own, cmax_);
-                const float alpha_own = exp2f(m_own - m_new);
-                m_own = m_new;
-                float psum = 0.f;
-#pragma unroll
-                for (int k = 0; k < C::NVO; ++k) {
-                    const float p = exp2f(v[k] - m_new);
-                    psum += p;
-                    const int t = (idx0 + k) % C::TPC;
-                    p_w[(r * C::TPC + t) * G + g_own] = p;
-                }
-                l_own = l_own * alpha_own + psum;
-                m_w[g_own] = m_new;
+                unsigned char* stage = smem + st * P::STAGE_BYTES;
+                cons.block(stage, stage + P::TILE_BYTES, min(TR, L - tok0 - (i - first) * TR));
                 __syncwarp();
-
-                // rescale the accumulators of heads whose max moved
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float mg = m_w[g];
-                    if (mg != m_run[g]) {
-                        const float alpha = exp2f(m_run[g] - mg);
-#pragma unroll
-                        for (int e = 0; e < C::EPL; ++e) acc[g][e] *= alpha;
-                        m_run[g] = mg;
-                    }
-                }
-                // P . V for this chunk's rows
-#pragma unroll
-                for (int t = 0; t < C::TPC; ++t) {
-                    const int j = (ch * C::TPC + t) * C::RPW + r;
-                    if (j < nvalid) {
-                        float vf[C::EPL];
-                        load16_f32<T>(vt + j * D + c * C::EPL, vf);
-                        float pg[G];
-                        const float* pp = p_w + (r * C::TPC + t) * G;
-#pragma unroll
-                        for (int g = 0; g < G; ++g) pg[g] = pp[g];
-#pragma unroll
-                        for (int g = 0; g < G; ++g)
-#pragma unroll
-                            for (int e = 0; e < C::EPL; ++e) acc[g][e] = fmaf(pg[g], vf[e], acc[g][e]);
-                    }
-                }
-                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);
             }
-            if (lane == 0) mbar_arrive(&empty_bar[st]);
+            if (!ok) break;
+            cons.end_unit(mg_m, mg_l, mg_acc, warp);
+            if (!consumer_sync(group, nsync++, lane, abort_flag)) {
+                ok = false;
+                break;
+            }
+            finish_partition<T, D, G, NCW, NCW * 32>(a, mg_m, mg_l, mg_acc, info->s, info->kvh, info->part,
+                                                     (info->flags & kSplitUnit) != 0, threadIdx.x);
+            if (!consumer_sync(group, nsync++, lane, abort_flag)) {
+                ok = false;
+                break;
+            }
+            if (threadIdx.x == 0) mbar_arrive(&uempty[k % UR]);
         }
-
-        // fold the row groups together (same columns, different rows)
-#pragma unroll
-        for (int o = C::LPR; o < 32; o <<= 1)
-#pragma unroll
-            for (int g = 0; g < G; ++g)
-#pragma unroll
-                for (int e = 0; e < C::EPL; ++e) acc[g][e] += __shfl_xor_sync(0xffffffffu, acc[g][e], o);
-        l_own = head_allreduce<C::LPH, C::LPR, false>(l_own) * (1.0f / C::DUP);
-    }
-
-    __syncthreads();  // the stage ring is free from here on: reuse it for the merge
-
-    float* mg_m = reinterpret_cast<float*>(smem);       // [NCW][G]
-    float* mg_l = mg_m + C::NCW * G;                    // [NCW][G]
-    float* mg_acc = mg_l + C::NCW * G;                  // [NCW][G][D]
-    if (warp < C::NCW) {
-        if (lane == 0)
-#pragma unroll
-            for (int g = 0; g < G; ++g) mg_m[warp * G + g] = m_run[g];
-        if (r == 0) {
-#pragma unroll
-            for (int g = 0; g < G; ++g)
-#pragma unroll
-                for (int e = 0; e < C::EPL; ++e) mg_acc[(warp * G + g) * D + c * C::EPL + e] = acc[g][e];
+        if (!ok) {
+            if (lane == 0) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+            *abort_flag = 1;
         }
-        if (c % C::LPH == 0 && r == 0) mg_l[warp * G + g_own] = l_own;
     }
-    __syncthreads();
-
-    finish_partition<T, D, G, C::NCW, C::THREADS>(a, mg_m, mg_l, mg_acc, s, kvh, part, split);
 }
 
-template <typename T, int D, int B, int G>
-cudaError_t launch_typed(const DecodeArgs& a, cudaStream_t stream)
-{
-    using C = Cfg<T, D, B, G>;
-    // The shared-memory opt-in is a per-device function attribute: set it once per device.
-    static std::atomic<uint64_t> attr_set{0};
-    int dev = 0;
-    cudaError_t e0 = cudaGetDevice(&dev);
-    if (e0 != cudaSuccess) return e0;
-    const uint64_t bit = 1ull << (dev & 63);
-    if (!(attr_set.load() & bit)) {
-        cudaError_t e = cudaFuncSetAttribute(decode_partition_kernel<T, D, B, G>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set.fetch_or(bit);
-    }
-    dim3 grid(a.num_kv_heads, a.num_seqs, a.num_partitions);
-    decode_partition_kernel<T, D, B, G><<<grid, C::THREADS, C::SMEM, stream>>>(a);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess || a.num_partitions <= 1) return e;
+// ---------------------------------------------------------------- tensor maps
 
-    return launch_merge<T, D>(a, B, stream);
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// The pool [num_blocks][kv_heads][B][D] as a 2-D bf16 tensor of rows of D elements;
+// boxes of 64 columns x `B` rows (one stage tile), 128-byte swizzle.  A small cache avoids re-encoding
+// the maps of the same pools on every call.
+cudaError_t tensor_map(CUtensorMap* out, const void* pool, uint64_t rows, int D, int B)
+{
+    struct Entry {
+        const void* ptr;
+        uint64_t rows;
+        int d, b, dev;
+        CUtensorMap map;
+    };
+    static std::mutex mu;
+    static Entry cache[16] = {};
+    static int next = 0;
+    int dev = 0;
+    cudaError_t ce = cudaGetDevice(&dev);
+    if (ce != cudaSuccess) return ce;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        for (auto& en : cache)
+            if (en.ptr == pool && en.rows == rows && en.d == D && en.b == B && en.dev == dev) {
+                *out = en.map;
+                return cudaSuccess;
+            }
+    }
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    CUtensorMap m;
+    std::memset(&m, 0, sizeof(m));
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)B};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    std::lock_guard<std::mutex> lk(mu);
+    Entry& en = cache[next];
+    next = (next + 1) % 16;
+    en.ptr = pool;
+    en.rows = rows;
+    en.d = D;
+    en.b = B;
+    en.dev = dev;
+    en.map = m;
+    *out = m;
+    return cudaSuccess;
+}
+
+// ---------------------------------------------------------------- launch
+
+// CTAs of the persistent kernel resident on the current device at once (cached per device).
+template <class Cons, int BS>
+cudaError_t resident_ctas(int* out)
+{
+    using P = Persist<Cons, BS>;
+    static std::atomic<int> cached[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const int d = dev & 63;
+    int v = cached[d].load();
+    if (v == 0) {
+        e = cudaFuncSetAttribute(decode_persistent_kernel<Cons, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 P::SMEM);
+        if (e != cudaSuccess) return e;
+        int occ = 0, sms = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_persistent_kernel<Cons, BS>, P::THREADS,
+                                                          P::SMEM);
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        v = (occ < 1 ? 1 : occ) * sms;
+        cached[d].store(v);
+    }
+    *out = v;
+    return cudaSuccess;
+}
+
+template <class Cons, int BS>
+cudaError_t launch_persistent(const DecodeArgs& a, cudaStream_t stream)
+{
+    using P = Persist<Cons, BS>;
+    CUtensorMap tk, tv;
+    std::memset(&tk, 0, sizeof(tk));
+    std::memset(&tv, 0, sizeof(tv));
+    if constexpr (Cons::kTensorLoads) {
+        const uint64_t rows = (uint64_t)a.num_blocks * a.num_kv_heads * BS;
+        cudaError_t e = tensor_map(&tk, a.k_cache, rows, P::D, P::TR);
+        if (e != cudaSuccess) return e;
+        e = tensor_map(&tv, a.v_cache, rows, P::D, P::TR);
+        if (e != cudaSuccess) return e;
+    }
+    int ctas = 0;
+    cudaError_t e = resident_ctas<Cons, BS>(&ctas);
+    if (e != cudaSuccess) return e;
+    const int64_t units = (int64_t)a.num_kv_heads * a.num_seqs * a.num_partitions;
+    const unsigned grid = (unsigned)(units < ctas ? units : ctas);
+    DecodeArgs args = a;
+    args.num_ctas = (int)grid;
+
+    decode_plan_kernel<<<1, 1024, 0, stream>>>(args, BS);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(decode_persistent_kernel<Cons, BS>, dim3(grid), dim3(P::THREADS), (size_t)P::SMEM, stream, args,
+                   tk, tv);
+    if (e != cudaSuccess || a.num_partitions <= 1) return e;
+    return launch_merge<typename Cons::T, P::D>(args, BS, stream);
 }
 
 template <typename T, int D, int B>
 cudaError_t dispatch_group(const DecodeArgs& a, int group, cudaStream_t stream)
 {
-    switch (group) {
-        case 1: return launch_typed<T, D, B, 1>(a, stream);
-        case 2: return launch_typed<T, D, B, 2>(a, stream);
-        case 4: return launch_typed<T, D, B, 4>(a, stream);
-        case 8: return launch_typed<T, D, B, 8>(a, stream);
-        default: return cudaErrorInvalidValue;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        switch (group) {
+            case 1: return launch_persistent<FmaConsumer<T, D, 16, 1>, B>(a, stream);
+            case 2: return launch_persistent<MmaConsumer<D, 16, 2>, B>(a, stream);
+            case 4: return launch_persistent<MmaConsumer<D, 16, 4>, B>(a, stream);
+            case 8: return launch_persistent<MmaConsumer<D, 16, 8>, B>(a, stream);
+            default: return cudaErrorInvalidValue;
+        }
+    } else {
+        switch (group) {
+            case 1: return launch_persistent<FmaConsumer<T, D, 16, 1>, B>(a, stream);
+            case 2: return launch_persistent<FmaConsumer<T, D, 16, 2>, B>(a, stream);
+            case 4: return launch_persistent<FmaConsumer<T, D, 16, 4>, B>(a, stream);
+            case 8: return launch_persistent<FmaConsumer<T, D, 16, 8>, B>(a, stream);
+            default: return cudaErrorInvalidValue;
+        }
     }
 }
 
@@ -430,10 +521,14 @@ cudaError_t dispatch_dim(const DecodeArgs& a, int head_dim, int block_size, int 
 
 }  // namespace
 
+bool decode_uses_tensor_cores(pa_dtype dtype, int head_dim, int group)
+{
+    return dtype == PA_DTYPE_BF16 && (head_dim == 64 || head_dim == 128) && (group == 2 || group == 4 || group == 8);
+}
+
 cudaError_t launch_decode(const DecodeArgs& a, pa_dtype dtype, int head_dim, int block_size, int group,
                           cudaStream_t stream)
 {
-    if (decode_uses_tensor_cores(dtype, head_dim, group)) return launch_decode_mma(a, head_dim, block_size, group, stream);
     if (dtype == PA_DTYPE_F32) return dispatch_dim<float>(a, head_dim, block_size, group, stream);
     return dispatch_dim<__nv_bfloat16>(a, head_dim, block_size, group, stream);
 }

@@ -1,12 +1,14 @@
-// Pieces shared by the two decode kernels (CUDA-core and tensor-core consumers):
-// vector loads, the per-partition epilogue that merges the consumer warps'
-// softmax states, and the log-sum-exp merge kernel across partitions.
+// Pieces of the paged decode path shared by its two consumers (CUDA cores and
+// tensor cores): vector loads, the longest-first work plan, the per-partition
+// epilogue that merges the consumer warps' softmax states, and the log-sum-exp
+// merge of a sequence's context partitions.
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <utility>
 
 #include "pa_internal.h"
 #include "pa_ptx.cuh"
@@ -53,27 +55,143 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x)
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
 constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
+// Context length of sequence s as the kernels use it: clamped to what the launch
+// covers (a value outside [0, Lcap] raises PA_DEV_BAD_CONTEXT where flag is set).
+__device__ __forceinline__ int clamped_context(const DecodeArgs& a, int s, int block_size, bool flag)
+{
+    int L = __ldg(a.context_lens + s);
+    const int Lcap = min(a.max_context_len, a.max_blocks_per_seq * block_size);
+    if (L < 0 || L > Lcap) {
+        if (flag) atomicOr(a.status, PA_DEV_BAD_CONTEXT);
+        L = L < 0 ? 0 : Lcap;
+    }
+    return L;
+}
+
+// Work plan: every (sequence, context partition) pair, longest first.  A pair
+// covers the partition's blocks; its kv heads are separate work units, handed
+// out in list order by an atomic counter.  Full partitions come first, then the
+// sequences' last partitions by decreasing length (a counting sort on the block
+// count), so the units left at the end of the grid are the short ones.  Order
+// within a length is arbitrary and does not change any result.  Each entry also
+// carries the (clamped) context length.
+//
+// With `adaptive` set the partition may grow (doubling from partition_blocks, up to
+// the longest context) while the largest unit stays within a quarter of one CTA's
+// share of all the work: fewer sequences are split, yet every CTA still gets
+// several units to balance with.  The choice is written to plan[2].
+__global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeArgs a, int block_size)
+{
+    __shared__ int bucket[kMaxPartitionTokens / 16 + 1];
+    __shared__ unsigned long long s_tok[32];
+    __shared__ int s_max[32];
+    __shared__ int s_pb;
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+    // total and longest context
+    unsigned long long tok = 0;
+    int lmax = 0;
+    for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
+        const int L = clamped_context(a, s, block_size, true);
+        tok += (unsigned long long)L;
+        lmax = max(lmax, L);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        tok += __shfl_xor_sync(0xffffffffu, tok, o);
+        lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+    }
+    if (lane == 0) {
+        s_tok[warp] = tok;
+        s_max[warp] = lmax;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned long long t = 0;
+        int m = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+            t += s_tok[w];
+            m = max(m, s_max[w]);
+        }
+        int pb = a.partition_blocks;
+        if (a.adaptive) {
+            const int max_pb = kMaxPartitionTokens / block_size;
+            const double share = (double)t / (double)(a.num_ctas > 0 ? a.num_ctas : 1);  // tokens per CTA, per kv head
+            while (2 * pb <= max_pb && pb * block_size < m &&
+                   (double)min(2 * pb * block_size, m) * 4.0 <= share)
+                pb *= 2;
+        }
+        s_pb = pb;
+        a.plan[2] = (unsigned)pb;
+    }
+    __syncthreads();
+    const int pb = s_pb;
+    const int P = pb * block_size;
+    for (int i = threadIdx.x; i <= pb; i += blockDim.x) bucket[i] = 0;
+    __syncthreads();
+    for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
+        const int L = clamped_context(a, s, block_size, false);
+        const int np = L > 0 ? (L + P - 1) / P : 1;
+        const int last = L > 0 ? (L - (np - 1) * P + block_size - 1) / block_size : 0;
+        if (np > 1) atomicAdd(&bucket[pb], np - 1);
+        atomicAdd(&bucket[last], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // exclusive scan over sizes, largest first: start[sz] = pairs of size > sz
+        int running = 0;
+        for (int base = pb; base >= 0; base -= 32) {
+            const int sz = base - lane;
+            const int c = sz >= 0 ? bucket[sz] : 0;
+            int x = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (sz >= 0) bucket[sz] = running + x - c;
+            running += __shfl_sync(0xffffffffu, x, 31);
+        }
+        if (lane == 0) {
+            a.plan[0] = 0u;                 // work counter
+            a.plan[1] = (unsigned)running;  // number of (sequence, partition) pairs
+        }
+    }
+    __syncthreads();
+    for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
+        const int L = clamped_context(a, s, block_size, false);
+        const int np = L > 0 ? (L + P - 1) / P : 1;
+        const int last = L > 0 ? (L - (np - 1) * P + block_size - 1) / block_size : 0;
+        for (int p = 0; p < np; ++p) {
+            const int sz = p < np - 1 ? pb : last;
+            const int pos = atomicAdd(&bucket[sz], 1);
+            a.plan_list[pos] = make_uint2(((unsigned)s << 11) | (unsigned)p, (unsigned)L);
+        }
+    }
+}
+
 // Merges the NCW consumer warps' states (m: running max, l: softmax sum, acc:
 // unnormalised output, all relative to m) of one (sequence, kv head, partition)
 // and writes either the final output row (the sequence fits in one partition) or
-// the partition's state to the workspace.
-template <typename T, int D, int G, int NCW, int THREADS>
+// the partition's state to the workspace.  Run by the NTHR consumer threads.
+template <typename T, int D, int G, int NCW, int NTHR>
 __device__ __forceinline__ void finish_partition(const DecodeArgs& a, const float* mg_m, const float* mg_l,
-                                                 const float* mg_acc, int s, int kvh, int part, bool split)
+                                                 const float* mg_acc, int s, int kvh, int part, bool split, int tid)
 {
     const int NP = a.num_partitions;
-    for (int idx = threadIdx.x; idx < G * D; idx += THREADS) {
+    for (int idx = tid; idx < G * D; idx += NTHR) {
         const int g = idx / D;
         const int d = idx % D;
-        float M = (-INFINITY);
+        float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < NCW; ++w) M = fmaxf(M, mg_m[w * G + g]);
         float num = 0.f, den = 0.f;
-        if (M != (-INFINITY)) {
+        if (M != -INFINITY) {
 #pragma unroll
             for (int w = 0; w < NCW; ++w) {
                 const float mw = mg_m[w * G + g];
-                if (mw != (-INFINITY)) {
+                if (mw != -INFINITY) {
                     const float sc = exp2f(mw - M);
                     num = fmaf(sc, mg_acc[(w * G + g) * D + d], num);
                     den = fmaf(sc, mg_l[w * G + g], den);
@@ -95,76 +213,118 @@ __device__ __forceinline__ void finish_partition(const DecodeArgs& a, const floa
     }
 }
 
-// Log-sum-exp merge of the partitions of one (sequence, query head):
-// M = max_p m_p, out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p.
+// Log-sum-exp merge of the partitions of one (sequence, query head) per CTA:
+// M = max_p m_p, out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p.  The four
+// warps take partitions p = w, w+4, ...; a lane owns D/32 consecutive columns (16-byte
+// loads for D = 128).  Each warp computes the weights of 32 of its partitions at once
+// (one per lane) and broadcasts them, keeping the column loads of four partitions in
+// flight; the warps' sums meet in shared memory.
 template <typename T, int D>
-__global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a, int partition_tokens, int block_size)
+__global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a, int block_size)
 {
-    pdl_wait_primary();
-    __shared__ float s_w[kMaxPartitions];
+    constexpr int EPL = D / 32;
     __shared__ float s_red[4];
-    __shared__ float s_den;
-    const int h = blockIdx.x;
-    const int s = blockIdx.y;
-    int L = __ldg(a.context_lens + s);
-    const int Lcap = min(a.max_context_len, a.max_blocks_per_seq * block_size);
-    L = L < 0 ? 0 : (L > Lcap ? Lcap : L);
-    const int np = (L + partition_tokens - 1) / partition_tokens;
-    if (np <= 1) return;  // written directly by the partition kernel
-    const int NP = a.num_partitions;
-    const size_t row0 = ((size_t)s * a.num_heads + h) * NP;
-    const float* ml = a.ws_ml + row0 * 2;
+    __shared__ float s_den[4];
+    __shared__ float s_num[4][D];
+    pdl_wait_primary();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int row = blockIdx.x;  // s * num_heads + h
+    const int s = row / a.num_heads;
+    const int P = (int)a.plan[2] * block_size;
+    const int L = clamped_context(a, s, block_size, false);
+    const int np = (L + P - 1) / P;
+    if (np <= 1) return;  // written directly by the persistent kernel
+    const size_t row0 = (size_t)row * a.num_partitions;
+    const float2* ml = reinterpret_cast<const float2*>(a.ws_ml) + row0;
 
     float M = -INFINITY;
-    for (int p = threadIdx.x; p < np; p += blockDim.x) M = fmaxf(M, ml[2 * p]);
+    for (int p = threadIdx.x; p < np; p += 128) M = fmaxf(M, ml[p].x);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = M;
+    if (lane == 0) s_red[warp] = M;
     __syncthreads();
     M = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
-    __syncthreads();
 
+    float num[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) num[e] = 0.f;
     float den = 0.f;
-    for (int p = threadIdx.x; p < np; p += blockDim.x) {
-        const float mp = ml[2 * p];
-        const float w = (mp == -INFINITY) ? 0.f : exp2f(mp - M);
-        s_w[p] = w;
-        den = fmaf(w, ml[2 * p + 1], den);
+    const float* acc = a.ws_acc + row0 * D + lane * EPL;
+    const int mine = np > warp ? (np - warp + 3) / 4 : 0;  // partitions of this warp: warp + 4 * j
+    for (int jc = 0; jc < mine; jc += 32) {
+        float w = 0.f;
+        if (jc + lane < mine) {
+            const float2 v = ml[warp + 4 * (jc + lane)];
+            w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
+            den = fmaf(w, v.y, den);
+        }
+        const int cnt = min(32, mine - jc);
+        int j = 0;
+        for (; j + 4 <= cnt; j += 4) {
+            float x[4][EPL];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float* src = acc + (size_t)(warp + 4 * (jc + j + u)) * D;
+                if constexpr (EPL == 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(src);
+                    x[u][0] = v.x; x[u][1] = v.y; x[u][2] = v.z; x[u][3] = v.w;
+                } else {
+                    const float2 v = *reinterpret_cast<const float2*>(src);
+                    x[u][0] = v.x; x[u][1] = v.y;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float wj = __shfl_sync(0xffffffffu, w, j + u);
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) num[e] = fmaf(wj, x[u][e], num[e]);
+            }
+        }
+        for (; j < cnt; ++j) {
+            const float wj = __shfl_sync(0xffffffffu, w, j);
+            const float* src = acc + (size_t)(warp + 4 * (jc + j)) * D;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) num[e] = fmaf(wj, src[e], num[e]);
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = den;
+    if (lane == 0) s_den[warp] = den;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) s_num[warp][lane * EPL + e] = num[e];
     __syncthreads();
-    if (threadIdx.x == 0) s_den = s_red[0] + s_red[1] + s_red[2] + s_red[3];
-    __syncthreads();
-    const float inv = s_den > 0.f ? 1.f / s_den : 0.f;
-
-    T* o = static_cast<T*>(a.out) + ((size_t)s * a.num_heads + h) * D;
-    for (int d = threadIdx.x; d < D; d += blockDim.x) {
-        float num = 0.f;
-        const float* accp = a.ws_acc + row0 * D + d;
-        for (int p = 0; p < np; ++p) num = fmaf(s_w[p], accp[(size_t)p * D], num);
-        o[d] = from_f32<T>(num * inv);
-    }
+    const float tot = s_den[0] + s_den[1] + s_den[2] + s_den[3];
+    const float inv = tot > 0.f ? 1.f / tot : 0.f;
+    T* o = static_cast<T*>(a.out) + (size_t)row * D;
+    for (int d = threadIdx.x; d < D; d += 128)
+        o[d] = from_f32<T>((s_num[0][d] + s_num[1][d] + s_num[2][d] + s_num[3][d]) * inv);
 }
 
-// Launches the merge kernel after a partition kernel with programmatic dependent
-// launch: its CTAs may be scheduled while the partition kernel drains and wait
-// (griddepcontrol.wait) until that kernel's writes are visible.
-template <typename T, int D>
-cudaError_t launch_merge(const DecodeArgs& a, int block_size, cudaStream_t stream)
+// Launches a kernel with programmatic dependent launch: its CTAs may be scheduled
+// while the previous kernel in the stream drains; they wait (griddepcontrol.wait)
+// before touching that kernel's results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args)
 {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.num_heads, a.num_seqs, 1);
-    cfg.blockDim = dim3(128, 1, 1);
-    cfg.dynamicSmemBytes = 0;
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_merge_kernel<T, D>, a, a.partition_blocks * block_size, block_size);
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename T, int D>
+cudaError_t launch_merge(const DecodeArgs& a, int block_size, cudaStream_t stream)
+{
+    const unsigned rows = (unsigned)(a.num_seqs * a.num_heads);
+    return launch_pdl(decode_merge_kernel<T, D>, dim3(rows), dim3(128), 0, stream, a, block_size);
 }
 
 }  // namespace

@@ -21,7 +21,9 @@ struct DecodeArgs {
     const void* v_cache;
     const int32_t* block_tables;
     const int32_t* context_lens;
-    float* ws_acc;             // [S][Hq][NP][D] unnormalised partition outputs
+    unsigned int* plan;        // [0] work counter, [1] (sequence, partition) pairs, [2] blocks per partition
+    uint2* plan_list;          // [S * NP] longest first: {sequence << 11 | partition, context length}
+    float* ws_acc;             // [S][Hq][NP][D] unnormalised partition outputs (NP > 1)
     float* ws_ml;              // [S][Hq][NP][2] (running max in log2 units, softmax sum)
     unsigned int* status;      // device status word (PA_DEV_* bits)
     int num_seqs;
@@ -30,18 +32,42 @@ struct DecodeArgs {
     int max_blocks_per_seq;
     int num_blocks;
     int max_context_len;
-    int partition_blocks;      // blocks per context partition
-    int num_partitions;        // NP = ceil(max_context_len / partition tokens)
+    int partition_blocks;      // blocks per context partition (the smallest the plan may use)
+    int adaptive;              // non-zero: the plan may use a multiple of partition_blocks
+    int num_ctas;              // CTAs of the persistent kernel
+    int num_partitions;        // NP = ceil(max_context_len / smallest partition tokens)
     float scale_log2;          // scale * log2(e): logits are kept in base-2 units
 };
 
+// Byte layout of the decode workspace: the work plan, then (when a sequence may
+// span several partitions) the partition states.
+struct DecodeWorkspace {
+    size_t plan;       // 16 bytes: counter, pair count, blocks per partition
+    size_t list;       // 8 * S * NP bytes
+    size_t acc;        // 4 * S * Hq * NP * D bytes (0 bytes when NP == 1)
+    size_t ml;         // 8 * S * Hq * NP bytes (0 bytes when NP == 1)
+    size_t total;
+};
+
+inline DecodeWorkspace decode_workspace(size_t S, size_t Hq, size_t D, size_t NP)
+{
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    const bool split = NP > 1;
+    DecodeWorkspace w{};
+    w.plan = 0;
+    w.list = 16;
+    w.acc = up(w.list + 8 * S * NP);
+    w.ml = up(w.acc + (split ? 4 * S * Hq * NP * D : 0));
+    w.total = up(w.ml + (split ? 8 * S * Hq * NP : 0));
+    return w;
+}
+
+// One call: the plan kernel, the persistent kernel (tensor cores for bf16 with a group
+// of 2, 4 or 8 query heads per kv head, CUDA cores otherwise) and, when a sequence may
+// span several partitions, the log-sum-exp merge kernel.
 cudaError_t launch_decode(const DecodeArgs& a, pa_dtype dtype, int head_dim, int block_size, int group,
                           cudaStream_t stream);
-
-// bf16 with a group of 2, 4 or 8 query heads per kv head runs on the tensor cores
-// (pa_decode_mma.cu); everything else on the CUDA cores (pa_decode.cu).
 bool decode_uses_tensor_cores(pa_dtype dtype, int head_dim, int group);
-cudaError_t launch_decode_mma(const DecodeArgs& a, int head_dim, int block_size, int group, cudaStream_t stream);
 
 struct ReshapeArgs {
     const void* key;

@@ -121,7 +121,8 @@ def pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_
 
 def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale, partition_size=0,
               workspace=None, stream=None):
-    """out[S,Hq,D] <- paged decode attention of q[S,Hq,D] over k/v_cache[NB,Hkv,B,D]."""
+    """out[S,Hq,D] <- paged decode attention of q[S,Hq,D] over k/v_cache[NB,Hkv,B,D].
+    Without `workspace` a buffer of pa_decode_workspace_size() bytes is allocated for the call."""
     S, Hq, D = q.shape
     NB, Hkv, B, D2 = k_cache.shape
     if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
@@ -134,9 +135,10 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
     import torch
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
         raise TypeError("block_tables and context_lens must be int32")
-    ws_ptr, ws_bytes = None, 0
-    if workspace is not None:
-        ws_ptr, ws_bytes = _dev_ptr(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    if workspace is None:
+        need = pa_decode_workspace_size(S, Hq, Hkv, D, B, int(max_context_len), int(partition_size))
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    ws_ptr, ws_bytes = _dev_ptr(workspace, "workspace"), workspace.numel() * workspace.element_size()
     st = lib.pa_decode(_dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
                        _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables"),
                        _dev_ptr(context_lens, "context_lens"), S, Hq, Hkv, D, B, block_tables.shape[1], NB,

@@ -137,6 +137,37 @@ def test_zero_length_context_gives_zero_row(pa, dtype):
     _status_clean(pa)
 
 
+@pytest.mark.parametrize("dtype,G", [("bf16", 1), ("bf16", 4), ("f32", 2)])
+def test_many_short_and_empty_sequences(pa, dtype, G):
+    """Hundreds of tiny or empty contexts: many work units per persistent CTA, units
+    without blocks, partial blocks everywhere, a few sequences split in partitions."""
+    rng = np.random.default_rng(G)
+    S, Hkv, D, B = 600, 2, 128, 16
+    lens = rng.choice([0, 0, 1, 2, 15, 16, 17, 33, 100], size=S).astype(np.int32)
+    lens[::97] = 700
+    dt = W.torch_dtype(dtype)
+    nblk = [(int(L) + B - 1) // B for L in lens]
+    NB = sum(nblk) + 11
+    perm = rng.permutation(NB)
+    tables = np.full((S, max(nblk)), -1, np.int32)
+    pos = 0
+    for s_, n in enumerate(nblk):
+        tables[s_, :n] = perm[pos:pos + n]
+        pos += n
+    g = torch.Generator().manual_seed(G)
+    q = torch.randn(S, Hkv * G, D, generator=g).to(dt)
+    k = torch.randn(NB, Hkv, B, D, generator=g).to(dt)
+    v = torch.randn(NB, Hkv, B, D, generator=g).to(dt)
+    out = torch.full((S, Hkv * G, D), 3.0, dtype=dt, device="cuda")
+    pa.pa_decode(out, q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda(),
+                 int(lens.max()), 0.2, partition_size=256)
+    ref = oracle.decode(q.float().numpy(), k.float().numpy(), v.float().numpy(), tables, lens, 0.2, nthreads=8)
+    o = out.float().cpu().numpy()
+    assert np.all(o[lens == 0] == 0)
+    assert max_abs(o, ref) <= TOL[dtype]
+    _status_clean(pa)
+
+
 # ------------------------------------------------------------------ companions, bit-exact
 
 @pytest.mark.parametrize("dtype,D,B", [("f32", 64, 16), ("bf16", 128, 16), ("bf16", 128, 32), ("f32", 128, 32)])

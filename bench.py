@@ -69,22 +69,31 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+DECODE_SOURCES = ("pa_decode.cu", "pa_decode_common.cuh", "pa_decode_fma.cuh", "pa_decode_mma.cuh", "pa_ptx.cuh")
+
+
+def decode_source_hash():
+    """Hash of the decode kernel sources (ties a committed profile to the code it measured)."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "paged_kv_cache_363_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def profile_traffic(kernel, workload):
     """dram bytes per launch from the committed ncu summary for this kernel and workload,
-    if its recorded source hash still matches the kernel source; else None."""
-    import hashlib
+    if its recorded source hash still matches the decode sources; else None."""
     path = os.path.join(ROOT, "profiles", "%s_%s.md" % (kernel, workload))
-    src = os.path.join(ROOT, "paged_kv_cache_363_b200", "csrc", "pa_decode.cu")
     try:
-        with open(src, "rb") as f:
-            h = hashlib.sha256(f.read()).hexdigest()[:16]
         fields = {}
         with open(path) as f:
             for line in f:
                 if ":" in line and line.startswith("- "):
                     k, v = line[2:].split(":", 1)
                     fields[k.strip()] = v.strip().strip("`")
-        if fields.get("source_sha256_16") != h:
+        if fields.get("source_sha256_16") != decode_source_hash():
             return None
         return float(fields["traffic_bytes_per_launch"])
     except Exception:
@@ -400,7 +409,7 @@ def run_gpu(args):
         "roofline": {"bound": "hbm", "kernel": "pa_decode (plan kernel + persistent decode kernel)",
                      "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": profile_traffic("decode_partition_kernel", wl.name),
+                     "traffic": profile_traffic("decode_persistent_kernel", wl.name),
                      "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_us": round(dec_avg_max * 1e3, 3)},
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,

@@ -188,6 +188,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     unsigned char* ws = static_cast<unsigned char*>(workspace);
     a.plan = reinterpret_cast<unsigned int*>(ws + wl.plan);
     a.plan_list = reinterpret_cast<uint2*>(ws + wl.list);
+    a.split_list = reinterpret_cast<unsigned int*>(ws + wl.splits);
     if (np > 1) {
         a.ws_acc = reinterpret_cast<float*>(ws + wl.acc);
         a.ws_ml = reinterpret_cast<float*>(ws + wl.ml);

@@ -86,6 +86,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeArgs a, i
     __shared__ unsigned long long s_tok[32];
     __shared__ int s_max[32];
     __shared__ int s_pb;
+    __shared__ int s_nsplit;
     pdl_launch_dependents();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
@@ -123,6 +124,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeArgs a, i
                 pb *= 2;
         }
         s_pb = pb;
+        s_nsplit = 0;
         a.plan[2] = (unsigned)pb;
     }
     __syncthreads();
@@ -134,7 +136,10 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeArgs a, i
         const int L = clamped_context(a, s, block_size, false);
         const int np = L > 0 ? (L + P - 1) / P : 1;
         const int last = L > 0 ? (L - (np - 1) * P + block_size - 1) / block_size : 0;
-        if (np > 1) atomicAdd(&bucket[pb], np - 1);
+        if (np > 1) {
+            atomicAdd(&bucket[pb], np - 1);
+            a.split_list[atomicAdd(&s_nsplit, 1)] = (unsigned)s;
+        }
         atomicAdd(&bucket[last], 1);
     }
     __syncthreads();
@@ -156,6 +161,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeArgs a, i
         if (lane == 0) {
             a.plan[0] = 0u;                 // work counter
             a.plan[1] = (unsigned)running;  // number of (sequence, partition) pairs
+            a.plan[3] = (unsigned)s_nsplit; // sequences that need the merge
         }
     }
     __syncthreads();
@@ -213,91 +219,78 @@ __device__ __forceinline__ void finish_partition(const DecodeArgs& a, const floa
     }
 }
 
-// Log-sum-exp merge of the partitions of one (sequence, query head) per CTA:
-// M = max_p m_p, out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p.  The four
-// warps take partitions p = w, w+4, ...; a lane owns D/32 consecutive columns (16-byte
-// loads for D = 128).  Each warp computes the weights of 32 of its partitions at once
-// (one per lane) and broadcasts them, keeping the column loads of four partitions in
-// flight; the warps' sums meet in shared memory.
+// Log-sum-exp merge of the partitions of the split sequences the plan listed, one
+// (sequence, query head) row per warp, warps striding over the rows:
+// M = max_p m_p, out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p.  A lane owns
+// D/32 consecutive columns (16-byte loads for D = 128); the weights of 32 partitions
+// are computed at once (one per lane) and broadcast, and the column loads of eight
+// partitions are in flight together.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a, int block_size)
 {
     constexpr int EPL = D / 32;
-    __shared__ float s_red[4];
-    __shared__ float s_den[4];
-    __shared__ float s_num[4][D];
+    constexpr int U = 8;
     pdl_wait_primary();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int row = blockIdx.x;  // s * num_heads + h
-    const int s = row / a.num_heads;
+    const int lane = threadIdx.x & 31;
     const int P = (int)a.plan[2] * block_size;
-    const int L = clamped_context(a, s, block_size, false);
-    const int np = (L + P - 1) / P;
-    if (np <= 1) return;  // written directly by the persistent kernel
-    const size_t row0 = (size_t)row * a.num_partitions;
-    const float2* ml = reinterpret_cast<const float2*>(a.ws_ml) + row0;
+    const int rows = (int)a.plan[3] * a.num_heads;
+    const int nwarps = gridDim.x * (blockDim.x >> 5);
+    for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += nwarps) {
+        const int s = (int)a.split_list[r / a.num_heads];
+        const int row = s * a.num_heads + r % a.num_heads;
+        const int L = clamped_context(a, s, block_size, false);
+        const int np = (L + P - 1) / P;
+        const size_t row0 = (size_t)row * a.num_partitions;
+        const float2* ml = reinterpret_cast<const float2*>(a.ws_ml) + row0;
 
-    float M = -INFINITY;
-    for (int p = threadIdx.x; p < np; p += 128) M = fmaxf(M, ml[p].x);
+        float M = -INFINITY;
+        for (int p = lane; p < np; p += 32) M = fmaxf(M, ml[p].x);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if (lane == 0) s_red[warp] = M;
-    __syncthreads();
-    M = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
-
-    float num[EPL];
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float num[EPL];
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) num[e] = 0.f;
-    float den = 0.f;
-    const float* acc = a.ws_acc + row0 * D + lane * EPL;
-    const int mine = np > warp ? (np - warp + 3) / 4 : 0;  // partitions of this warp: warp + 4 * j
-    for (int jc = 0; jc < mine; jc += 32) {
-        float w = 0.f;
-        if (jc + lane < mine) {
-            const float2 v = ml[warp + 4 * (jc + lane)];
-            w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
-            den = fmaf(w, v.y, den);
-        }
-        const int cnt = min(32, mine - jc);
-        int j = 0;
-        for (; j + 4 <= cnt; j += 4) {
-            float x[4][EPL];
+        for (int e = 0; e < EPL; ++e) num[e] = 0.f;
+        float den = 0.f;
+        const float* acc = a.ws_acc + row0 * D + lane * EPL;
+        for (int pc = 0; pc < np; pc += 32) {
+            float w = 0.f;
+            if (pc + lane < np) {
+                const float2 v = ml[pc + lane];
+                w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
+                den = fmaf(w, v.y, den);
+            }
+            const int cnt = min(32, np - pc);
+            for (int j = 0; j < cnt; j += U) {
+                float x[U][EPL];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float* src = acc + (size_t)(warp + 4 * (jc + j + u)) * D;
-                if constexpr (EPL == 4) {
-                    const float4 v = *reinterpret_cast<const float4*>(src);
-                    x[u][0] = v.x; x[u][1] = v.y; x[u][2] = v.z; x[u][3] = v.w;
-                } else {
-                    const float2 v = *reinterpret_cast<const float2*>(src);
-                    x[u][0] = v.x; x[u][1] = v.y;
+                for (int u = 0; u < U; ++u) {
+                    const float* src = acc + (size_t)(pc + min(j + u, cnt - 1)) * D;
+                    if constexpr (EPL == 4) {
+                        const float4 v = *reinterpret_cast<const float4*>(src);
+                        x[u][0] = v.x; x[u][1] = v.y; x[u][2] = v.z; x[u][3] = v.w;
+                    } else {
+                        const float2 v = *reinterpret_cast<const float2*>(src);
+                        x[u][0] = v.x; x[u][1] = v.y;
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    // lanes past the partition count hold weight 0, so the clamped
+                    // (repeated) loads above add nothing
+                    const float wj = __shfl_sync(0xffffffffu, w, min(j + u, 31));
+                    const float wu = j + u < cnt ? wj : 0.f;
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) num[e] = fmaf(wu, x[u][e], num[e]);
                 }
             }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float wj = __shfl_sync(0xffffffffu, w, j + u);
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) num[e] = fmaf(wj, x[u][e], num[e]);
-            }
         }
-        for (; j < cnt; ++j) {
-            const float wj = __shfl_sync(0xffffffffu, w, j);
-            const float* src = acc + (size_t)(warp + 4 * (jc + j)) * D;
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) num[e] = fmaf(wj, src[e], num[e]);
-        }
+        for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        T* o = static_cast<T*>(a.out) + (size_t)row * D + lane * EPL;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) o[e] = from_f32<T>(num[e] * inv);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    if (lane == 0) s_den[warp] = den;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) s_num[warp][lane * EPL + e] = num[e];
-    __syncthreads();
-    const float tot = s_den[0] + s_den[1] + s_den[2] + s_den[3];
-    const float inv = tot > 0.f ? 1.f / tot : 0.f;
-    T* o = static_cast<T*>(a.out) + (size_t)row * D;
-    for (int d = threadIdx.x; d < D; d += 128)
-        o[d] = from_f32<T>((s_num[0][d] + s_num[1][d] + s_num[2][d] + s_num[3][d]) * inv);
 }
 
 // Launches a kernel with programmatic dependent launch: its CTAs may be scheduled
@@ -323,8 +316,12 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 template <typename T, int D>
 cudaError_t launch_merge(const DecodeArgs& a, int block_size, cudaStream_t stream)
 {
-    const unsigned rows = (unsigned)(a.num_seqs * a.num_heads);
-    return launch_pdl(decode_merge_kernel<T, D>, dim3(rows), dim3(128), 0, stream, a, block_size);
+    // up to eight CTAs (32 warps) per SM; the warps loop over the rows of the split sequences
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long ctas = ((long)a.num_seqs * a.num_heads + 3) / 4;
+    const unsigned grid = (unsigned)(ctas < 8L * sms ? ctas : 8L * sms);
+    return launch_pdl(decode_merge_kernel<T, D>, dim3(grid), dim3(128), 0, stream, a, block_size);
 }
 
 }  // namespace

@@ -21,8 +21,10 @@ struct DecodeArgs {
     const void* v_cache;
     const int32_t* block_tables;
     const int32_t* context_lens;
-    unsigned int* plan;        // [0] work counter, [1] (sequence, partition) pairs, [2] blocks per partition
+    unsigned int* plan;        // [0] work counter, [1] (sequence, partition) pairs, [2] blocks per
+                               // partition, [3] sequences split into several partitions
     uint2* plan_list;          // [S * NP] longest first: {sequence << 11 | partition, context length}
+    unsigned int* split_list;  // [S] the sequences split into several partitions (plan[3] of them)
     float* ws_acc;             // [S][Hq][NP][D] unnormalised partition outputs (NP > 1)
     float* ws_ml;              // [S][Hq][NP][2] (running max in log2 units, softmax sum)
     unsigned int* status;      // device status word (PA_DEV_* bits)
@@ -42,8 +44,9 @@ struct DecodeArgs {
 // Byte layout of the decode workspace: the work plan, then (when a sequence may
 // span several partitions) the partition states.
 struct DecodeWorkspace {
-    size_t plan;       // 16 bytes: counter, pair count, blocks per partition
+    size_t plan;       // 16 bytes: counter, pair count, blocks per partition, split count
     size_t list;       // 8 * S * NP bytes
+    size_t splits;     // 4 * S bytes
     size_t acc;        // 4 * S * Hq * NP * D bytes (0 bytes when NP == 1)
     size_t ml;         // 8 * S * Hq * NP bytes (0 bytes when NP == 1)
     size_t total;
@@ -56,7 +59,8 @@ inline DecodeWorkspace decode_workspace(size_t S, size_t Hq, size_t D, size_t NP
     DecodeWorkspace w{};
     w.plan = 0;
     w.list = 16;
-    w.acc = up(w.list + 8 * S * NP);
+    w.splits = up(w.list + 8 * S * NP);
+    w.acc = up(w.splits + 4 * S);
     w.ml = up(w.acc + (split ? 4 * S * Hq * NP * D : 0));
     w.total = up(w.ml + (split ? 8 * S * Hq * NP : 0));
     return w;

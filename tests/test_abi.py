@@ -72,11 +72,11 @@ def test_partition_and_workspace_sizes():
     with pytest.raises(pa.PAError):
         pa.pa_decode_partition_size(8, 32, 8, 128, 16, 10 ** 7, 16)      # too many partitions
     up = lambda x: (x + 255) // 256 * 256
-    # one partition: only the work plan (16-byte header, one 8-byte entry per sequence)
-    assert pa.pa_decode_workspace_size(4, 4, 4, 64, 16, 100, 512) == up(16 + 8 * 4)
-    # plan (S * NP entries), then S * Hq * NP * D floats and S * Hq * NP (max, sum) pairs
+    # one partition: only the work plan (16-byte header, one 8-byte entry and a split slot per sequence)
+    assert pa.pa_decode_workspace_size(4, 4, 4, 64, 16, 100, 512) == up(up(16 + 8 * 4) + 4 * 4)
+    # plan (S * NP entries, S split slots), then S * Hq * NP * D floats and S * Hq * NP (max, sum) pairs
     S, Hq, Hkv, D, NP = 8, 32, 8, 128, 64
-    acc = up(16 + 8 * S * NP)
+    acc = up(up(16 + 8 * S * NP) + 4 * S)
     ml = up(acc + 4 * S * Hq * NP * D)
     assert pa.pa_decode_workspace_size(S, Hq, Hkv, D, 32, 32768, 512) == up(ml + 8 * S * Hq * NP)
     assert pa.pa_decode_workspace_size(0, 32, 8, 128, 32, 32768, 512) == 0

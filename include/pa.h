@@ -124,6 +124,38 @@ PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const 
                     int max_context_len, float scale, int partition_size, void* workspace,
                     size_t workspace_bytes, pa_dtype dtype, void* stream);
 
+/*
+ * Fixed size of the library's own decode workspace used by
+ * pa_decode_static_workspace: 16 MiB of device memory on every GPU that loads
+ * the library, held until the process exits.
+ */
+#define PA_STATIC_WORKSPACE_BYTES (16u * 1024u * 1024u)
+
+/*
+ * pa_decode without a caller workspace, for callers that cannot allocate device
+ * memory: for example a plugin or script host that only hands out pointers to
+ * tensors it already owns, or a process whose memory pool must not be bypassed.
+ * The pages describe no such call (no counterpart there); it exists for these
+ * callers only.  Arguments, layouts and results are those of pa_decode; the
+ * workspace is a fixed array in the library (PA_STATIC_WORKSPACE_BYTES).
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *  - The first call made on a device resolves that device's array address
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Arguments whose pa_decode_workspace_size() exceeds
+ *    PA_STATIC_WORKSPACE_BYTES return PA_ERR_UNSUPPORTED before any device work
+ *    (a larger partition_size needs less).
+ *  - All calls on a device share one array, which keeps the last call's
+ *    contents; no part of it needs to start at zero (every call writes what it
+ *    later reads).  Calls that may run at the same time on one device (for
+ *    example on two unordered streams) race on it: order them on one stream.
+ */
+PA_API pa_status pa_decode_static_workspace(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                            const int32_t* block_tables, const int32_t* context_lens,
+                                            int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                            int block_size, int max_blocks_per_seq, int num_blocks,
+                                            int max_context_len, float scale, int partition_size,
+                                            pa_dtype dtype, void* stream);
+
 /* ------------------------------------------------------------------ KV append */
 
 /*

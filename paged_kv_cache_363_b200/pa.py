@@ -36,6 +36,7 @@ SIGNATURES = [
     ("pa_decode_partition_size", _int, [_int] * 7),
     ("pa_decode_workspace_size", _sz, [_int] * 7),
     ("pa_decode", _int, [_vp, _vp, _vp, _vp, _vp, _vp] + [_int] * 8 + [_f32, _int, _vp, _sz, _int, _vp]),
+    ("pa_decode_static_workspace", _int, [_vp, _vp, _vp, _vp, _vp, _vp] + [_int] * 8 + [_f32, _int, _int, _vp]),
     ("pa_reshape_and_cache", _int, [_vp, _vp, _vp, _vp, _vp] + [_int] * 6 + [_vp]),
     ("pa_copy_blocks", _int, [_vp, _vp, _vp] + [_int] * 6 + [_vp]),
     ("pa_device_status", _int, [ctypes.POINTER(_u32), _vp]),
@@ -145,6 +146,30 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
                        int(max_context_len), float(scale), int(partition_size), ws_ptr, ws_bytes, dt,
                        _stream(stream))
     _check(st, "pa_decode")
+    return out
+
+
+PA_STATIC_WORKSPACE_BYTES = 16 * 1024 * 1024
+
+
+def pa_decode_static_workspace(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
+                               partition_size=0, stream=None):
+    """pa_decode for callers that cannot allocate device memory: the workspace is the
+    library's own fixed 16 MiB device array (see include/pa.h).  Calls on one device
+    share that array, so calls that could overlap must be ordered on one stream."""
+    S, Hq, D = q.shape
+    NB, Hkv, B, D2 = k_cache.shape
+    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or tuple(context_lens.shape) != (S,):
+        raise ValueError("block_tables must be [S, max_blocks] and context_lens [S]")
+    dt = _dtype_code(q)
+    st = lib.pa_decode_static_workspace(_dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
+                                        _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables"),
+                                        _dev_ptr(context_lens, "context_lens"), S, Hq, Hkv, D, B,
+                                        block_tables.shape[1], NB, int(max_context_len), float(scale),
+                                        int(partition_size), dt, _stream(stream))
+    _check(st, "pa_decode_static_workspace")
     return out
 
 

@@ -289,6 +289,36 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ the CUDA path
 
+def e2e_leg(stepper, args, world, dev):
+    """Device time of `args.steps` host-fed steps (upload, kernels, read-back), max over ranks."""
+    import torch
+    import torch.distributed as dist
+
+    for _ in range(args.warmup):
+        stepper.submit()
+    stepper.drain()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e_s = torch.cuda.Event(enable_timing=True)
+    e_e = torch.cuda.Event(enable_timing=True)
+    # the first upload is ordered after e_s: the copy stream waits for the compute stream
+    e_s.record(stepper.stream)
+    stepper.h2d_stream.wait_event(e_s)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        i = stepper.submit()
+        stepper.host_inputs(i)            # the host may refill the buffer: its upload is done
+    stepper.drain()
+    e_e.record(stepper.stream)
+    host_s = time.perf_counter() - t0
+    torch.cuda.synchronize(dev)
+    ms = reduce_max(e_s.elapsed_time(e_e), dev)
+    if world > 1:
+        dist.barrier()
+    return {"ms": ms, "h2d": stepper.h2d_bytes, "d2h": stepper.d2h_bytes, "host_us": 1e6 * host_s / args.steps}
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -328,7 +358,8 @@ def run_gpu(args):
     dec_bytes = batch.decode_bytes()
     step_bytes = dec_bytes + batch.append_bytes()
     cow_launch = 1 if getattr(batch, "cow_pairs", None) is not None and batch.cow_pairs.numel() else 0
-    launches_per_step = 1 + cow_launch + 2   # append, [copy], plan + persistent decode
+    # [copy-on-write copies], append, plan, persistent decode, [merge of split sequences]
+    launches_per_step = cow_launch + 1 + 2 + (1 if n_part > 1 else 0)
 
     # ---- device-resident timing
     for _ in range(args.warmup):
@@ -362,38 +393,19 @@ def run_gpu(args):
 
     e2e = None
     if not args.skip_e2e:
-        # ---- end to end through the API, inputs and result in pinned host memory
-        host = {}
-        for name in ("q", "new_k", "new_v", "slot_mapping", "block_tables", "context_lens"):
-            t = getattr(batch, name)
-            host[name] = t.cpu().pin_memory()
-        out_host = torch.empty(batch.out.shape, dtype=batch.out.dtype).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in host.values())
-        d2h = out_host.numel() * out_host.element_size()
-
-        def e2e_step():
-            for name, t in host.items():
-                getattr(batch, name).copy_(t, non_blocking=True)
-            batch.step(stream)
-            out_host.copy_(batch.out, non_blocking=True)
-
-        for _ in range(args.warmup):
-            e2e_step()
-        torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
-        e_s = torch.cuda.Event(enable_timing=True)
-        e_e = torch.cuda.Event(enable_timing=True)
-        e_s.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e_e.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = reduce_max(e_s.elapsed_time(e_e), dev)
-        if world > 1:
-            dist.barrier()
-        e2e = {"value": round(world * step_bytes * args.steps / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 5)}
+        # ---- end to end through the API: every step uploads its inputs from pinned host
+        # memory in one copy and reads its output back; two buffers overlap the copies of
+        # neighbouring steps with this step's kernels (depth 1 = no overlap, also reported)
+        gbs = lambda ms: round(world * step_bytes * args.steps / (ms * 1e-3) / 1e9, 2)
+        nbuf, graph = args.e2e_buffers, bool(args.e2e_graph)
+        main_leg = e2e_leg(runner.HostStepper(batch, depth=nbuf, stream=stream, graph=graph), args, world, dev)
+        serial = e2e_leg(runner.HostStepper(batch, depth=1, stream=stream), args, world, dev)
+        e2e = {"value": gbs(main_leg["ms"]), "unit": "GB/s",
+               "h2d_bytes_per_step": main_leg["h2d"], "d2h_bytes_per_step": main_leg["d2h"],
+               "ms_per_step": round(main_leg["ms"] / args.steps, 5), "buffers": nbuf, "cuda_graph": graph,
+               "host_us_per_submit": round(main_leg["host_us"], 2),
+               "serial": {"value": gbs(serial["ms"]), "ms_per_step": round(serial["ms"] / args.steps, 5),
+                          "buffers": 1, "cuda_graph": False}}
 
     peak, peak_kind = measured_hbm_peak()
     achieved = dec_bytes / (dec_avg_max * 1e-3) / 1e9
@@ -439,6 +451,10 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=8.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
+    ap.add_argument("--e2e-buffers", type=int, default=2,
+                    help="host/device buffer pairs the end-to-end leg rotates (1 = no copy/compute overlap)")
+    ap.add_argument("--e2e-graph", type=int, default=1, choices=(0, 1),
+                    help="replay each buffer's kernels from a captured CUDA graph in the end-to-end leg")
     ap.add_argument("--pool-blocks", type=int, default=None,
                     help="override the pool size (profiling runs on a smaller device footprint)")
     ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",

@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
                 break;
             }
             finish_partition<T, D, G, NCW, NCW * 32>(a, mg_m, mg_l, mg_acc, info->s, info->kvh, info->part,
-                                                     (info->flags & kSplitUnit) != 0, threadIdx.x);
+                                                     (info->flags & kSplitUnit) != 0, first % NCW, threadIdx.x);
             if (!consumer_sync(group, nsync++, lane, abort_flag)) {
                 ok = false;
                 break;

@@ -181,9 +181,16 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeArgs a, i
 // unnormalised output, all relative to m) of one (sequence, kv head, partition)
 // and writes either the final output row (the sequence fits in one partition) or
 // the partition's state to the workspace.  Run by the NTHR consumer threads.
+//
+// Tile j of the unit (j = 0, 1, ...) was consumed by warp (rot + j) % NCW, rot being
+// where the unit started in the CTA's stage stream, which depends on the units the
+// CTA ran before.  The states are summed in tile-phase order (j mod NCW), not in
+// warp order, so the result is the same bits whichever CTA ran the unit and after
+// what: the decode is reproducible run to run under the dynamic work counter.
 template <typename T, int D, int G, int NCW, int NTHR>
 __device__ __forceinline__ void finish_partition(const DecodeArgs& a, const float* mg_m, const float* mg_l,
-                                                 const float* mg_acc, int s, int kvh, int part, bool split, int tid)
+                                                 const float* mg_acc, int s, int kvh, int part, bool split, int rot,
+                                                 int tid)
 {
     const int NP = a.num_partitions;
     for (int idx = tid; idx < G * D; idx += NTHR) {
@@ -195,7 +202,8 @@ __device__ __forceinline__ void finish_partition(const DecodeArgs& a, const floa
         float num = 0.f, den = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
-            for (int w = 0; w < NCW; ++w) {
+            for (int j = 0; j < NCW; ++j) {
+                const int w = (rot + j) % NCW;
                 const float mw = mg_m[w * G + g];
                 if (mw != -INFINITY) {
                     const float sc = exp2f(mw - M);

@@ -220,3 +220,156 @@ class CowBatch:
 def make_batch(wl, device="cuda", values=None, fill=float("nan"), partition_size=None):
     cls = CowBatch if isinstance(wl, W.CowWorkload) else DecodeBatch
     return cls(wl, device=device, values=values, fill=fill, partition_size=partition_size)
+
+
+# ---- stepping a batch whose inputs live in host memory
+
+STEP_INPUTS = ("q", "new_k", "new_v", "slot_mapping", "cow_pairs", "block_tables", "context_lens")
+
+
+def pack_layout(tensors, align=256):
+    """Byte layout of one step's inputs packed into a single buffer.
+
+    `tensors` maps a name to a tensor (or None / empty, which is left out).  Each
+    field starts on an `align`-byte boundary so that the typed views into the packed
+    buffer are aligned for every kernel that reads them.  Returns (fields, nbytes):
+    fields = [(name, offset, nbytes, dtype, shape)], nbytes = the end of the last
+    field, i.e. the size of the one copy that moves them all.
+    """
+    fields, off, end = [], 0, 0
+    for name, t in tensors.items():
+        if t is None or t.numel() == 0:
+            continue
+        n = t.numel() * t.element_size()
+        fields.append((name, off, n, t.dtype, tuple(t.shape)))
+        end = off + n
+        off = _round_up(end, align)
+    return fields, end
+
+
+class HostStepper:
+    """Decode steps fed from pinned host memory and read back into it.
+
+    Every step's inputs (q, the new K/V rows and their slots, copy-on-write pairs,
+    block tables, context lengths) sit packed in one pinned host buffer and cross to
+    the device in ONE copy; the step's output comes back in one copy.  `depth`
+    input/output buffer pairs rotate on three streams, so that the upload of step
+    k+1 and the read-back of step k-1 run on the copy engines while step k's
+    kernels run: each step's own upload still precedes its kernels and its
+    read-back follows them (events order them), and the host may refill a buffer
+    only after its upload has finished (`host_inputs` waits for that).
+
+    The kernels are the batch's: the copy-on-write copies, the slot-mapped append
+    and paged decode attention, all on the compute stream, so steps run in order.
+    With `graph=True` each buffer's kernel sequence is captured once as a CUDA graph
+    and replayed, which takes the per-launch host work off every step; the captured
+    launches have the batch's max_context_len and partition size fixed in them.
+    """
+
+    def __init__(self, batch, depth=2, stream=None, graph=False):
+        if depth < 1:
+            raise ValueError("depth must be >= 1")
+        self.batch = batch
+        self.depth = depth
+        dev = batch.device
+        self.stream = stream if stream is not None else torch.cuda.current_stream(dev)
+        self.h2d_stream = torch.cuda.Stream(dev)
+        self.d2h_stream = torch.cuda.Stream(dev)
+        self.fields, self.h2d_bytes = pack_layout({n: getattr(batch, n, None) for n in STEP_INPUTS})
+        self.d2h_bytes = batch.out.numel() * batch.out.element_size()
+        self.host_in, self.dev_in, self.host_out, self.dev_out = [], [], [], []
+        self.host_views, self.dev_views = [], []
+        for _ in range(depth):
+            h = torch.empty(max(self.h2d_bytes, 1), dtype=torch.uint8).pin_memory()
+            d = torch.empty(max(self.h2d_bytes, 1), dtype=torch.uint8, device=dev)
+            self.host_in.append(h)
+            self.dev_in.append(d)
+            self.host_views.append(self._views(h))
+            self.dev_views.append(self._views(d))
+            self.host_out.append(torch.empty(batch.out.shape, dtype=batch.out.dtype).pin_memory())
+            self.dev_out.append(torch.empty_like(batch.out))
+            for name, t in self.host_views[-1].items():
+                t.copy_(getattr(batch, name))
+        ev = lambda: [torch.cuda.Event() for _ in range(depth)]
+        self.uploaded, self.computed, self.downloaded = ev(), ev(), ev()
+        self.used = [False] * depth
+        self.k = 0
+        self.graphs = [None] * depth if graph else None
+
+    def _views(self, buf):
+        return {name: buf[off:off + n].view(dt).view(shape) for name, off, n, dt, shape in self.fields}
+
+    def host_inputs(self, slot):
+        """The pinned input views of buffer `slot`, once its last upload has finished."""
+        if self.used[slot]:
+            self.uploaded[slot].synchronize()
+        return self.host_views[slot]
+
+    def output(self, slot):
+        """The pinned output of buffer `slot`, once its last read-back has finished."""
+        self.downloaded[slot].synchronize()
+        return self.host_out[slot]
+
+    def submit(self, max_context_len=None):
+        """Queue one step on buffer k % depth; returns that buffer's index."""
+        b, i = self.batch, self.k % self.depth
+        mcl = b.max_context_len if max_context_len is None else int(max_context_len)
+        with torch.cuda.stream(self.h2d_stream):
+            if self.used[i]:
+                self.h2d_stream.wait_event(self.computed[i])
+            self.dev_in[i].copy_(self.host_in[i], non_blocking=True)
+            self.uploaded[i].record(self.h2d_stream)
+        s = self.stream
+        s.wait_event(self.uploaded[i])
+        if self.used[i]:
+            s.wait_event(self.downloaded[i])
+        if self.graphs is None:
+            self._kernels(i, mcl, s)
+        else:
+            if mcl != b.max_context_len:
+                raise ValueError("a captured step has max_context_len %d fixed in it" % b.max_context_len)
+            if self.graphs[i] is None:
+                self.graphs[i] = self._capture(i, mcl)
+            with torch.cuda.stream(s):
+                self.graphs[i].replay()
+        self.computed[i].record(s)
+        with torch.cuda.stream(self.d2h_stream):
+            self.d2h_stream.wait_event(self.computed[i])
+            self.host_out[i].copy_(self.dev_out[i], non_blocking=True)
+            self.downloaded[i].record(self.d2h_stream)
+        self.used[i] = True
+        self.k += 1
+        return i
+
+    def _kernels(self, i, mcl, s):
+        b, v = self.batch, self.dev_views[i]
+        if "cow_pairs" in v:
+            pa.pa_copy_blocks(b.k_cache, b.v_cache, v["cow_pairs"], stream=s)
+        pa.pa_reshape_and_cache(v["new_k"], v["new_v"], b.k_cache, b.v_cache, v["slot_mapping"], stream=s)
+        pa.pa_decode(self.dev_out[i], v["q"], b.k_cache, b.v_cache, v["block_tables"], v["context_lens"], mcl,
+                     b.wl.scale, b.partition_size, b.workspace_for(b.partition_size), stream=s)
+
+    def _capture(self, i, mcl):
+        b = self.batch
+        b.workspace_for(b.partition_size)             # sized before capture: nothing allocates inside
+        self.stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(b.device)
+        with torch.cuda.graph(g, stream=cap, capture_error_mode="relaxed"):
+            self._kernels(i, mcl, cap)
+        return g
+
+    def launches_per_step(self, max_context_len=None):
+        """Kernels one step launches: [copy-on-write copies], append, plan, decode, [merge]."""
+        b = self.batch
+        mcl = b.max_context_len if max_context_len is None else int(max_context_len)
+        wl = b.wl
+        part = pa.pa_decode_partition_size(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size,
+                                           mcl, b.partition_size)
+        return (1 if "cow_pairs" in self.dev_views[0] else 0) + 1 + 2 + (1 if mcl > part else 0)
+
+    def drain(self):
+        """Make the compute stream wait for every queued read-back."""
+        for i in range(self.depth):
+            if self.used[i]:
+                self.stream.wait_event(self.downloaded[i])

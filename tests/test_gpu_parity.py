@@ -118,6 +118,27 @@ def test_placement_does_not_change_a_single_bit(pa, runner):
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
 
 
+@pytest.mark.parametrize("wid,overrides", [(3, {}), (2, {}), (5, {}), (3, {"dtype": "f32", "num_seqs": 48})])
+def test_decode_is_reproducible_under_a_changing_schedule(pa, runner, wid, overrides):
+    """Units go to CTAs through a dynamic work counter, so which CTA runs a unit, and
+    after which others, changes from call to call.  The result must not: repeat the
+    decode while a matmul on another stream takes SMs away at different moments."""
+    wl = W.make_workload(wid, seed=1, **overrides)
+    batch = runner.DecodeBatch(wl, "cuda", values=W.decode_values(wl, "cuda"))
+    batch.append()
+    ref = batch.decode(out=torch.empty_like(batch.q)).clone()
+    side = torch.cuda.Stream()
+    a = torch.randn(4096, 4096, device="cuda", dtype=torch.bfloat16)
+    for k in range(6):
+        with torch.cuda.stream(side):
+            for _ in range(k):
+                a = (a @ a).clamp_(-1, 1)
+        out = batch.decode(out=torch.empty_like(batch.q))
+        torch.cuda.synchronize()
+        assert np.array_equal(bits(out), bits(ref)), "call %d differs" % k
+    _status_clean(pa)
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_zero_length_context_gives_zero_row(pa, dtype):
     dt = W.torch_dtype(dtype)

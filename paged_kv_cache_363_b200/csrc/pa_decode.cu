@@ -81,7 +81,7 @@ struct Persist {
     static constexpr int SLOT_BYTES = (QBYTES + MAX_PBLK * 4 + (int)sizeof(UnitInfo) + 127) / 128 * 128;
     static constexpr int THREADS = (NCW + 2) * 32;      // consumers, tile producer, unit producer
     static constexpr int MERGE_FLOATS = NCW * G * (D + 2);
-    static constexpr int NBAR_FIXED = 3 * UR + 1;
+    static constexpr int NBAR_FIXED = 3 * UR + 2;
     static constexpr int FIXED_BYTES = UR * SLOT_BYTES + MERGE_FLOATS * 4 + NCW * Cons::SCRATCH_FLOATS * 4 +
                                        NBAR_FIXED * 8 + 16 + 1024;
     // Stage i of the CTA's stream is consumed by warp i % NCW.  With NSTAGES a multiple
@@ -129,14 +129,6 @@ __device__ __forceinline__ void issue_tile(unsigned char* stage, const DecodeArg
     }
 }
 
-// Barrier among the consumer warps (an mbarrier, so the wait is bounded).
-__device__ __forceinline__ bool consumer_sync(uint64_t* bar, int n, int lane, volatile int* abort_flag)
-{
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar);
-    return mbar_wait_bounded(bar, n & 1, abort_flag);
-}
-
 template <class Cons, int BS>
 __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
     decode_persistent_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap tmap_k,
@@ -155,7 +147,8 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
     uint64_t* ufull = bars + 2 * NS;  // unit slot filled (q bytes)
     uint64_t* uempty = ufull + UR;    // unit slot released (consumers and tile producer)
     uint64_t* utab = uempty + UR;     // unit slot's block-table slice written (tile producer)
-    uint64_t* group = utab + UR;      // consumer-warp barrier
+    uint64_t* mg_full = utab + UR;    // every consumer warp's state of the unit is in the merge buffer
+    uint64_t* mg_free = mg_full + 1;  // the unit's finish has read the merge buffer
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + P::OFF_ABORT);
     float* mg_m = reinterpret_cast<float*>(smem + P::OFF_MERGE);
     float* mg_l = mg_m + NCW * G;
@@ -174,7 +167,8 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
             mbar_init(&uempty[u], 2);
             mbar_init(&utab[u], 1);
         }
-        mbar_init(group, NCW);
+        mbar_init(mg_full, NCW);
+        mbar_init(mg_free, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -304,9 +298,15 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
         }
     } else {
         // ---------------- consumers
+        // At a unit's end each warp puts its state in the merge buffer and moves on to
+        // the next unit without waiting.  The warp that consumed the unit's last tile
+        // (usually the last to get there) waits for the other states, merges them and
+        // writes the result, then frees the buffer and the unit slot.  A warp may write
+        // its state for unit k only after the finish of unit k-1 has freed the buffer,
+        // so arrivals on mg_full for unit k all belong to phase k, and one-bit parities
+        // on both barriers are never stale.
         Cons cons;
         cons.init(reinterpret_cast<float*>(smem + P::OFF_SCRATCH) + warp * Cons::SCRATCH_FLOATS, lane);
-        int nsync = 0;
         bool ok = true;
         for (int k = 0; ok; ++k) {
             if (!mbar_wait_bounded(&ufull[k % UR], (k / UR) & 1, abort_flag)) {
@@ -330,18 +330,27 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
                 if (lane == 0) mbar_arrive(&empty[st]);
             }
             if (!ok) break;
+            if (k > 0 && !mbar_wait_bounded(mg_free, (k - 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
             cons.end_unit(mg_m, mg_l, mg_acc, warp);
-            if (!consumer_sync(group, nsync++, lane, abort_flag)) {
-                ok = false;
-                break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(mg_full);
+            const int finisher = ((first + nt - 1) % NCW + NCW) % NCW;
+            if (warp == finisher) {
+                if (!mbar_wait_bounded(mg_full, k & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                finish_unit_warp<T, D, G, NCW>(a, mg_m, mg_l, mg_acc, info->s, info->kvh, info->part,
+                                               (info->flags & kSplitUnit) != 0, first % NCW, lane);
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(mg_free);
+                    mbar_arrive(&uempty[k % UR]);
+                }
             }
-            finish_partition<T, D, G, NCW, NCW * 32>(a, mg_m, mg_l, mg_acc, info->s, info->kvh, info->part,
-                                                     (info->flags & kSplitUnit) != 0, first % NCW, threadIdx.x);
-            if (!consumer_sync(group, nsync++, lane, abort_flag)) {
-                ok = false;
-                break;
-            }
-            if (threadIdx.x == 0) mbar_arrive(&uempty[k % UR]);
         }
         if (!ok) {
             if (lane == 0) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
@@ -468,7 +477,9 @@ cudaError_t launch_persistent(const DecodeArgs& a, cudaStream_t stream)
     DecodeArgs args = a;
     args.num_ctas = (int)grid;
 
-    decode_plan_kernel<<<1, 1024, 0, stream>>>(args, BS);
+    // one CTA; fewer threads for small batches keep its barriers short
+    const int plan_threads = a.num_seqs <= 256 ? 256 : (a.num_seqs <= 512 ? 512 : 1024);
+    decode_plan_kernel<<<1, plan_threads, 0, stream>>>(args, BS);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     e = launch_pdl(decode_persistent_kernel<Cons, BS>, dim3(grid), dim3(P::THREADS), (size_t)P::SMEM, stream, args,

@@ -180,48 +180,71 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeArgs a, i
 // Merges the NCW consumer warps' states (m: running max, l: softmax sum, acc:
 // unnormalised output, all relative to m) of one (sequence, kv head, partition)
 // and writes either the final output row (the sequence fits in one partition) or
-// the partition's state to the workspace.  Run by the NTHR consumer threads.
+// the partition's state to the workspace.  Run by one warp: a lane owns four
+// consecutive columns of one query head's row (float4 reads of the states).
 //
 // Tile j of the unit (j = 0, 1, ...) was consumed by warp (rot + j) % NCW, rot being
 // where the unit started in the CTA's stage stream, which depends on the units the
 // CTA ran before.  The states are summed in tile-phase order (j mod NCW), not in
 // warp order, so the result is the same bits whichever CTA ran the unit and after
 // what: the decode is reproducible run to run under the dynamic work counter.
-template <typename T, int D, int G, int NCW, int NTHR>
-__device__ __forceinline__ void finish_partition(const DecodeArgs& a, const float* mg_m, const float* mg_l,
+template <typename T, int D, int G, int NCW>
+__device__ __forceinline__ void finish_unit_warp(const DecodeArgs& a, const float* mg_m, const float* mg_l,
                                                  const float* mg_acc, int s, int kvh, int part, bool split, int rot,
-                                                 int tid)
+                                                 int lane)
 {
-    const int NP = a.num_partitions;
-    for (int idx = tid; idx < G * D; idx += NTHR) {
-        const int g = idx / D;
-        const int d = idx % D;
-        float M = -INFINITY;
+    constexpr int LPG = D / 4;     // lanes per head row
+    constexpr int GPP = 32 / LPG;  // head rows per pass
+    static_assert(D % 4 == 0 && 32 % LPG == 0, "a warp covers whole head rows");
+    const int sub = lane / LPG;
+    const int d0 = (lane % LPG) * 4;
 #pragma unroll
-        for (int w = 0; w < NCW; ++w) M = fmaxf(M, mg_m[w * G + g]);
-        float num = 0.f, den = 0.f;
-        if (M != -INFINITY) {
+    for (int g0 = 0; g0 < G; g0 += GPP) {
+        const int g = g0 + sub;
+        if (g < G) {
+            float M = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < NCW; ++j) {
-                const int w = (rot + j) % NCW;
-                const float mw = mg_m[w * G + g];
-                if (mw != -INFINITY) {
-                    const float sc = exp2f(mw - M);
-                    num = fmaf(sc, mg_acc[(w * G + g) * D + d], num);
-                    den = fmaf(sc, mg_l[w * G + g], den);
+            for (int w = 0; w < NCW; ++w) M = fmaxf(M, mg_m[w * G + g]);
+            float n0 = 0.f, n1 = 0.f, n2 = 0.f, n3 = 0.f, den = 0.f;
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int j = 0; j < NCW; ++j) {
+                    const int w = (rot + j) % NCW;
+                    const float mj = mg_m[w * G + g];
+                    if (mj != -INFINITY) {
+                        const float sc = exp2f(mj - M);
+                        const float4 v = *reinterpret_cast<const float4*>(mg_acc + (w * G + g) * D + d0);
+                        n0 = fmaf(sc, v.x, n0);
+                        n1 = fmaf(sc, v.y, n1);
+                        n2 = fmaf(sc, v.z, n2);
+                        n3 = fmaf(sc, v.w, n3);
+                        den = fmaf(sc, mg_l[w * G + g], den);
+                    }
                 }
             }
-        }
-        const int h = kvh * G + g;
-        if (!split) {
-            T* o = static_cast<T*>(a.out) + ((size_t)s * a.num_heads + h) * D;
-            o[d] = from_f32<T>(den > 0.f ? num / den : 0.f);
-        } else {
-            const size_t row = ((size_t)s * a.num_heads + h) * NP + part;
-            a.ws_acc[row * D + d] = num;
-            if (d == 0) {
-                a.ws_ml[row * 2] = M;
-                a.ws_ml[row * 2 + 1] = den;
+            const int h = kvh * G + g;
+            if (!split) {
+                T* o = static_cast<T*>(a.out) + ((size_t)s * a.num_heads + h) * D + d0;
+                const bool any = den > 0.f;
+                const float r0 = any ? n0 / den : 0.f, r1 = any ? n1 / den : 0.f;
+                const float r2 = any ? n2 / den : 0.f, r3 = any ? n3 / den : 0.f;
+                if constexpr (sizeof(T) == 4) {
+                    *reinterpret_cast<float4*>(o) = make_float4(r0, r1, r2, r3);
+                } else {
+                    const __nv_bfloat162 lo = __floats2bfloat162_rn(r0, r1);
+                    const __nv_bfloat162 hi = __floats2bfloat162_rn(r2, r3);
+                    uint2 pk;
+                    pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+                    pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+                    *reinterpret_cast<uint2*>(o) = pk;
+                }
+            } else {
+                const size_t row = ((size_t)s * a.num_heads + h) * a.num_partitions + part;
+                *reinterpret_cast<float4*>(a.ws_acc + row * D + d0) = make_float4(n0, n1, n2, n3);
+                if (d0 == 0) {
+                    a.ws_ml[row * 2] = M;
+                    a.ws_ml[row * 2 + 1] = den;
+                }
             }
         }
     }

@@ -289,6 +289,54 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ the CUDA path
 
+def companion_timing(batch, stream, reps=200, num_pairs=96):
+    """Latency and GB/s of the two companions alone: the step's slot-mapped append, and a
+    copy-on-write batch of `num_pairs` whole-block copies from blocks in use to free ones.
+    `us` is the median of per-call CUDA-event brackets; `us_back_to_back` the mean over
+    `reps` calls queued without gaps."""
+    import torch
+    from paged_kv_cache_363_b200 import pa
+
+    wl = batch.wl
+    elt = 4 if wl.dtype == "f32" else 2
+    used = np.unique(batch.block_tables.cpu().numpy())
+    used = used[used >= 0]
+    free = np.setdiff1d(np.arange(wl.num_blocks), used)
+    n = int(min(num_pairs, len(used), len(free)))
+    rng = np.random.default_rng(7)
+    pairs = np.stack([rng.choice(used, n, replace=False), rng.choice(free, n, replace=False)], 1).astype(np.int64)
+    pairs_d = torch.from_numpy(pairs).to(batch.device)
+    row = wl.num_kv_heads * wl.head_dim * elt
+    calls = {
+        "reshape_and_cache": (lambda: pa.pa_reshape_and_cache(batch.new_k, batch.new_v, batch.k_cache, batch.v_cache,
+                                                              batch.slot_mapping, stream=stream),
+                              batch.new_k.shape[0] * (2 * row * 2 + 8), {"tokens": int(batch.new_k.shape[0])}),
+        "copy_blocks": (lambda: pa.pa_copy_blocks(batch.k_cache, batch.v_cache, pairs_d, stream=stream),
+                        n * 2 * (row * wl.block_size) * 2 + 16 * n, {"pairs": n}),
+    }
+    out = {}
+    for name, (fn, nbytes, extra) in calls.items():
+        for _ in range(5):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in ev:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(reps):
+            fn()
+        t1.record(stream)
+        torch.cuda.synchronize(batch.device)
+        med = statistics.median(a.elapsed_time(b) for a, b in ev)
+        b2b = t0.elapsed_time(t1) / reps
+        out[name] = dict(extra, bytes=nbytes, us=round(med * 1e3, 3), gbs=round(nbytes / (med * 1e-3) / 1e9, 1),
+                         us_back_to_back=round(b2b * 1e3, 3), gbs_back_to_back=round(nbytes / (b2b * 1e-3) / 1e9, 1))
+    return out
+
+
 def e2e_leg(stepper, args, world, dev):
     """Device time of `args.steps` host-fed steps (upload, kernels, read-back), max over ranks."""
     import torch
@@ -407,6 +455,8 @@ def run_gpu(args):
                "serial": {"value": gbs(serial["ms"]), "ms_per_step": round(serial["ms"] / args.steps, 5),
                           "buffers": 1, "cuda_graph": False}}
 
+    companions = companion_timing(batch, stream) if not args.skip_e2e else None
+
     peak, peak_kind = measured_hbm_peak()
     achieved = dec_bytes / (dec_avg_max * 1e-3) / 1e9
     value = world * step_bytes * args.steps / (ms_max * 1e-3) / 1e9
@@ -422,7 +472,9 @@ def run_gpu(args):
                      "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
                      "traffic": profile_traffic("decode_persistent_kernel", wl.name),
-                     "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_us": round(dec_avg_max * 1e3, 3)},
+                     "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_us": round(dec_avg_max * 1e3, 3),
+                     "launch_us_p10_p50_p90": [round(float(np.percentile(dec_ms, q)) * 1e3, 3) for q in (10, 50, 90)]},
+        "companions": companions,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),

@@ -168,12 +168,35 @@ class ClockSampler:
                 "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
 
 
+L2_BYTES = 126e6
+
+
+def l2_note(batch, logical_bytes):
+    """How the timed steps stand to the 126 MB L2: the distinct K/V blocks a step reads."""
+    wl = batch.wl
+    elt = 4 if wl.dtype == "f32" else 2
+    used = np.unique(batch.block_tables.cpu().numpy())
+    unique = int((used >= 0).sum()) * wl.block_size * 2 * wl.num_kv_heads * wl.head_dim * elt
+    if unique >= L2_BYTES:
+        return "inputs larger than L2: %.0f MB of distinct KV per step (%.0f MB logical) vs 126 MB" % (
+            unique / 1e6, logical_bytes / 1e6)
+    return ("distinct KV %.0f MB per step fits the 126 MB L2 (shared blocks are re-read from L2); value counts "
+            "the %.0f MB of logical bytes" % (unique / 1e6, logical_bytes / 1e6))
+
+
 def workload_config(wl, partition, batch=None):
     cfg = {"workload": wl.name, "num_heads": wl.num_heads, "num_kv_heads": wl.num_kv_heads,
            "head_dim": wl.head_dim, "block_size": wl.block_size, "num_blocks": wl.num_blocks,
            "partition_size": partition, "seed": wl.seed}
     if isinstance(wl, W.CowWorkload):
         cfg.update(num_seqs=wl.num_seqs, prompts=wl.num_prompts, streams_per_prompt=wl.streams_per_prompt)
+    elif isinstance(wl, W.PrefixWorkload):
+        cfg.update(num_seqs=wl.num_seqs, prompts=wl.num_prompts, requests_per_prompt=wl.requests_per_prompt,
+                   context_tokens=int(np.sum(wl.context_lens)), max_context_len=int(np.max(wl.context_lens)))
+        if batch is not None:
+            cfg.update(cached_prompt_tokens=int(batch.cached_tokens.sum()), written_prompt_tokens=batch.written_tokens,
+                       unique_kv_mb=round(batch.unique_kv_bytes() / 1e6, 1),
+                       allocator_us_per_request=round(batch.alloc_us_per_request, 2))
     else:
         cfg.update(num_seqs=wl.num_seqs, context_tokens=int(np.sum(wl.context_lens)),
                    max_context_len=int(np.max(wl.context_lens)))
@@ -261,7 +284,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     wl = W.make_workload(W.NAME_TO_ID[args.workload], seed=args.seed)
-    if isinstance(wl, W.CowWorkload):
+    if not isinstance(wl, W.DecodeWorkload):
         print(json.dumps({"impl": "reference", "unavailable": "oracle leg covers the decode workloads only"}))
         return 0
     total = args.steps + args.warmup
@@ -391,6 +414,8 @@ def run_gpu(args):
         wl.partition_size = args.partition
     if isinstance(wl, W.CowWorkload):
         values = W.cow_values(wl, dev)
+    elif isinstance(wl, W.PrefixWorkload):
+        values = W.prefix_values(wl, dev)
     else:
         values = W.decode_values(wl, dev)
     batch = runner.make_batch(wl, dev, values=values)
@@ -464,8 +489,8 @@ def run_gpu(args):
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
-        "config": dict(workload_config(wl, part), l2="inputs larger than L2: %.0f MB of KV per step vs 126 MB"
-                       % (dec_bytes / 1e6), parallelism="replicas: one batch per GPU (dp%d)" % world),
+        "config": dict(workload_config(wl, part, batch), l2=l2_note(batch, dec_bytes),
+                       parallelism="replicas: one batch per GPU (dp%d)" % world),
         "seqs_per_s": round(world * wl.num_seqs * args.steps / (ms_max * 1e-3), 1),
         "pct_of_peak": round(100.0 * value / peak, 2),
         "roofline": {"bound": "hbm", "kernel": "pa_decode (plan kernel + persistent decode kernel)",
@@ -480,7 +505,7 @@ def run_gpu(args):
         "clocks": clk.summary(),
         "device_status": flags, "output_finite": out_ok,
     }
-    if world == 1 and not args.no_cpu_baseline and not isinstance(wl, W.CowWorkload):
+    if world == 1 and not args.no_cpu_baseline and isinstance(wl, W.DecodeWorkload):
         gbs, seqs_s, cores, sample, _ = oracle_leg(wl, args.cpu_budget, values)
         line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                                 "sample": sample}

@@ -199,11 +199,18 @@ PA_API pa_status pa_device_status(uint32_t* flags, void* stream);
 
 /*
  * Host block allocator with reference-counted copy-on-write ([INIT] sections 1
- * and 3, "Why Internal Fragmentation is Bounded"; [FSAH] sections 2 and 3).
+ * and 3, "Why Internal Fragmentation is Bounded"; [FSAH] sections 2 and 3) and a
+ * prefix cache ([FSAH] "Paper Methods": shared prefix caching in a radix tree).
  * It owns only host memory.  The free pool is a FIFO queue initialised from
  * free_order (a permutation of 0..num_blocks-1; NULL = ascending); blocks freed
  * later join its tail.  A handle is not thread-safe.  On every error the
  * allocator state is left unchanged.
+ *
+ * Prefix cache: prompts added with pa_alloc_add_seq_cached build a tree whose
+ * nodes are full blocks (edge = the block's B token ids, parent = the block before
+ * it).  An unreferenced cached block stays in the tree until a block is needed and
+ * the free queue is empty; then the one released longest ago among those with no
+ * cached children is evicted and reused.  Every call that takes blocks can evict.
  */
 typedef struct pa_allocator pa_allocator;
 
@@ -215,6 +222,8 @@ typedef struct {
     int64_t cow_copies;        /* copy-on-write copies made so far */
     int64_t tokens;            /* sum of the sequences' token counts */
     int64_t waste_tokens;      /* unused slots in the sequences' last blocks */
+    int64_t cached_blocks;     /* blocks in the prefix tree (referenced or not) */
+    int64_t cached_free;       /* unreferenced cached blocks (reusable by eviction) */
 } pa_alloc_stats_t;
 
 /* Returns NULL on bad arguments (see pa_last_error_string). */
@@ -225,6 +234,21 @@ PA_API void pa_alloc_destroy(pa_allocator* a);
  * each with reference count 1.  slots_out (nullable, num_tokens entries) receives
  * the slot of every token.  PA_ERR_INVALID if seq_id exists. */
 PA_API pa_status pa_alloc_add_seq(pa_allocator* a, int64_t seq_id, int num_tokens, int64_t* slots_out);
+
+/*
+ * New sequence of num_tokens tokens whose ids are token_ids[num_tokens] (HOST),
+ * sharing cached prompt blocks.  The leading full blocks whose token ids (and
+ * everything before them) match a cached prefix are reused (count + 1); the other
+ * full blocks are taken fresh and cached under their token ids; a partial last
+ * block is taken fresh and stays private.  *num_cached_out = tokens covered by the
+ * reused blocks (a multiple of B): their K/V are already in the cache, so the
+ * caller appends only tokens num_cached .. num_tokens-1 (pa_reshape_and_cache with
+ * those slots).  slots_out (nullable) receives the slot of every token.  A fresh
+ * cached block must be written before any later call can reuse it, i.e. before the
+ * decode of a sequence that shares it, in stream order.
+ */
+PA_API pa_status pa_alloc_add_seq_cached(pa_allocator* a, int64_t seq_id, const int32_t* token_ids, int num_tokens,
+                                         int64_t* slots_out, int* num_cached_out);
 
 /* child shares every block of parent (each reference count + 1) and its token count. */
 PA_API pa_status pa_alloc_fork(pa_allocator* a, int64_t parent_id, int64_t child_id);
@@ -248,7 +272,8 @@ PA_API pa_status pa_alloc_append_slot(pa_allocator* a, int64_t seq_id, int64_t* 
 PA_API pa_status pa_alloc_append_slots(pa_allocator* a, const int64_t* seq_ids, int n, int64_t* slots_out,
                                 int64_t* cow_pairs_out, int* num_cow_out);
 
-/* Drops one reference to each block of seq_id; blocks reaching zero rejoin the free pool. */
+/* Drops one reference to each block of seq_id; blocks reaching zero rejoin the free
+ * pool, or stay in the prefix tree as unreferenced cached blocks. */
 PA_API pa_status pa_alloc_free_seq(pa_allocator* a, int64_t seq_id);
 
 /* Copies seq_id's block table into out[capacity]; *n_out = its length.
@@ -261,7 +286,8 @@ PA_API pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq
                                 int max_blocks, int32_t fill, int32_t* context_lens_out);
 
 PA_API int pa_alloc_ref_count(const pa_allocator* a, int32_t block);   /* -1 if out of range */
-PA_API int pa_alloc_num_free(const pa_allocator* a);
+PA_API int pa_alloc_num_free(const pa_allocator* a);          /* blocks in the free queue */
+PA_API int pa_alloc_num_cached_free(const pa_allocator* a);   /* unreferenced cached blocks */
 PA_API int pa_alloc_num_tokens(const pa_allocator* a, int64_t seq_id); /* -1 if unknown */
 PA_API pa_status pa_alloc_stats(const pa_allocator* a, pa_alloc_stats_t* out);
 

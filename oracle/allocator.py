@@ -15,16 +15,29 @@ What it follows, by page and section:
       later writes go to the private block.
   "PagedAttention Paper Breakdown" (fullstackaihub.com), section 2 Address
     Translation Formula (slot = T[floor(i/B)]*B + i mod B) and section 3
-    (a copy-on-write trigger leaves the other streams' tables untouched).
+    (a copy-on-write trigger leaves the other streams' tables untouched);
+    "Paper Methods": shared prefix caching kept in a radix tree.
 
 Readings where the pages are silent: the free pool is a FIFO queue seeded by a
 given order (the "random placement"), freed blocks join its tail in table order;
 a forked child copies the parent's table and token count, every shared block's
 count going up by one; copy-on-write happens only on a write into a shared,
 partially filled last block; running out of blocks raises OutOfBlocks and
-changes nothing.
+changes nothing (a batch of appends included).
+
+Prefix cache (the pages name the radix tree only).  The tree is read at block
+granularity: each node is one full physical block, labelled by the B token ids it
+holds and hanging under the node of the block before it, so the path from the root
+spells the token prefix.  Adding a prompt by its token ids reuses the blocks along
+the longest matching path (count + 1), takes fresh blocks for its other full blocks
+and hangs them under that path, and gives a partial last block a fresh private
+block.  A cached block whose count reaches zero stays in the tree, unreferenced.
+Blocks come from the free queue first; when it is empty, the unreferenced cached
+block released earliest among those with no child in the tree is removed from the
+tree and reused.
 """
-from collections import deque
+import copy
+from collections import OrderedDict, deque
 
 
 class OutOfBlocks(RuntimeError):
@@ -45,17 +58,46 @@ class OracleAllocator:
         self.tables = {}
         self.ntokens = {}
         self.cow_count = 0
+        self.tree = {}            # (parent block or -1, token ids of the block) -> block
+        self.key_of = {}          # cached block -> its key in the tree
+        self.nchildren = {}       # cached block -> number of cached children
+        self.unreferenced = OrderedDict()   # cached blocks with count 0, earliest release first
 
     # [fullstackaihub] section 2: PhysicalAddr = T[floor(i/B)]*B + (i mod B)
     def slot(self, seq_id, i):
         table = self.tables[seq_id]
         return table[i // self.B] * self.B + i % self.B
 
+    def available(self):
+        return len(self.free) + len(self.unreferenced)
+
     def _take(self):
-        blk = self.free.popleft()
+        if self.free:
+            blk = self.free.popleft()
+        else:
+            blk = next(b for b in self.unreferenced if self.nchildren[b] == 0)
+            key = self.key_of.pop(blk)
+            del self.tree[key]
+            del self.nchildren[blk]
+            del self.unreferenced[blk]
+            if key[0] >= 0:
+                self.nchildren[key[0]] -= 1
         assert self.ref[blk] == 0
         self.ref[blk] = 1
         return blk
+
+    def _hold(self, blk):
+        if self.ref[blk] == 0:
+            del self.unreferenced[blk]
+        self.ref[blk] += 1
+
+    def _release(self, blk):
+        self.ref[blk] -= 1
+        if self.ref[blk] == 0:
+            if blk in self.key_of:
+                self.unreferenced[blk] = None
+            else:
+                self.free.append(blk)
 
     def add_seq(self, seq_id, num_tokens):
         """New sequence holding num_tokens tokens; returns their slots."""
@@ -64,11 +106,49 @@ class OracleAllocator:
         if num_tokens < 0:
             raise ValueError("negative token count")
         need = -(-num_tokens // self.B)
-        if need > len(self.free):
+        if need > self.available():
             raise OutOfBlocks()
         self.tables[seq_id] = [self._take() for _ in range(need)]
         self.ntokens[seq_id] = num_tokens
         return [self.slot(seq_id, i) for i in range(num_tokens)]
+
+    def add_seq_cached(self, seq_id, token_ids):
+        """New sequence with these token ids, reusing the cached blocks of its longest
+        cached full-block prefix.  Returns (slots, number of tokens already cached)."""
+        if seq_id in self.tables:
+            raise ValueError("sequence exists")
+        tokens = [int(t) for t in token_ids]
+        n, B = len(tokens), self.B
+        full = [tuple(tokens[j * B:(j + 1) * B]) for j in range(n // B)]
+        hits, parent = [], -1
+        for blk_tokens in full:
+            blk = self.tree.get((parent, blk_tokens))
+            if blk is None:
+                break
+            hits.append(blk)
+            parent = blk
+        need = len(full) - len(hits) + (1 if n % B else 0)
+        if need > self.available() - sum(1 for b in hits if self.ref[b] == 0):
+            raise OutOfBlocks()
+        table = []
+        for blk in hits:
+            self._hold(blk)
+            table.append(blk)
+        for blk_tokens in full[len(hits):]:
+            blk = self._take()
+            key = (parent, blk_tokens)
+            self.tree[key] = blk
+            self.key_of[blk] = key
+            self.nchildren[blk] = 0
+            if parent >= 0:
+                self.nchildren[parent] += 1
+            table.append(blk)
+            parent = blk
+        if n % B:
+            table.append(self._take())
+        self.tables[seq_id] = table
+        self.ntokens[seq_id] = n
+        return [self.slot(seq_id, i) for i in range(n)], len(hits) * B
 
     def fork(self, parent, child):
         """Child shares every block of the parent (each count + 1)."""
@@ -77,7 +157,7 @@ class OracleAllocator:
         self.tables[child] = list(self.tables[parent])
         self.ntokens[child] = self.ntokens[parent]
         for blk in self.tables[child]:
-            self.ref[blk] += 1
+            self._hold(blk)
 
     def append_slot(self, seq_id):
         """Slot for one new token; returns (slot, (src, dst) or None)."""
@@ -88,30 +168,36 @@ class OracleAllocator:
         cow = None
         if i % self.B == 0:
             # the last block is full (or there is none): take a fresh block
-            if not self.free:
+            if not self.available():
                 raise OutOfBlocks()
             table.append(self._take())
         else:
             last = table[-1]
             if self.ref[last] > 1:
                 # write into a shared block: copy-on-write
-                if not self.free:
+                if not self.available():
                     raise OutOfBlocks()
                 dst = self._take()
-                self.ref[last] -= 1
+                self._release(last)
                 table[-1] = dst
                 cow = (last, dst)
                 self.cow_count += 1
         self.ntokens[seq_id] = i + 1
         return self.slot(seq_id, i), cow
 
+    def append_slots(self, seq_ids):
+        """One append per listed sequence in order, all or nothing: on OutOfBlocks
+        (or an unknown sequence) the allocator is left as it was."""
+        trial = copy.deepcopy(self)
+        res = [trial.append_slot(s) for s in seq_ids]
+        self.__dict__.update(trial.__dict__)
+        return res
+
     def free_seq(self, seq_id):
         if seq_id not in self.tables:
             raise ValueError("unknown sequence")
         for blk in self.tables.pop(seq_id):
-            self.ref[blk] -= 1
-            if self.ref[blk] == 0:
-                self.free.append(blk)
+            self._release(blk)
         del self.ntokens[seq_id]
 
     def block_table(self, seq_id):
@@ -119,6 +205,9 @@ class OracleAllocator:
 
     def num_free(self):
         return len(self.free)
+
+    def num_cached_free(self):
+        return len(self.unreferenced)
 
     def waste_tokens(self, seq_id):
         """Unused slots in the sequence's table (only its last block can be partial)."""

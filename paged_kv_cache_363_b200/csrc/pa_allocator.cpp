@@ -1,4 +1,4 @@
-// Host block allocator with reference-counted copy-on-write.
+// Host block allocator with reference-counted copy-on-write and a prefix cache.
 //
 // Follows, by page and section:
 //  "PagedAttention and vLLM Architecture" (initnode.dev): section 1, a fixed pool
@@ -11,16 +11,28 @@
 //  the writer's table.
 //  "PagedAttention Paper Breakdown" (fullstackaihub.com): section 2, the slot of
 //  token i is T[floor(i/B)]*B + (i mod B); section 3, the other streams keep the
-//  shared blocks untouched.
+//  shared blocks untouched; "Paper Methods", shared prefix caching in a radix tree.
 //
 // Where the pages are silent: the free pool is a FIFO queue (initial order given
 // by the caller, freed blocks appended in table order); a fork copies the parent's
 // table and token count; a copy happens only for a write into a shared, partially
 // filled last block (full shared blocks are never written); every failing call
 // leaves the state as it was.
+//
+// Prefix cache (the pages name a radix tree and nothing more).  The tree is kept at
+// block granularity: a node is a full physical block, its edge the B token ids it
+// holds, its parent the block before it, so a node stands for the whole token
+// prefix that ends with it.  A prompt added with its token ids walks the tree and
+// reuses the blocks of its longest cached full-block prefix (their counts go up);
+// its remaining full blocks are taken fresh and become new nodes; a partial last
+// block stays private (it will be written).  A cached block whose count drops to
+// zero is kept, unreferenced, for later prompts.  A block is taken from the free
+// queue first; when that is empty, the unreferenced cached block released longest
+// ago that has no cached children (a leaf) is evicted from the tree and reused.
 #include <cstdint>
 #include <cstring>
 #include <deque>
+#include <map>
 #include <new>
 #include <string>
 #include <unordered_map>
@@ -44,88 +56,124 @@ struct pa_allocator {
     std::unordered_map<int64_t, Seq> seqs;
     int64_t cow_copies = 0;
 
+    // prefix tree: key = (parent block or -1, the block's B token ids) -> block
+    std::map<std::vector<int32_t>, int32_t> tree;
+    std::vector<std::vector<int32_t>> node_key;  // per block: its key (empty = not in the tree)
+    std::vector<int32_t> nchild;                 // per block: cached children
+    std::map<uint64_t, int32_t> lru;             // unreferenced cached blocks by release stamp
+    std::vector<uint64_t> stamp;                 // per block: its key in lru
+    uint64_t clock = 0;
+
+    bool cached(int32_t b) const { return !node_key[(size_t)b].empty(); }
+    int64_t available() const { return (int64_t)free_q.size() + (int64_t)lru.size(); }
+
     int64_t slot_of(const Seq& q, int64_t i) const
     {
         return (int64_t)q.table[(size_t)(i / block_size)] * block_size + i % block_size;
     }
 
+    void evict(int32_t b)
+    {
+        const std::vector<int32_t>& k = node_key[(size_t)b];
+        if (k[0] >= 0) nchild[(size_t)k[0]] -= 1;
+        tree.erase(k);
+        node_key[(size_t)b].clear();
+        lru.erase(stamp[(size_t)b]);
+    }
+
+    // A block with count 1: the free queue's head, else the oldest unreferenced cached
+    // leaf.  Callers check available() first, so there always is one.
     int32_t take()
     {
-        const int32_t b = free_q.front();
-        free_q.pop_front();
+        int32_t b;
+        if (!free_q.empty()) {
+            b = free_q.front();
+            free_q.pop_front();
+        } else {
+            b = -1;
+            for (const auto& e : lru)
+                if (nchild[(size_t)e.second] == 0) {
+                    b = e.second;
+                    break;
+                }
+            evict(b);
+        }
         ref[(size_t)b] = 1;
         return b;
     }
 
-    void give_back_front(int32_t b)
+    void add_ref(int32_t b)
     {
-        ref[(size_t)b] = 0;
-        free_q.push_front(b);
+        if (ref[(size_t)b]++ == 0) lru.erase(stamp[(size_t)b]);
     }
 
-    // Undo record of one append, so a failing batch can be rolled back exactly.
-    struct Undo {
-        int64_t seq;
-        int32_t fresh;     // block appended to the table (or -1)
-        int32_t cow_src;   // block replaced by copy-on-write (or -1)
-        int32_t cow_dst;
-    };
-
-    pa_status append(int64_t seq_id, int64_t* slot, int32_t* src, int32_t* dst, Undo* undo)
+    void drop_ref(int32_t b)
     {
-        auto it = seqs.find(seq_id);
-        if (it == seqs.end()) {
-            pa::set_error("pa_alloc_append_slot: unknown sequence " + std::to_string(seq_id));
-            return PA_ERR_INVALID;
+        if (--ref[(size_t)b] > 0) return;
+        if (cached(b)) {
+            stamp[(size_t)b] = clock++;
+            lru.emplace(stamp[(size_t)b], b);
+        } else {
+            free_q.push_back(b);
         }
-        Seq& q = it->second;
+    }
+
+    // Blocks that appends of seq_ids[0..n) in order would take (fresh or copy-on-write),
+    // without changing anything; -1 if a sequence is unknown.
+    int64_t blocks_for_appends(const int64_t* seq_ids, int n) const
+    {
+        std::unordered_map<int64_t, std::pair<int64_t, int32_t>> st;  // seq -> (tokens, last block or -1)
+        std::unordered_map<int32_t, int32_t> dref;                    // reference count changes
+        int64_t need = 0;
+        for (int k = 0; k < n; ++k) {
+            auto it = st.find(seq_ids[k]);
+            if (it == st.end()) {
+                auto q = seqs.find(seq_ids[k]);
+                if (q == seqs.end()) return -1;
+                it = st.emplace(seq_ids[k], std::make_pair(q->second.tokens,
+                                                           q->second.table.empty() ? -1 : q->second.table.back()))
+                         .first;
+            }
+            auto& [tokens, last] = it->second;
+            if (tokens % block_size == 0) {
+                need += 1;
+                last = -1;  // a private fresh block
+            } else if (last >= 0) {
+                auto d = dref.find(last);
+                const int32_t r = ref[(size_t)last] + (d == dref.end() ? 0 : d->second);
+                if (r > 1) {
+                    need += 1;
+                    dref[last] -= 1;
+                    last = -1;  // a private copy
+                }
+            }
+            tokens += 1;
+        }
+        return need;
+    }
+
+    // One append; the caller has checked that the blocks it may take are available.
+    int64_t append(int64_t seq_id, int32_t* src, int32_t* dst)
+    {
+        Seq& q = seqs.find(seq_id)->second;
         const int64_t i = q.tokens;
-        Undo u{seq_id, -1, -1, -1};
         *src = -1;
         *dst = -1;
         if (i % block_size == 0) {
-            if (free_q.empty()) {
-                pa::set_error("pa_alloc_append_slot: out of blocks");
-                return PA_ERR_OOM;
-            }
-            u.fresh = take();
-            q.table.push_back(u.fresh);
+            q.table.push_back(take());
         } else {
             const int32_t last = q.table.back();
             if (ref[(size_t)last] > 1) {
-                if (free_q.empty()) {
-                    pa::set_error("pa_alloc_append_slot: out of blocks (copy-on-write)");
-                    return PA_ERR_OOM;
-                }
                 const int32_t d = take();
-                ref[(size_t)last] -= 1;
+                drop_ref(last);
                 q.table.back() = d;
-                u.cow_src = last;
-                u.cow_dst = d;
                 *src = last;
                 *dst = d;
                 cow_copies += 1;
             }
         }
         q.tokens = i + 1;
-        *slot = slot_of(q, i);
-        if (undo) *undo = u;
-        return PA_OK;
-    }
-
-    void rollback(const Undo& u)
-    {
-        Seq& q = seqs[u.seq];
-        q.tokens -= 1;
-        if (u.fresh >= 0) {
-            q.table.pop_back();
-            give_back_front(u.fresh);
-        } else if (u.cow_dst >= 0) {
-            q.table.back() = u.cow_src;
-            ref[(size_t)u.cow_src] += 1;
-            give_back_front(u.cow_dst);
-            cow_copies -= 1;
-        }
+        return slot_of(q, i);
     }
 };
 
@@ -145,6 +193,9 @@ pa_allocator* pa_alloc_create(int num_blocks, int block_size, const int32_t* fre
     a->num_blocks = num_blocks;
     a->block_size = block_size;
     a->ref.assign((size_t)num_blocks, 0);
+    a->node_key.assign((size_t)num_blocks, std::vector<int32_t>());
+    a->nchild.assign((size_t)num_blocks, 0);
+    a->stamp.assign((size_t)num_blocks, 0);
     if (free_order) {
         std::vector<char> seen((size_t)num_blocks, 0);
         for (int i = 0; i < num_blocks; ++i) {
@@ -176,7 +227,7 @@ pa_status pa_alloc_add_seq(pa_allocator* a, int64_t seq_id, int num_tokens, int6
         return PA_ERR_INVALID;
     }
     const int64_t need = ((int64_t)num_tokens + a->block_size - 1) / a->block_size;
-    if (need > (int64_t)a->free_q.size()) {
+    if (need > a->available()) {
         pa::set_error("pa_alloc_add_seq: out of blocks");
         return PA_ERR_OOM;
     }
@@ -199,8 +250,65 @@ pa_status pa_alloc_fork(pa_allocator* a, int64_t parent_id, int64_t child_id)
         return PA_ERR_INVALID;
     }
     pa_allocator::Seq child = it->second;
-    for (int32_t b : child.table) a->ref[(size_t)b] += 1;
+    for (int32_t b : child.table) a->add_ref(b);
     a->seqs.emplace(child_id, std::move(child));
+    return PA_OK;
+}
+
+pa_status pa_alloc_add_seq_cached(pa_allocator* a, int64_t seq_id, const int32_t* token_ids, int num_tokens,
+                                  int64_t* slots_out, int* num_cached_out)
+{
+    if (!a || num_tokens < 0 || (num_tokens > 0 && !token_ids) || !num_cached_out) {
+        pa::set_error("pa_alloc_add_seq_cached: bad argument");
+        return PA_ERR_INVALID;
+    }
+    if (a->seqs.count(seq_id)) {
+        pa::set_error("pa_alloc_add_seq_cached: sequence " + std::to_string(seq_id) + " exists");
+        return PA_ERR_INVALID;
+    }
+    const int B = a->block_size;
+    const int nfull = num_tokens / B;
+    // longest cached prefix of full blocks
+    std::vector<int32_t> key((size_t)B + 1);
+    std::vector<int32_t> hits;
+    int32_t parent = -1;
+    int64_t hits_unreferenced = 0;
+    for (int j = 0; j < nfull; ++j) {
+        key[0] = parent;
+        std::memcpy(key.data() + 1, token_ids + (size_t)j * B, (size_t)B * sizeof(int32_t));
+        auto it = a->tree.find(key);
+        if (it == a->tree.end()) break;
+        hits.push_back(it->second);
+        hits_unreferenced += a->ref[(size_t)it->second] == 0 ? 1 : 0;
+        parent = it->second;
+    }
+    const int64_t need = (int64_t)(nfull - (int)hits.size()) + (num_tokens % B ? 1 : 0);
+    if (need > a->available() - hits_unreferenced) {
+        pa::set_error("pa_alloc_add_seq_cached: out of blocks");
+        return PA_ERR_OOM;
+    }
+    pa_allocator::Seq q;
+    q.table.reserve((size_t)(hits.size() + need));
+    for (int32_t b : hits) {
+        a->add_ref(b);
+        q.table.push_back(b);
+    }
+    for (int j = (int)hits.size(); j < nfull; ++j) {
+        const int32_t b = a->take();
+        key[0] = parent;
+        std::memcpy(key.data() + 1, token_ids + (size_t)j * B, (size_t)B * sizeof(int32_t));
+        a->tree.emplace(key, b);
+        a->node_key[(size_t)b] = key;
+        if (parent >= 0) a->nchild[(size_t)parent] += 1;
+        q.table.push_back(b);
+        parent = b;
+    }
+    if (num_tokens % B) q.table.push_back(a->take());
+    q.tokens = num_tokens;
+    if (slots_out)
+        for (int64_t i = 0; i < num_tokens; ++i) slots_out[i] = a->slot_of(q, i);
+    *num_cached_out = (int)hits.size() * B;
+    a->seqs.emplace(seq_id, std::move(q));
     return PA_OK;
 }
 
@@ -211,9 +319,17 @@ pa_status pa_alloc_append_slot(pa_allocator* a, int64_t seq_id, int64_t* slot_ou
         pa::set_error("pa_alloc_append_slot: bad argument");
         return PA_ERR_INVALID;
     }
+    const int64_t need = a->blocks_for_appends(&seq_id, 1);
+    if (need < 0) {
+        pa::set_error("pa_alloc_append_slot: unknown sequence " + std::to_string(seq_id));
+        return PA_ERR_INVALID;
+    }
+    if (need > a->available()) {
+        pa::set_error("pa_alloc_append_slot: out of blocks");
+        return PA_ERR_OOM;
+    }
     int32_t src, dst;
-    const pa_status st = a->append(seq_id, slot_out, &src, &dst, nullptr);
-    if (st != PA_OK) return st;
+    *slot_out = a->append(seq_id, &src, &dst);
     if (cow_src_out) *cow_src_out = src;
     if (cow_dst_out) *cow_dst_out = dst;
     return PA_OK;
@@ -226,15 +342,24 @@ pa_status pa_alloc_append_slots(pa_allocator* a, const int64_t* seq_ids, int n, 
         pa::set_error("pa_alloc_append_slots: bad argument");
         return PA_ERR_INVALID;
     }
-    std::vector<pa_allocator::Undo> log((size_t)n);
+    // all or nothing: count the blocks the whole batch takes before changing anything
+    const int64_t need = a->blocks_for_appends(seq_ids, n);
+    if (need < 0) {
+        for (int k = 0; k < n; ++k)
+            if (!a->seqs.count(seq_ids[k])) {
+                pa::set_error("pa_alloc_append_slot: unknown sequence " + std::to_string(seq_ids[k]));
+                break;
+            }
+        return PA_ERR_INVALID;
+    }
+    if (need > a->available()) {
+        pa::set_error("pa_alloc_append_slots: out of blocks");
+        return PA_ERR_OOM;
+    }
     int ncow = 0;
     for (int k = 0; k < n; ++k) {
         int32_t src, dst;
-        const pa_status st = a->append(seq_ids[k], &slots_out[k], &src, &dst, &log[(size_t)k]);
-        if (st != PA_OK) {
-            for (int u = k - 1; u >= 0; --u) a->rollback(log[(size_t)u]);
-            return st;
-        }
+        slots_out[k] = a->append(seq_ids[k], &src, &dst);
         if (src >= 0) {
             cow_pairs_out[2 * ncow] = src;
             cow_pairs_out[2 * ncow + 1] = dst;
@@ -253,10 +378,7 @@ pa_status pa_alloc_free_seq(pa_allocator* a, int64_t seq_id)
         pa::set_error("pa_alloc_free_seq: unknown sequence " + std::to_string(seq_id));
         return PA_ERR_INVALID;
     }
-    for (int32_t b : it->second.table) {
-        a->ref[(size_t)b] -= 1;
-        if (a->ref[(size_t)b] == 0) a->free_q.push_back(b);
-    }
+    for (int32_t b : it->second.table) a->drop_ref(b);
     a->seqs.erase(it);
     return PA_OK;
 }
@@ -314,6 +436,8 @@ int pa_alloc_ref_count(const pa_allocator* a, int32_t block)
 
 int pa_alloc_num_free(const pa_allocator* a) { return a ? (int)a->free_q.size() : -1; }
 
+int pa_alloc_num_cached_free(const pa_allocator* a) { return a ? (int)a->lru.size() : -1; }
+
 int pa_alloc_num_tokens(const pa_allocator* a, int64_t seq_id)
 {
     if (!a) return -1;
@@ -330,6 +454,8 @@ pa_status pa_alloc_stats(const pa_allocator* a, pa_alloc_stats_t* out)
     s.num_seqs = (int64_t)a->seqs.size();
     for (int32_t r : a->ref) s.shared_blocks += r > 1 ? 1 : 0;
     s.cow_copies = a->cow_copies;
+    s.cached_blocks = (int64_t)a->tree.size();
+    s.cached_free = (int64_t)a->lru.size();
     for (const auto& kv : a->seqs) {
         s.tokens += kv.second.tokens;
         s.waste_tokens += (int64_t)kv.second.table.size() * a->block_size - kv.second.tokens;

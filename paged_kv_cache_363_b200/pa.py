@@ -28,7 +28,7 @@ _u32 = ctypes.c_uint32
 
 class pa_alloc_stats_t(ctypes.Structure):
     _fields_ = [(n, _i64) for n in ("num_blocks", "num_free", "num_seqs", "shared_blocks", "cow_copies",
-                                   "tokens", "waste_tokens")]
+                                   "tokens", "waste_tokens", "cached_blocks", "cached_free")]
 
 
 # (name, restype, argtypes) of every symbol declared in include/pa.h
@@ -43,6 +43,7 @@ SIGNATURES = [
     ("pa_alloc_create", _vp, [_int, _int, _vp]),
     ("pa_alloc_destroy", None, [_vp]),
     ("pa_alloc_add_seq", _int, [_vp, _i64, _int, _vp]),
+    ("pa_alloc_add_seq_cached", _int, [_vp, _i64, _vp, _int, _vp, ctypes.POINTER(_int)]),
     ("pa_alloc_fork", _int, [_vp, _i64, _i64]),
     ("pa_alloc_append_slot", _int, [_vp, _i64, ctypes.POINTER(_i64), ctypes.POINTER(_i32), ctypes.POINTER(_i32)]),
     ("pa_alloc_append_slots", _int, [_vp, _vp, _int, _vp, _vp, ctypes.POINTER(_int)]),
@@ -51,6 +52,7 @@ SIGNATURES = [
     ("pa_alloc_block_tables", _int, [_vp, _vp, _int, _vp, _int, _i32, _vp]),
     ("pa_alloc_ref_count", _int, [_vp, _i32]),
     ("pa_alloc_num_free", _int, [_vp]),
+    ("pa_alloc_num_cached_free", _int, [_vp]),
     ("pa_alloc_num_tokens", _int, [_vp, _i64]),
     ("pa_alloc_stats", _int, [_vp, ctypes.POINTER(pa_alloc_stats_t)]),
     ("pa_last_error_string", ctypes.c_char_p, []),
@@ -244,6 +246,17 @@ class Allocator:
         _check(lib.pa_alloc_add_seq(self._h, int(seq_id), int(num_tokens), _np_ptr(slots)), "pa_alloc_add_seq")
         return slots[:int(num_tokens)]
 
+    def add_seq_cached(self, seq_id, token_ids):
+        """New sequence with these token ids, reusing cached prompt blocks.
+        Returns (slots of all tokens, number of leading tokens already cached)."""
+        ids = np.ascontiguousarray(token_ids, dtype=np.int32)
+        n = ids.shape[0]
+        slots = np.empty(max(1, n), np.int64)
+        ncached = _int(0)
+        _check(lib.pa_alloc_add_seq_cached(self._h, int(seq_id), _np_ptr(ids) if n else None, n, _np_ptr(slots),
+                                           ctypes.byref(ncached)), "pa_alloc_add_seq_cached")
+        return slots[:n], int(ncached.value)
+
     def fork(self, parent_id, child_id):
         _check(lib.pa_alloc_fork(self._h, int(parent_id), int(child_id)), "pa_alloc_fork")
 
@@ -287,6 +300,9 @@ class Allocator:
 
     def num_free(self):
         return int(lib.pa_alloc_num_free(self._h))
+
+    def num_cached_free(self):
+        return int(lib.pa_alloc_num_cached_free(self._h))
 
     def num_tokens(self, seq_id):
         return int(lib.pa_alloc_num_tokens(self._h, int(seq_id)))

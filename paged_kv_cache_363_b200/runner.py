@@ -13,6 +13,7 @@ copy-on-write of the shared partial last blocks.
 The torch calls here only allocate memory, move bytes and index tensors.
 """
 import math
+import time
 
 import numpy as np
 import torch
@@ -217,8 +218,98 @@ class CowBatch:
         return wl.num_seqs * (2 * wl.num_kv_heads * wl.head_dim * 2 * 2 + 8)
 
 
+class PrefixBatch:
+    """Requests sharing system prompts through the allocator's prefix cache.
+
+    Each request's prompt (all its tokens but the last) is added by token ids; only
+    the tokens past the cached full-block prefix are written into the pools, so a
+    stem's full blocks are written once and read by every request that shares it.
+    The decode step appends each request's last token and runs decode attention.
+    """
+
+    def __init__(self, wl, device="cuda", values=None, fill=float("nan"), partition_size=None):
+        self.wl = wl
+        self.device = torch.device(device)
+        S, Hq, Hkv, D, B, NB = (wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size,
+                                wl.num_blocks)
+        dt = W.torch_dtype(wl.dtype)
+        if values is None:
+            values = W.prefix_values(wl, self.device)
+        q, sk, sv, soff, xk, xv, xoff = values
+        self.k_cache = torch.full((NB, Hkv, B, D), fill, dtype=dt, device=self.device)
+        self.v_cache = torch.full((NB, Hkv, B, D), fill, dtype=dt, device=self.device)
+        self.alloc = pa.Allocator(NB, B, wl.free_order)
+        self.cached_tokens = np.zeros(S, np.int64)
+        write = {0: ([], []), 1: ([], [])}          # source -> (rows, slots)
+        prompts = [wl.tokens(r)[:-1] for r in range(S)]
+        t0 = time.perf_counter()
+        placed = [self.alloc.add_seq_cached(r, prompts[r]) for r in range(S)]
+        self.alloc_us_per_request = 1e6 * (time.perf_counter() - t0) / max(1, S)
+        for r in range(S):
+            slots, nc = placed[r]
+            self.cached_tokens[r] = nc
+            rows = W.prefix_logical_rows(wl, r, soff, xoff)[:-1]
+            for (src, row), slot in zip(rows[nc:], slots[nc:]):
+                write[src][0].append(row)
+                write[src][1].append(int(slot))
+        for src, (kk, vv) in ((0, (sk, sv)), (1, (xk, xv))):
+            rows, slots = write[src]
+            if rows:
+                idx = torch.tensor(rows, dtype=torch.int64, device=kk.device)
+                pa.pa_reshape_and_cache(kk.index_select(0, idx).to(self.device).contiguous(),
+                                        vv.index_select(0, idx).to(self.device).contiguous(),
+                                        self.k_cache, self.v_cache,
+                                        torch.tensor(slots, dtype=torch.int64, device=self.device))
+        self.written_tokens = sum(len(write[s][0]) for s in write)
+        self.prefill_tables = self.tables_now()
+        # the step: each request's last token
+        slots, pairs = self.alloc.append_slots(np.arange(S, dtype=np.int64))
+        last = torch.from_numpy(xoff[1:] - 1).to(xk.device)
+        self.new_k = xk.index_select(0, last).to(self.device).contiguous()
+        self.new_v = xv.index_select(0, last).to(self.device).contiguous()
+        self.slot_mapping = torch.from_numpy(slots.copy()).to(self.device)
+        self.cow_pairs = torch.from_numpy(pairs.copy()).to(self.device)
+        self.q = q.to(self.device).contiguous()
+        tables, ctx = self.tables_now()
+        self.context_lens_np = ctx
+        self.block_tables = torch.from_numpy(tables).to(self.device)
+        self.context_lens = torch.from_numpy(ctx).to(self.device)
+        self.max_context_len = int(ctx.max()) if S else 0
+        self.partition_size = wl.partition_size if partition_size is None else partition_size
+        self.out = torch.empty_like(self.q)
+        ws = pa.pa_decode_workspace_size(S, Hq, Hkv, D, B, self.max_context_len, self.partition_size)
+        self.workspace = torch.empty(max(ws, 16) // 4 + 4, dtype=torch.float32, device=self.device)
+
+    tables_now = DecodeBatch.tables_now
+    append = DecodeBatch.append
+    decode = DecodeBatch.decode
+    workspace_for = DecodeBatch.workspace_for
+    step = DecodeBatch.step
+
+    def decode_bytes(self):
+        """Logical bytes: every request's context read in full, as the decode does."""
+        wl = self.wl
+        tok = int(np.sum(self.context_lens_np))
+        blocks = int(sum((int(L) + wl.block_size - 1) // wl.block_size for L in self.context_lens_np))
+        return tok * 2 * wl.num_kv_heads * wl.head_dim * 2 + 2 * wl.num_seqs * wl.num_heads * wl.head_dim * 2 + \
+            4 * (blocks + wl.num_seqs)
+
+    def unique_kv_bytes(self):
+        """K/V bytes of the distinct blocks the decode reads (each read at least once)."""
+        wl = self.wl
+        used = np.unique(self.block_tables.cpu().numpy())
+        return int((used >= 0).sum()) * wl.block_size * 2 * wl.num_kv_heads * wl.head_dim * 2
+
+    append_bytes = DecodeBatch.append_bytes
+
+
 def make_batch(wl, device="cuda", values=None, fill=float("nan"), partition_size=None):
-    cls = CowBatch if isinstance(wl, W.CowWorkload) else DecodeBatch
+    if isinstance(wl, W.CowWorkload):
+        cls = CowBatch
+    elif isinstance(wl, W.PrefixWorkload):
+        cls = PrefixBatch
+    else:
+        cls = DecodeBatch
     return cls(wl, device=device, values=values, fill=fill, partition_size=partition_size)
 
 

@@ -39,6 +39,9 @@ WORKLOADS = {
             num_blocks=20000, partition_size=0),
     5: dict(name="long-splitk-bf16", num_seqs=8, num_heads=32, num_kv_heads=8, head_dim=128, block_size=32,
             dtype="bf16", lens=("uniform", 16384, 32768), num_blocks=12000, partition_size=512),
+    6: dict(name="prefix-cache-bf16", num_prompts=8, requests_per_prompt=16, num_heads=32, num_kv_heads=8,
+            head_dim=128, block_size=16, dtype="bf16", stem_lens=(512, 1536), suffix_lens=(16, 256),
+            vocab=32000, num_blocks=20000, partition_size=0),
 }
 
 NAME_TO_ID = {v["name"]: k for k, v in WORKLOADS.items()}
@@ -96,6 +99,46 @@ class CowWorkload:
         return self.num_prompts * self.streams_per_prompt
 
 
+@dataclass
+class PrefixWorkload:
+    """Requests that share system prompts: request r = stem[r % P] + its own suffix.
+    Token ids are seeded; the allocator's prefix cache shares the stems' full blocks."""
+    wid: int
+    name: str
+    seed: int
+    num_prompts: int
+    requests_per_prompt: int
+    num_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    dtype: str
+    num_blocks: int
+    partition_size: int
+    stem_lens: np.ndarray               # int32 [P]
+    suffix_lens: np.ndarray             # int32 [S]
+    stem_tokens: list                   # P lists of token ids
+    suffix_tokens: list                 # S lists of token ids
+    free_order: np.ndarray              # int32 [num_blocks]
+    scale: float = field(default=0.0)
+
+    @property
+    def num_seqs(self):
+        return self.num_prompts * self.requests_per_prompt
+
+    def prompt_of(self, r):
+        return r % self.num_prompts
+
+    def tokens(self, r):
+        """Token ids of request r (its decode step appends the last one)."""
+        return self.stem_tokens[self.prompt_of(r)] + self.suffix_tokens[r]
+
+    @property
+    def context_lens(self):
+        return np.array([int(self.stem_lens[self.prompt_of(r)]) + int(self.suffix_lens[r])
+                         for r in range(self.num_seqs)], np.int32)
+
+
 def _rng(seed, salt):
     return np.random.default_rng([int(seed), int(salt)])
 
@@ -129,6 +172,21 @@ def make_workload(wid, seed=0, **overrides):
                          head_dim=spec["head_dim"], block_size=spec["block_size"], dtype=spec["dtype"],
                          num_blocks=spec["num_blocks"], partition_size=spec["partition_size"],
                          prompt_lens=prompt_lens, private_tokens=private, free_order=free_order)
+    elif wid == 6:
+        P, n = spec["num_prompts"], spec["requests_per_prompt"]
+        slo, shi = spec["stem_lens"]
+        xlo, xhi = spec["suffix_lens"]
+        stem_lens = rng.integers(slo, shi + 1, size=P).astype(np.int32)
+        suffix_lens = rng.integers(xlo, xhi + 1, size=P * n).astype(np.int32)
+        stems = [rng.integers(0, spec["vocab"], size=int(L)).tolist() for L in stem_lens]
+        suffixes = [rng.integers(0, spec["vocab"], size=int(L)).tolist() for L in suffix_lens]
+        free_order = rng.permutation(spec["num_blocks"]).astype(np.int32)
+        wl = PrefixWorkload(wid=wid, name=spec["name"], seed=seed, num_prompts=P, requests_per_prompt=n,
+                            num_heads=spec["num_heads"], num_kv_heads=spec["num_kv_heads"],
+                            head_dim=spec["head_dim"], block_size=spec["block_size"], dtype=spec["dtype"],
+                            num_blocks=spec["num_blocks"], partition_size=spec["partition_size"],
+                            stem_lens=stem_lens, suffix_lens=suffix_lens, stem_tokens=stems, suffix_tokens=suffixes,
+                            free_order=free_order)
     else:
         lens = spec.pop("context_lens", None)
         if lens is None:
@@ -190,6 +248,30 @@ def cow_values(wl, device="cpu"):
     xoff = np.zeros(wl.num_seqs + 1, np.int64)
     xoff[1:] = np.cumsum(wl.private_tokens)
     return q, pk, pv, poff, xk, xv, xoff
+
+
+def prefix_values(wl, device="cpu"):
+    """q [S, Hq, D]; stem K/V rows [sum stem_lens, Hkv, D] with offsets (a stem token's
+    K/V are the same for every request that shares the stem: they depend only on the
+    prefix up to that token); suffix K/V rows [sum suffix_lens, Hkv, D] with offsets."""
+    Hq, Hkv, D = wl.num_heads, wl.num_kv_heads, wl.head_dim
+    q = normal((wl.num_seqs, Hq, D), wl.dtype, device, wl.seed, 1)
+    sk = normal((int(wl.stem_lens.sum()), Hkv, D), wl.dtype, device, wl.seed, 2)
+    sv = normal((int(wl.stem_lens.sum()), Hkv, D), wl.dtype, device, wl.seed, 3)
+    xk = normal((int(wl.suffix_lens.sum()), Hkv, D), wl.dtype, device, wl.seed, 4)
+    xv = normal((int(wl.suffix_lens.sum()), Hkv, D), wl.dtype, device, wl.seed, 5)
+    soff = np.zeros(wl.num_prompts + 1, np.int64)
+    soff[1:] = np.cumsum(wl.stem_lens)
+    xoff = np.zeros(wl.num_seqs + 1, np.int64)
+    xoff[1:] = np.cumsum(wl.suffix_lens)
+    return q, sk, sv, soff, xk, xv, xoff
+
+
+def prefix_logical_rows(wl, r, soff, xoff):
+    """(source, row) of every token of request r: source 0 = stem rows, 1 = suffix rows."""
+    p = wl.prompt_of(r)
+    stem = [(0, int(soff[p]) + i) for i in range(int(wl.stem_lens[p]))]
+    return stem + [(1, int(xoff[r]) + i) for i in range(int(wl.suffix_lens[r]))]
 
 
 def direct_block_tables(wl):

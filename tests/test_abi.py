@@ -108,29 +108,31 @@ def _replay(ops, NB, B, order):
                 continue
             assert lib_a.append_slot(op[1]) == want
         elif kind == "batch":
-            snap = (list(ora.free), list(ora.ref), {k: list(v) for k, v in ora.tables.items()},
-                    dict(ora.ntokens), ora.cow_count)
             try:
-                res = [ora.append_slot(s) for s in op[1]]
+                res = ora.append_slots(op[1])
             except OracleOOM:
-                # all-or-nothing: restore the oracle and expect the library to refuse the batch
-                ora.free.clear()
-                ora.free.extend(snap[0])
-                ora.ref[:] = snap[1]
-                ora.tables = snap[2]
-                ora.ntokens = snap[3]
-                ora.cow_count = snap[4]
+                # all-or-nothing: the oracle is unchanged and the library must refuse the batch
                 with pytest.raises(pa.OutOfBlocks):
                     lib_a.append_slots(op[1])
                 continue
             slots, pairs = lib_a.append_slots(op[1])
             assert slots.tolist() == [r[0] for r in res]
             assert [tuple(p) for p in pairs.tolist()] == [r[1] for r in res if r[1] is not None]
+        elif kind == "cached":
+            try:
+                want = ora.add_seq_cached(op[1], op[2])
+            except OracleOOM:
+                with pytest.raises(pa.OutOfBlocks):
+                    lib_a.add_seq_cached(op[1], op[2])
+                continue
+            slots, ncached = lib_a.add_seq_cached(op[1], op[2])
+            assert (slots.tolist(), ncached) == want
         elif kind == "free":
             ora.free_seq(op[1])
             lib_a.free_seq(op[1])
         # full state comparison after every op
         assert lib_a.num_free() == ora.num_free()
+        assert lib_a.num_cached_free() == ora.num_cached_free()
         for b in range(NB):
             assert lib_a.ref_count(b) == ora.ref[b]
         for sid in ora.tables:
@@ -138,6 +140,7 @@ def _replay(ops, NB, B, order):
             assert lib_a.num_tokens(sid) == ora.ntokens[sid]
     st = lib_a.stats()
     assert st["cow_copies"] == ora.cow_count
+    assert st["cached_blocks"] == len(ora.tree) and st["cached_free"] == ora.num_cached_free()
     assert st["waste_tokens"] == sum(ora.waste_tokens(s) for s in ora.tables)
     return lib_a, ora
 
@@ -148,10 +151,20 @@ def test_allocator_matches_oracle_on_random_scripts(seed):
     NB, B = int(rng.integers(20, 80)), int(rng.choice([4, 16]))
     order = rng.permutation(NB)
     ops, live, nxt = [], [], 0
+    # prompts for the prefix cache: a few shared stems over a tiny vocabulary, so that
+    # full blocks repeat, prefixes diverge part-way and evictions happen
+    stems = [rng.integers(0, 3, size=int(rng.integers(B, 5 * B))).tolist() for _ in range(3)]
     for _ in range(300):
         r = rng.random()
-        if r < 0.15 or not live:
+        if r < 0.08 or not live:
             ops.append(("add", nxt, int(rng.integers(0, 3 * B))))
+            live.append(nxt)
+            nxt += 1
+        elif r < 0.15:
+            stem = stems[int(rng.integers(0, len(stems)))]
+            cut = int(rng.integers(0, len(stem) + 1))
+            toks = stem[:cut] + rng.integers(0, 3, size=int(rng.integers(0, 2 * B))).tolist()
+            ops.append(("cached", nxt, toks))
             live.append(nxt)
             nxt += 1
         elif r < 0.3:
@@ -191,19 +204,20 @@ def test_allocator_matches_oracle_on_random_scripts(seed):
                 except OracleOOM:
                     pass
                 clean.append(op)
+        elif op[0] == "cached":
+            try:
+                sim.add_seq_cached(op[1], op[2])
+                known.add(op[1])
+            except OracleOOM:
+                pass
+            clean.append(op)
         elif op[0] == "batch":
             ids = [s for s in op[1] if s in known]
             if ids:
-                snap = (list(sim.free), list(sim.ref), {k: list(v) for k, v in sim.tables.items()},
-                        dict(sim.ntokens), sim.cow_count)
                 try:
-                    for s in ids:
-                        sim.append_slot(s)
+                    sim.append_slots(ids)
                 except OracleOOM:
-                    sim.free.clear()
-                    sim.free.extend(snap[0])
-                    sim.ref[:] = snap[1]
-                    sim.tables, sim.ntokens, sim.cow_count = snap[2], snap[3], snap[4]
+                    pass
                 clean.append(("batch", ids))
         elif op[0] == "free":
             if op[1] in known:

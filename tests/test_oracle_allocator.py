@@ -126,3 +126,143 @@ def test_out_of_blocks_changes_nothing():
     with pytest.raises(OutOfBlocks):
         a.append_slot(1)      # token 48 needs a fresh block
     assert snap == (list(a.free), list(a.ref), {k: list(v) for k, v in a.tables.items()}, dict(a.ntokens))
+
+
+# ---------------------------------------------------------------- prefix cache
+# "PagedAttention Paper Breakdown" (fullstackaihub.com), "Paper Methods": shared prefix
+# caching in a radix tree.  Read at block granularity: a node is one full block, its
+# label the block's token ids, its parent the block before it.
+
+def _state(a):
+    return (list(a.free), list(a.ref), {k: list(v) for k, v in a.tables.items()}, dict(a.ntokens),
+            dict(a.tree), list(a.unreferenced))
+
+
+def test_prefix_cache_shares_the_common_full_blocks():
+    a = OracleAllocator(32, 4)
+    s0, c0 = a.add_seq_cached(0, list(range(10)))                        # 2 full blocks + 2 tokens
+    assert c0 == 0 and len(a.tree) == 2
+    s1, c1 = a.add_seq_cached(1, list(range(8)) + [50, 51, 52, 53, 54])  # same 2 blocks, 1 new full, 1 partial
+    t0, t1 = a.block_table(0), a.block_table(1)
+    assert c1 == 8 and t1[:2] == t0[:2] and t1[2] not in t0 and t1[3] not in t0
+    assert [a.ref[b] for b in t0] == [2, 2, 1] and a.ref[t1[2]] == 1 and a.ref[t1[3]] == 1
+    assert len(a.tree) == 3                        # the partial blocks are private, never cached
+    assert s1[:8] == s0[:8]                        # shared tokens sit at the same slots
+
+
+def test_prefix_match_follows_the_path_not_the_block_content():
+    """A block is reused only under the same prefix: equal content after a divergence is not shared."""
+    a = OracleAllocator(32, 4)
+    X, Y, W, Z = [1, 1, 1, 1], [2, 2, 2, 2], [3, 3, 3, 3], [4, 4, 4, 4]
+    a.add_seq_cached(0, X + Y + Z)
+    _, c = a.add_seq_cached(1, X + W + Z)
+    t0, t1 = a.block_table(0), a.block_table(1)
+    assert c == 4 and t1[0] == t0[0] and t1[2] != t0[2]
+    _, c = a.add_seq_cached(2, Y + Z)              # Y at the root is a different node from Y under X
+    assert c == 0
+
+
+def test_cached_blocks_outlive_their_sequences_and_are_reused():
+    a = OracleAllocator(16, 4)
+    a.add_seq_cached(0, list(range(9)))            # 2 cached full blocks + 1 private partial
+    full = a.block_table(0)[:2]
+    partial = a.block_table(0)[2]
+    free_before = a.num_free()
+    a.free_seq(0)
+    assert a.num_free() == free_before + 1 and a.free[-1] == partial      # only the private block returns
+    assert a.num_cached_free() == 2 and all(a.ref[b] == 0 for b in full)
+    _, c = a.add_seq_cached(1, list(range(8)) + [99])
+    assert c == 8 and a.block_table(1)[:2] == full and a.num_cached_free() == 0
+    assert all(a.ref[b] == 1 for b in full)
+
+
+def test_eviction_takes_the_oldest_unreferenced_leaf():
+    a = OracleAllocator(5, 2)
+    a.add_seq_cached(0, [1, 1, 2, 2])              # chain p1 -> p2
+    p1, p2 = a.block_table(0)
+    a.add_seq_cached(1, [7, 7])                    # single node c1
+    (c1,) = a.block_table(1)
+    a.free_seq(0)                                  # released first: p1, then p2
+    a.free_seq(1)                                  # released later: c1
+    a.add_seq(2, 4)                                # the two free blocks
+    assert a.num_free() == 0 and a.num_cached_free() == 3
+    a.add_seq(3, 2)                                # p1 is older but has a child: the leaf p2 goes
+    assert a.block_table(3) == [p2] and p2 not in a.key_of and a.nchildren[p1] == 0
+    a.add_seq(4, 2)                                # now p1 is a leaf, and older than c1
+    assert a.block_table(4) == [p1]
+    _, c = a.add_seq_cached(5, [7, 7])             # c1 is still cached
+    assert c == 2 and a.block_table(5) == [c1]
+    with pytest.raises(OutOfBlocks):
+        a.add_seq(6, 1)
+
+
+def test_blocks_in_use_equal_distinct_prefixes_plus_partials():
+    rng = np.random.default_rng(5)
+    B = 4
+    stems = [rng.integers(0, 2, size=int(rng.integers(4, 30))).tolist() for _ in range(4)]
+    a = OracleAllocator(400, B, free_order=rng.permutation(400))
+    prompts = []
+    for sid in range(40):
+        stem = stems[sid % 4]
+        p = stem[:int(rng.integers(0, len(stem) + 1))] + rng.integers(0, 2, size=int(rng.integers(0, 9))).tolist()
+        slots, cached = a.add_seq_cached(sid, p)
+        assert cached % B == 0 and cached <= len(p) - len(p) % B
+        prompts.append(p)
+    prefixes = {tuple(p[:(j + 1) * B]) for p in prompts for j in range(len(p) // B)}
+    partials = sum(1 for p in prompts if len(p) % B)
+    assert sum(1 for r in a.ref if r > 0) == len(prefixes) + partials
+    assert len(a.tree) == len(prefixes)
+    for sid in range(40):
+        a.free_seq(sid)
+    assert a.num_free() + a.num_cached_free() == 400 and not any(a.ref)
+
+
+def test_cached_add_out_of_blocks_changes_nothing():
+    a = OracleAllocator(6, 4)
+    a.add_seq_cached(0, list(range(12)))
+    a.free_seq(0)
+    a.add_seq(1, 12)                               # 3 free blocks taken, 3 cached unreferenced remain
+    before = _state(a)
+    with pytest.raises(OutOfBlocks):
+        a.add_seq_cached(2, list(range(8)) + [9, 9, 9, 9, 9, 9, 9, 9, 9])  # 2 hits, needs 3 more, 1 evictable
+    assert _state(a) == before
+
+
+def test_prefix_shared_tables_give_the_contiguous_attention():
+    """Only the uncached tokens of each prompt are written; decode through the shared
+    tables must equal plain softmax attention over each prompt's own tokens."""
+    rng = np.random.default_rng(11)
+    B, Hkv, G, D = 4, 2, 2, 8
+    stem = rng.integers(0, 3, size=13).tolist()
+    prompts = [stem[:c] + rng.integers(0, 3, size=n).tolist() for c, n in ((13, 3), (9, 6), (13, 0), (4, 7))]
+
+    def kv_of(prefix):                              # a token's K/V depend on the whole prefix up to it
+        g = np.random.default_rng(abs(hash(tuple(prefix))) % (2 ** 32))
+        return g.standard_normal((2, Hkv, D)).astype(np.float32)
+
+    NB = 64
+    a = OracleAllocator(NB, B, free_order=rng.permutation(NB))
+    kc = np.full((NB, Hkv, B, D), np.nan, np.float32)
+    vc = np.full((NB, Hkv, B, D), np.nan, np.float32)
+    written = 0
+    for sid, p in enumerate(prompts):
+        slots, cached = a.add_seq_cached(sid, p)
+        rows = np.stack([kv_of(p[:i + 1]) for i in range(cached, len(p))]) if len(p) > cached else None
+        if rows is not None:
+            kc, vc = oracle.reshape_and_cache(rows[:, 0], rows[:, 1], kc, vc, np.asarray(slots[cached:]))
+            written += len(p) - cached
+    assert written < sum(len(p) for p in prompts)   # some K/V really are shared
+    S = len(prompts)
+    q = rng.standard_normal((S, Hkv * G, D)).astype(np.float32)
+    mb = max(len(a.block_table(s)) for s in range(S))
+    tables = np.array([a.block_table(s) + [-1] * (mb - len(a.block_table(s))) for s in range(S)], np.int32)
+    lens = np.array([len(p) for p in prompts], np.int32)
+    scale = D ** -0.5
+    out = oracle.decode(q, kc, vc, tables, lens, scale)
+    for s, p in enumerate(prompts):
+        kv = np.stack([kv_of(p[:i + 1]) for i in range(len(p))]).astype(np.float64)   # [L, 2, Hkv, D]
+        for h in range(Hkv * G):
+            z = scale * kv[:, 0, h // G] @ q[s, h].astype(np.float64)
+            w = np.exp(z - z.max())
+            w /= w.sum()
+            assert np.allclose(out[s, h], w @ kv[:, 1, h // G], rtol=0, atol=1e-12)

@@ -1,0 +1,94 @@
+"""The prefix-cache pins are strong enough: plausible mistakes planted in a subclass
+of the oracle allocator each fail at least one pin (CPU only).  The unmutated class
+passes them all.  Nothing here changes the real oracle or touches the library."""
+import pytest
+
+import test_oracle_allocator as pins
+from oracle.allocator import OracleAllocator
+
+PREFIX_PINS = [pins.test_prefix_cache_shares_the_common_full_blocks,
+               pins.test_prefix_match_follows_the_path_not_the_block_content,
+               pins.test_cached_blocks_outlive_their_sequences_and_are_reused,
+               pins.test_eviction_takes_the_oldest_unreferenced_leaf,
+               pins.test_blocks_in_use_equal_distinct_prefixes_plus_partials,
+               pins.test_cached_add_out_of_blocks_changes_nothing,
+               pins.test_prefix_shared_tables_give_the_contiguous_attention]
+
+
+class _EvictAnyOldest(OracleAllocator):
+    """Evicts the earliest-released cached block even when it still has children."""
+    def _take(self):
+        if not self.free and self.unreferenced:
+            blk = next(iter(self.unreferenced))
+            self.nchildren[blk] = 0
+        return super()._take()
+
+
+class _ContentTree(dict):
+    def get(self, key, default=None):
+        for (_, toks), blk in self.items():
+            if toks == key[1]:
+                return blk
+        return default
+
+
+class _MatchContentOnly(OracleAllocator):
+    """Looks blocks up by their token ids alone, ignoring the prefix before them."""
+    def __init__(self, *args, **kw):
+        super().__init__(*args, **kw)
+        self.tree = _ContentTree()
+
+
+class _ReleaseToFree(OracleAllocator):
+    """Returns cached blocks to the free queue at count zero (and forgets them)."""
+    def _release(self, blk):
+        self.ref[blk] -= 1
+        if self.ref[blk] == 0:
+            if blk in self.key_of:
+                key = self.key_of.pop(blk)
+                del self.tree[key]
+                del self.nchildren[blk]
+                if key[0] >= 0 and key[0] in self.nchildren:
+                    self.nchildren[key[0]] -= 1
+            self.free.append(blk)
+
+
+class _NoHoldOnHit(OracleAllocator):
+    """Reuses cached blocks without counting the new reference."""
+    def _hold(self, blk):
+        if self.ref[blk] == 0:
+            del self.unreferenced[blk]
+            self.ref[blk] = 1
+
+
+class _CachedCountsPartial(OracleAllocator):
+    """Reports the partial last block as cached too."""
+    def add_seq_cached(self, seq_id, token_ids):
+        slots, c = super().add_seq_cached(seq_id, token_ids)
+        n = len(token_ids)
+        return slots, (n if c == n - n % self.B and c > 0 else c)
+
+
+MUTANTS = {"none": OracleAllocator, "evict_any_oldest": _EvictAnyOldest, "match_content_only": _MatchContentOnly,
+           "release_to_free": _ReleaseToFree, "no_hold_on_hit": _NoHoldOnHit,
+           "cached_counts_partial": _CachedCountsPartial}
+
+
+def _failures(cls, monkeypatch):
+    monkeypatch.setattr(pins, "OracleAllocator", cls)
+    failed = []
+    for pin in PREFIX_PINS:
+        try:
+            pin()
+        except Exception:
+            failed.append(pin.__name__)
+    return failed
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_allocator_mistakes_fail_a_pin(name, monkeypatch):
+    failed = _failures(MUTANTS[name], monkeypatch)
+    if name == "none":
+        assert failed == []
+    else:
+        assert failed, "mutation %s passed every prefix-cache pin" % name

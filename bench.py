@@ -197,6 +197,14 @@ def workload_config(wl, partition, batch=None):
             cfg.update(cached_prompt_tokens=int(batch.cached_tokens.sum()), written_prompt_tokens=batch.written_tokens,
                        unique_kv_mb=round(batch.unique_kv_bytes() / 1e6, 1),
                        allocator_us_per_request=round(batch.alloc_us_per_request, 2))
+    elif isinstance(wl, W.BeamWorkload):
+        cfg.update(num_seqs=wl.num_seqs, requests=wl.num_requests, beam_width=wl.beam_width,
+                   beam_steps=wl.beam_steps, context_tokens=int(np.sum(wl.context_lens)),
+                   max_context_len=int(np.max(wl.context_lens)))
+        if batch is not None:
+            cfg.update(copies_in_timed_step=int(batch.cow_pairs.shape[0]),
+                       copies_per_beam_step=round(float(np.mean(batch.copies_per_step)), 2),
+                       allocator_us_per_beam_step=round(float(np.median(batch.host_us_per_step)), 2))
     else:
         cfg.update(num_seqs=wl.num_seqs, context_tokens=int(np.sum(wl.context_lens)),
                    max_context_len=int(np.max(wl.context_lens)))
@@ -416,6 +424,8 @@ def run_gpu(args):
         values = W.cow_values(wl, dev)
     elif isinstance(wl, W.PrefixWorkload):
         values = W.prefix_values(wl, dev)
+    elif isinstance(wl, W.BeamWorkload):
+        values = W.beam_values(wl, dev)
     else:
         values = W.decode_values(wl, dev)
     batch = runner.make_batch(wl, dev, values=values)

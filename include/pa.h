@@ -272,6 +272,23 @@ PA_API pa_status pa_alloc_append_slot(pa_allocator* a, int64_t seq_id, int64_t* 
 PA_API pa_status pa_alloc_append_slots(pa_allocator* a, const int64_t* seq_ids, int n, int64_t* slots_out,
                                 int64_t* cow_pairs_out, int* num_cow_out);
 
+/*
+ * One beam-search step ([FSAH] section 3 and [INIT] section 3: beams share blocks by
+ * copy-on-write until one writes).  The old beams are beam_ids[num_beams]; new beam
+ * j continues old beam parents[j] (an index into beam_ids) under id new_ids[j], and
+ * gets one new token.  In order: every new beam forks its parent (shares its blocks,
+ * counts + 1); the old beams are freed (in list order); then each new beam, in order,
+ * takes the slot of its token as pa_alloc_append_slots does.  Freeing before
+ * appending means a parent chosen once needs no copy, and a parent chosen k times
+ * needs k-1 copies of its partial last block.  slots_out[num_new] receives the
+ * slots; cow_pairs_out[2 * num_new] and *num_cow_out the (src, dst) copies, to be
+ * run with one pa_copy_blocks before the appends are written.  A new id may reuse
+ * an old beam's id; it must not be held by any other sequence.  All or nothing.
+ */
+PA_API pa_status pa_alloc_beam_step(pa_allocator* a, const int64_t* beam_ids, int num_beams, const int32_t* parents,
+                                    const int64_t* new_ids, int num_new, int64_t* slots_out, int64_t* cow_pairs_out,
+                                    int* num_cow_out);
+
 /* Drops one reference to each block of seq_id; blocks reaching zero rejoin the free
  * pool, or stay in the prefix tree as unreferenced cached blocks. */
 PA_API pa_status pa_alloc_free_seq(pa_allocator* a, int64_t seq_id);

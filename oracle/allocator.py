@@ -193,6 +193,33 @@ class OracleAllocator:
         self.__dict__.update(trial.__dict__)
         return res
 
+    def beam_step(self, beam_ids, parents, new_ids):
+        """A beam-search step, all or nothing ([fullstackaihub] section 3, [initnode]
+        section 3: beams share blocks by copy-on-write until one writes).  New beam j
+        continues old beam parents[j]: it is forked from it, the old beams are freed in
+        list order, the new beams take their ids, and each appends one token in order.
+        Returns [(slot, (src, dst) or None)] per new beam."""
+        beam_ids, new_ids = [int(b) for b in beam_ids], [int(b) for b in new_ids]
+        parents = [int(p) for p in parents]
+        if len(set(beam_ids)) != len(beam_ids) or any(b not in self.tables for b in beam_ids):
+            raise ValueError("old beams unknown or repeated")
+        if len(parents) != len(new_ids) or any(not 0 <= p < len(beam_ids) for p in parents):
+            raise ValueError("bad parent index")
+        if len(set(new_ids)) != len(new_ids) or any(b in self.tables and b not in beam_ids for b in new_ids):
+            raise ValueError("new beam ids repeated or taken")
+        trial = copy.deepcopy(self)
+        temp = [("beam", j) for j in range(len(new_ids))]      # ids no caller can hold
+        for j, p in enumerate(parents):
+            trial.fork(beam_ids[p], temp[j])
+        for b in beam_ids:
+            trial.free_seq(b)
+        for j, b in enumerate(new_ids):
+            trial.tables[b] = trial.tables.pop(temp[j])
+            trial.ntokens[b] = trial.ntokens.pop(temp[j])
+        res = trial.append_slots(new_ids)
+        self.__dict__.update(trial.__dict__)
+        return res
+
     def free_seq(self, seq_id):
         if seq_id not in self.tables:
             raise ValueError("unknown sequence")

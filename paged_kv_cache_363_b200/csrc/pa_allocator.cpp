@@ -370,6 +370,86 @@ pa_status pa_alloc_append_slots(pa_allocator* a, const int64_t* seq_ids, int n, 
     return PA_OK;
 }
 
+pa_status pa_alloc_beam_step(pa_allocator* a, const int64_t* beam_ids, int num_beams, const int32_t* parents,
+                             const int64_t* new_ids, int num_new, int64_t* slots_out, int64_t* cow_pairs_out,
+                             int* num_cow_out)
+{
+    if (!a || num_beams < 0 || num_new < 0 || (num_beams > 0 && !beam_ids) ||
+        (num_new > 0 && (!parents || !new_ids || !slots_out || !cow_pairs_out)) || !num_cow_out) {
+        pa::set_error("pa_alloc_beam_step: bad argument");
+        return PA_ERR_INVALID;
+    }
+    std::unordered_map<int64_t, int> old_index;
+    for (int i = 0; i < num_beams; ++i) {
+        if (!a->seqs.count(beam_ids[i]) || !old_index.emplace(beam_ids[i], i).second) {
+            pa::set_error("pa_alloc_beam_step: beam " + std::to_string(beam_ids[i]) + " unknown or listed twice");
+            return PA_ERR_INVALID;
+        }
+    }
+    std::unordered_map<int64_t, int> new_index;
+    for (int j = 0; j < num_new; ++j) {
+        if (parents[j] < 0 || parents[j] >= num_beams) {
+            pa::set_error("pa_alloc_beam_step: parent index out of range");
+            return PA_ERR_INVALID;
+        }
+        if (!new_index.emplace(new_ids[j], j).second || (a->seqs.count(new_ids[j]) && !old_index.count(new_ids[j]))) {
+            pa::set_error("pa_alloc_beam_step: new beam id " + std::to_string(new_ids[j]) +
+                          " repeated or held by a sequence outside the old beams");
+            return PA_ERR_INVALID;
+        }
+    }
+    // Count the blocks the appends take, on the reference counts the forks and frees leave.
+    std::unordered_map<int32_t, int32_t> delta;
+    for (int j = 0; j < num_new; ++j)
+        for (int32_t b : a->seqs.find(beam_ids[parents[j]])->second.table) delta[b] += 1;
+    for (int i = 0; i < num_beams; ++i)
+        for (int32_t b : a->seqs.find(beam_ids[i])->second.table) delta[b] -= 1;
+    int64_t released = 0;
+    for (const auto& d : delta)
+        if (a->ref[(size_t)d.first] > 0 && a->ref[(size_t)d.first] + d.second == 0) released += 1;
+    int64_t need = 0;
+    for (int j = 0; j < num_new; ++j) {
+        const pa_allocator::Seq& par = a->seqs.find(beam_ids[parents[j]])->second;
+        if (par.tokens % a->block_size == 0) {
+            need += 1;
+        } else {
+            const int32_t last = par.table.back();
+            if (a->ref[(size_t)last] + delta[last] > 1) {
+                need += 1;
+                delta[last] -= 1;
+            }
+        }
+    }
+    if (need > a->available() + released) {
+        pa::set_error("pa_alloc_beam_step: out of blocks");
+        return PA_ERR_OOM;
+    }
+    // fork the chosen parents, free the old beams, install the new ones, append one slot each
+    std::vector<pa_allocator::Seq> fresh((size_t)num_new);
+    for (int j = 0; j < num_new; ++j) {
+        fresh[(size_t)j] = a->seqs.find(beam_ids[parents[j]])->second;
+        for (int32_t b : fresh[(size_t)j].table) a->add_ref(b);
+    }
+    for (int i = 0; i < num_beams; ++i) {
+        auto it = a->seqs.find(beam_ids[i]);
+        for (int32_t b : it->second.table) a->drop_ref(b);
+        a->seqs.erase(it);
+    }
+    for (int j = 0; j < num_new; ++j) a->seqs.emplace(new_ids[j], std::move(fresh[(size_t)j]));
+    int ncow = 0;
+    for (int j = 0; j < num_new; ++j) {
+        int32_t src, dst;
+        slots_out[j] = a->append(new_ids[j], &src, &dst);
+        if (src >= 0) {
+            cow_pairs_out[2 * ncow] = src;
+            cow_pairs_out[2 * ncow + 1] = dst;
+            ++ncow;
+        }
+    }
+    *num_cow_out = ncow;
+    return PA_OK;
+}
+
 pa_status pa_alloc_free_seq(pa_allocator* a, int64_t seq_id)
 {
     if (!a) return PA_ERR_INVALID;

@@ -47,6 +47,7 @@ SIGNATURES = [
     ("pa_alloc_fork", _int, [_vp, _i64, _i64]),
     ("pa_alloc_append_slot", _int, [_vp, _i64, ctypes.POINTER(_i64), ctypes.POINTER(_i32), ctypes.POINTER(_i32)]),
     ("pa_alloc_append_slots", _int, [_vp, _vp, _int, _vp, _vp, ctypes.POINTER(_int)]),
+    ("pa_alloc_beam_step", _int, [_vp, _vp, _int, _vp, _vp, _int, _vp, _vp, ctypes.POINTER(_int)]),
     ("pa_alloc_free_seq", _int, [_vp, _i64]),
     ("pa_alloc_block_table", _int, [_vp, _i64, _vp, _int, ctypes.POINTER(_int)]),
     ("pa_alloc_block_tables", _int, [_vp, _vp, _int, _vp, _int, _i32, _vp]),
@@ -274,6 +275,22 @@ class Allocator:
         ncow = _int(0)
         _check(lib.pa_alloc_append_slots(self._h, _np_ptr(ids), n, _np_ptr(slots), _np_ptr(pairs),
                                          ctypes.byref(ncow)), "pa_alloc_append_slots")
+        return slots[:n], pairs[:ncow.value]
+
+    def beam_step(self, beam_ids, parents, new_ids):
+        """Beam j of the new set continues old beam parents[j] under new_ids[j] and gets
+        one token.  Returns (slots of the new tokens, copy-on-write pairs [k, 2])."""
+        old = np.ascontiguousarray(beam_ids, dtype=np.int64)
+        par = np.ascontiguousarray(parents, dtype=np.int32)
+        new = np.ascontiguousarray(new_ids, dtype=np.int64)
+        if par.shape != new.shape:
+            raise ValueError("parents and new_ids differ in length")
+        n = new.shape[0]
+        slots = np.empty(max(1, n), np.int64)
+        pairs = np.empty((max(1, n), 2), np.int64)
+        ncow = _int(0)
+        _check(lib.pa_alloc_beam_step(self._h, _np_ptr(old), old.shape[0], _np_ptr(par), _np_ptr(new), n,
+                                      _np_ptr(slots), _np_ptr(pairs), ctypes.byref(ncow)), "pa_alloc_beam_step")
         return slots[:n], pairs[:ncow.value]
 
     def free_seq(self, seq_id):

@@ -303,11 +303,88 @@ class PrefixBatch:
     append_bytes = DecodeBatch.append_bytes
 
 
+class BeamBatch:
+    """Beam search through the allocator's beam step.
+
+    Each request's prompt is written once and forked into its beams.  Every beam step
+    reshuffles the beams (pa_alloc_beam_step: fork the chosen parents, free the old
+    beams, append one slot per new beam), runs the step's copy-on-write copies as one
+    pa_copy_blocks, and writes the new tokens with pa_reshape_and_cache.  All steps but
+    the last run at construction; the last one is the batch's step (copies, append,
+    decode), which can be repeated: the copies and the append rewrite the same bytes.
+    """
+
+    def __init__(self, wl, device="cuda", values=None, fill=float("nan"), partition_size=None):
+        self.wl = wl
+        self.device = torch.device(device)
+        S, Hq, Hkv, D, B, NB = (wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size,
+                                wl.num_blocks)
+        Wd, T = wl.beam_width, wl.beam_steps
+        dt = W.torch_dtype(wl.dtype)
+        if values is None:
+            values = W.beam_values(wl, self.device)
+        q, pk, pv, poff, nk, nv = values
+        self.k_cache = torch.full((NB, Hkv, B, D), fill, dtype=dt, device=self.device)
+        self.v_cache = torch.full((NB, Hkv, B, D), fill, dtype=dt, device=self.device)
+        self.alloc = pa.Allocator(NB, B, wl.free_order)
+        ids = np.arange(S, dtype=np.int64)
+        slots = []
+        for r in range(wl.num_requests):
+            slots.append(self.alloc.add_seq(r * Wd, int(wl.prompt_lens[r])))
+            for j in range(1, Wd):
+                self.alloc.fork(r * Wd, r * Wd + j)
+        sl = torch.from_numpy(np.concatenate(slots)).to(self.device)
+        pa.pa_reshape_and_cache(pk.to(self.device).contiguous(), pv.to(self.device).contiguous(), self.k_cache,
+                                self.v_cache, sl)
+        self.copies_per_step = []
+        self.host_us_per_step = []
+        for t in range(T):
+            t0 = time.perf_counter()
+            st_slots, pairs = self.alloc.beam_step(ids, wl.parents[t], ids)
+            self.host_us_per_step.append(1e6 * (time.perf_counter() - t0))
+            self.copies_per_step.append(len(pairs))
+            new_k = nk[t * S:(t + 1) * S].to(self.device).contiguous()
+            new_v = nv[t * S:(t + 1) * S].to(self.device).contiguous()
+            slot_mapping = torch.from_numpy(st_slots.copy()).to(self.device)
+            cow_pairs = torch.from_numpy(pairs.copy()).to(self.device)
+            if t < T - 1:
+                if len(pairs):
+                    pa.pa_copy_blocks(self.k_cache, self.v_cache, cow_pairs)
+                pa.pa_reshape_and_cache(new_k, new_v, self.k_cache, self.v_cache, slot_mapping)
+        self.new_k, self.new_v, self.slot_mapping, self.cow_pairs = new_k, new_v, slot_mapping, cow_pairs
+        self.q = q.to(self.device).contiguous()
+        tables, ctx = self.tables_now()
+        self.context_lens_np = ctx
+        self.block_tables = torch.from_numpy(tables).to(self.device)
+        self.context_lens = torch.from_numpy(ctx).to(self.device)
+        self.max_context_len = int(ctx.max()) if S else 0
+        self.partition_size = wl.partition_size if partition_size is None else partition_size
+        self.out = torch.empty_like(self.q)
+        ws = pa.pa_decode_workspace_size(S, Hq, Hkv, D, B, self.max_context_len, self.partition_size)
+        self.workspace = torch.empty(max(ws, 16) // 4 + 4, dtype=torch.float32, device=self.device)
+
+    tables_now = DecodeBatch.tables_now
+    append = DecodeBatch.append
+    decode = DecodeBatch.decode
+    workspace_for = DecodeBatch.workspace_for
+    step = DecodeBatch.step
+    decode_bytes = PrefixBatch.decode_bytes
+    unique_kv_bytes = PrefixBatch.unique_kv_bytes
+
+    def append_bytes(self):
+        """The step's new rows (read and written) plus its whole-block copies."""
+        wl = self.wl
+        row = wl.num_kv_heads * wl.head_dim * 2
+        return wl.num_seqs * (2 * row * 2 + 8) + int(self.cow_pairs.shape[0]) * 2 * (row * wl.block_size) * 2
+
+
 def make_batch(wl, device="cuda", values=None, fill=float("nan"), partition_size=None):
     if isinstance(wl, W.CowWorkload):
         cls = CowBatch
     elif isinstance(wl, W.PrefixWorkload):
         cls = PrefixBatch
+    elif isinstance(wl, W.BeamWorkload):
+        cls = BeamBatch
     else:
         cls = DecodeBatch
     return cls(wl, device=device, values=values, fill=fill, partition_size=partition_size)

@@ -42,6 +42,9 @@ WORKLOADS = {
     6: dict(name="prefix-cache-bf16", num_prompts=8, requests_per_prompt=16, num_heads=32, num_kv_heads=8,
             head_dim=128, block_size=16, dtype="bf16", stem_lens=(512, 1536), suffix_lens=(16, 256),
             vocab=32000, num_blocks=20000, partition_size=0),
+    7: dict(name="beam-search-bf16", num_requests=16, beam_width=4, num_heads=32, num_kv_heads=8, head_dim=128,
+            block_size=16, dtype="bf16", prompt_lens=(256, 1024), beam_steps=24, num_blocks=20000,
+            partition_size=0),
 }
 
 NAME_TO_ID = {v["name"]: k for k, v in WORKLOADS.items()}
@@ -139,6 +142,41 @@ class PrefixWorkload:
                          for r in range(self.num_seqs)], np.int32)
 
 
+@dataclass
+class BeamWorkload:
+    """Beam search: each request's prompt is forked into beam_width beams; every step,
+    new beam j of a request continues a seeded choice of that request's beams (with
+    repeats, so beams die and others split) and appends one token."""
+    wid: int
+    name: str
+    seed: int
+    num_requests: int
+    beam_width: int
+    num_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    dtype: str
+    num_blocks: int
+    partition_size: int
+    prompt_lens: np.ndarray             # int32 [R]
+    parents: np.ndarray                 # int32 [steps, R * W]: index into the old beams (same request)
+    free_order: np.ndarray              # int32 [num_blocks]
+    scale: float = field(default=0.0)
+
+    @property
+    def num_seqs(self):
+        return self.num_requests * self.beam_width
+
+    @property
+    def beam_steps(self):
+        return int(self.parents.shape[0])
+
+    @property
+    def context_lens(self):
+        return np.repeat(self.prompt_lens, self.beam_width) + self.beam_steps
+
+
 def _rng(seed, salt):
     return np.random.default_rng([int(seed), int(salt)])
 
@@ -172,6 +210,18 @@ def make_workload(wid, seed=0, **overrides):
                          head_dim=spec["head_dim"], block_size=spec["block_size"], dtype=spec["dtype"],
                          num_blocks=spec["num_blocks"], partition_size=spec["partition_size"],
                          prompt_lens=prompt_lens, private_tokens=private, free_order=free_order)
+    elif wid == 7:
+        R, Wd, T = spec["num_requests"], spec["beam_width"], spec["beam_steps"]
+        plo, phi = spec["prompt_lens"]
+        prompt_lens = rng.integers(plo, phi + 1, size=R).astype(np.int32)
+        choice = rng.integers(0, Wd, size=(T, R, Wd))
+        parents = (np.arange(R)[None, :, None] * Wd + choice).reshape(T, R * Wd).astype(np.int32)
+        free_order = rng.permutation(spec["num_blocks"]).astype(np.int32)
+        wl = BeamWorkload(wid=wid, name=spec["name"], seed=seed, num_requests=R, beam_width=Wd,
+                          num_heads=spec["num_heads"], num_kv_heads=spec["num_kv_heads"], head_dim=spec["head_dim"],
+                          block_size=spec["block_size"], dtype=spec["dtype"], num_blocks=spec["num_blocks"],
+                          partition_size=spec["partition_size"], prompt_lens=prompt_lens, parents=parents,
+                          free_order=free_order)
     elif wid == 6:
         P, n = spec["num_prompts"], spec["requests_per_prompt"]
         slo, shi = spec["stem_lens"]
@@ -265,6 +315,30 @@ def prefix_values(wl, device="cpu"):
     xoff = np.zeros(wl.num_seqs + 1, np.int64)
     xoff[1:] = np.cumsum(wl.suffix_lens)
     return q, sk, sv, soff, xk, xv, xoff
+
+
+def beam_values(wl, device="cpu"):
+    """q [S, Hq, D]; prompt K/V rows [sum prompt_lens, Hkv, D] with offsets; the K/V of
+    the token beam j appends at step t: rows [t * S + j] of new K/V [steps * S, Hkv, D]."""
+    Hq, Hkv, D, S = wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.num_seqs
+    q = normal((S, Hq, D), wl.dtype, device, wl.seed, 1)
+    pk = normal((int(wl.prompt_lens.sum()), Hkv, D), wl.dtype, device, wl.seed, 2)
+    pv = normal((int(wl.prompt_lens.sum()), Hkv, D), wl.dtype, device, wl.seed, 3)
+    nk = normal((wl.beam_steps * S, Hkv, D), wl.dtype, device, wl.seed, 4)
+    nv = normal((wl.beam_steps * S, Hkv, D), wl.dtype, device, wl.seed, 5)
+    poff = np.zeros(wl.num_requests + 1, np.int64)
+    poff[1:] = np.cumsum(wl.prompt_lens)
+    return q, pk, pv, poff, nk, nv
+
+
+def beam_histories(wl, poff):
+    """Per final beam, the (source, row) of every token it holds: source 0 = prompt rows,
+    1 = new-token rows.  Follows the parent choices step by step."""
+    W, S = wl.beam_width, wl.num_seqs
+    hist = [[(0, int(poff[b // W]) + i) for i in range(int(wl.prompt_lens[b // W]))] for b in range(S)]
+    for t in range(wl.beam_steps):
+        hist = [hist[int(wl.parents[t, j])] + [(1, t * S + j)] for j in range(S)]
+    return hist
 
 
 def prefix_logical_rows(wl, r, soff, xoff):

@@ -118,6 +118,16 @@ def _replay(ops, NB, B, order):
             slots, pairs = lib_a.append_slots(op[1])
             assert slots.tolist() == [r[0] for r in res]
             assert [tuple(p) for p in pairs.tolist()] == [r[1] for r in res if r[1] is not None]
+        elif kind == "beam":
+            try:
+                res = ora.beam_step(op[1], op[2], op[3])
+            except OracleOOM:
+                with pytest.raises(pa.OutOfBlocks):
+                    lib_a.beam_step(op[1], op[2], op[3])
+                continue
+            slots, pairs = lib_a.beam_step(op[1], op[2], op[3])
+            assert slots.tolist() == [r[0] for r in res]
+            assert [tuple(p) for p in pairs.tolist()] == [r[1] for r in res if r[1] is not None]
         elif kind == "cached":
             try:
                 want = ora.add_seq_cached(op[1], op[2])
@@ -173,9 +183,25 @@ def test_allocator_matches_oracle_on_random_scripts(seed):
             nxt += 1
         elif r < 0.7:
             ops.append(("append", int(rng.choice(live))))
-        elif r < 0.85:
+        elif r < 0.78:
             k = int(rng.integers(1, len(live) + 1))
             ops.append(("batch", [int(x) for x in rng.choice(live, size=k, replace=False)]))
+        elif r < 0.85:
+            old = [int(x) for x in rng.choice(live, size=int(rng.integers(1, min(4, len(live)) + 1)),
+                                              replace=False)]
+            width = int(rng.integers(0, 5))
+            parents = rng.integers(0, len(old), size=width).tolist()
+            new = []
+            for j in range(width):                 # reuse an old beam's id or take a fresh one
+                if j < len(old) and rng.random() < 0.5:
+                    new.append(old[j])
+                else:
+                    new.append(nxt)
+                    nxt += 1
+            ops.append(("beam", old, parents, new))
+            for b in old:
+                live.remove(b)
+            live.extend(new)
         else:
             sid = int(rng.choice(live))
             ops.append(("free", sid))
@@ -211,6 +237,15 @@ def test_allocator_matches_oracle_on_random_scripts(seed):
             except OracleOOM:
                 pass
             clean.append(op)
+        elif op[0] == "beam":
+            if all(b in known for b in op[1]):
+                try:
+                    sim.beam_step(op[1], op[2], op[3])
+                    known.difference_update(op[1])
+                    known.update(op[3])
+                except OracleOOM:
+                    pass
+                clean.append(op)
         elif op[0] == "batch":
             ids = [s for s in op[1] if s in known]
             if ids:

@@ -266,3 +266,106 @@ def test_prefix_shared_tables_give_the_contiguous_attention():
             w = np.exp(z - z.max())
             w /= w.sum()
             assert np.allclose(out[s, h], w @ kv[:, 1, h // G], rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- beam search
+# [fullstackaihub] section 3 and "Summary & Key Takeaways" 3; [initnode] section 3:
+# beams share blocks by copy-on-write until one of them writes.
+
+def _beams(a, B, prompt, width):
+    a.add_seq(0, prompt)
+    for j in range(1, width):
+        a.fork(0, j)
+    return list(range(width))
+
+
+def test_beam_step_with_each_parent_once_copies_nothing():
+    a = OracleAllocator(64, 4)
+    beams = _beams(a, 4, 10, 3)                    # 3 beams sharing 3 blocks (last one partial)
+    for j in beams:                                # diverge: first appends copy the shared partial block
+        a.append_slot(j)
+    before = {j: a.block_table(j) for j in beams}
+    res = a.beam_step(beams, [2, 0, 1], [10, 11, 12])   # a permutation: every parent once
+    assert all(c is None for _, c in res)          # fork-then-free leaves every last block private
+    assert [a.block_table(n) for n in (10, 11, 12)] == [before[2], before[0], before[1]]
+    assert all(a.ntokens[n] == 12 for n in (10, 11, 12))
+    assert all(b not in a.tables for b in beams)
+
+
+def test_beam_step_parent_twice_copies_once_and_frees_the_dropped_beam():
+    a = OracleAllocator(64, 4)
+    beams = _beams(a, 4, 9, 2)
+    a.append_slot(0)                               # beam 0 copies the shared partial block
+    a.append_slot(1)                               # beam 1 now writes in place
+    t0, t1 = a.block_table(0), a.block_table(1)
+    private1 = [b for b in t1 if b not in t0]
+    free_before = a.num_free()
+    res = a.beam_step([0, 1], [0, 0], [0, 1])      # both new beams continue beam 0; beam 1 dropped
+    copies = [c for _, c in res if c is not None]
+    assert len(copies) == 1 and copies[0][0] == t0[-1]        # k children of one parent: k-1 copies
+    # the first child to write copies; the last one writes in place in the parent's block
+    assert a.block_table(0)[:-1] == t0[:-1] and a.block_table(0)[-1] == copies[0][1] and a.block_table(1) == t0
+    assert all(a.ref[b] == 0 for b in private1) and a.num_free() == free_before + len(private1) - 1
+    assert all(a.ref[b] == 2 for b in t0[:-1])                # full shared blocks are never copied
+
+
+def test_beam_steps_keep_every_beam_its_parent_plus_one_token():
+    """After random beam steps, decode through each beam's table equals plain attention
+    over the tokens that beam accumulated (its ancestors' tokens, then its own)."""
+    rng = np.random.default_rng(3)
+    B, Hkv, G, D, W, prompt = 4, 1, 2, 8, 4, 7
+    NB = 128
+    a = OracleAllocator(NB, B, free_order=rng.permutation(NB))
+    kc = np.full((NB, Hkv, B, D), np.nan, np.float32)
+    vc = np.full((NB, Hkv, B, D), np.nan, np.float32)
+    rows = [rng.standard_normal((2, Hkv, D)).astype(np.float32) for _ in range(prompt)]
+    slots = a.add_seq(0, prompt)
+    kc, vc = oracle.reshape_and_cache(np.stack([r[0] for r in rows]), np.stack([r[1] for r in rows]), kc, vc,
+                                      np.array(slots))
+    hist = {0: list(range(prompt))}                # beam -> indices into `rows`
+    beams = [0]
+    for step in range(9):
+        parents = rng.integers(0, len(beams), size=W).tolist()
+        new_ids = [100 * (step + 1) + j for j in range(W)]
+        res = a.beam_step(beams, parents, new_ids)
+        pairs = [c for _, c in res if c is not None]
+        if pairs:
+            kc, vc = oracle.copy_blocks(kc, vc, np.array(pairs))
+        new_rows = []
+        for j, (slot, _) in enumerate(res):
+            rows.append(rng.standard_normal((2, Hkv, D)).astype(np.float32))
+            new_rows.append(len(rows) - 1)
+        kc, vc = oracle.reshape_and_cache(np.stack([rows[i][0] for i in new_rows]),
+                                          np.stack([rows[i][1] for i in new_rows]), kc, vc,
+                                          np.array([s for s, _ in res]))
+        hist = {new_ids[j]: hist[beams[p]] + [new_rows[j]] for j, p in enumerate(parents)}
+        beams = new_ids
+    assert sum(1 for r in a.ref if r > 0) == len({b for n in beams for b in a.block_table(n)})
+    q = rng.standard_normal((W, Hkv * G, D)).astype(np.float32)
+    mb = max(len(a.block_table(n)) for n in beams)
+    tables = np.array([a.block_table(n) + [-1] * (mb - len(a.block_table(n))) for n in beams], np.int32)
+    lens = np.array([a.ntokens[n] for n in beams], np.int32)
+    scale = D ** -0.5
+    out = oracle.decode(q, kc, vc, tables, lens, scale)
+    for s, n in enumerate(beams):
+        kv = np.stack([rows[i] for i in hist[n]]).astype(np.float64)
+        assert len(hist[n]) == lens[s]
+        for h in range(Hkv * G):
+            z = scale * kv[:, 0, h // G] @ q[s, h].astype(np.float64)
+            w = np.exp(z - z.max())
+            w /= w.sum()
+            assert np.allclose(out[s, h], w @ kv[:, 1, h // G], rtol=0, atol=1e-12)
+
+
+def test_beam_step_out_of_blocks_changes_nothing():
+    a = OracleAllocator(5, 4)
+    beams = _beams(a, 4, 6, 2)                     # 2 blocks shared by 2 beams
+    a.add_seq(9, 12)                               # the other 3 blocks
+    before = _state(a)
+    with pytest.raises(OutOfBlocks):
+        a.beam_step(beams, [0, 0, 1], [5, 6, 7])   # 3 beams on one shared partial block: 2 copies, 0 free
+    assert _state(a) == before
+    with pytest.raises(ValueError):
+        a.beam_step(beams, [0, 2], [5, 6])
+    with pytest.raises(ValueError):
+        a.beam_step(beams, [0, 1], [9, 6])         # 9 is held by a sequence outside the beams

@@ -1,10 +1,15 @@
-"""The prefix-cache pins are strong enough: plausible mistakes planted in a subclass
-of the oracle allocator each fail at least one pin (CPU only).  The unmutated class
+"""The prefix-cache and beam-search pins are strong enough: plausible mistakes
+planted in a subclass of the oracle allocator each fail at least one pin (CPU only).  The unmutated class
 passes them all.  Nothing here changes the real oracle or touches the library."""
 import pytest
 
 import test_oracle_allocator as pins
 from oracle.allocator import OracleAllocator
+
+BEAM_PINS = [pins.test_beam_step_with_each_parent_once_copies_nothing,
+             pins.test_beam_step_parent_twice_copies_once_and_frees_the_dropped_beam,
+             pins.test_beam_steps_keep_every_beam_its_parent_plus_one_token,
+             pins.test_beam_step_out_of_blocks_changes_nothing]
 
 PREFIX_PINS = [pins.test_prefix_cache_shares_the_common_full_blocks,
                pins.test_prefix_match_follows_the_path_not_the_block_content,
@@ -69,18 +74,45 @@ class _CachedCountsPartial(OracleAllocator):
         return slots, (n if c == n - n % self.B and c > 0 else c)
 
 
+class _AppendBeforeFree(OracleAllocator):
+    """Beam step that appends the new tokens while the old beams still hold their blocks."""
+    def beam_step(self, beam_ids, parents, new_ids):
+        trial = __import__("copy").deepcopy(self)
+        temp = [("beam", j) for j in range(len(new_ids))]
+        for j, p in enumerate(parents):
+            trial.fork(beam_ids[p], temp[j])
+        res = trial.append_slots(temp)
+        for b in beam_ids:
+            trial.free_seq(b)
+        for j, b in enumerate(new_ids):
+            trial.tables[b] = trial.tables.pop(temp[j])
+            trial.ntokens[b] = trial.ntokens.pop(temp[j])
+        self.__dict__.update(trial.__dict__)
+        return res
+
+
+class _ForkWithoutReference(OracleAllocator):
+    """Fork that shares the parent's blocks without counting the child's reference."""
+    def fork(self, parent, child):
+        self.tables[child] = list(self.tables[parent])
+        self.ntokens[child] = self.ntokens[parent]
+
+
+BEAM_MUTANTS = {"none": OracleAllocator, "append_before_free": _AppendBeforeFree,
+                "fork_without_reference": _ForkWithoutReference}
+
 MUTANTS = {"none": OracleAllocator, "evict_any_oldest": _EvictAnyOldest, "match_content_only": _MatchContentOnly,
            "release_to_free": _ReleaseToFree, "no_hold_on_hit": _NoHoldOnHit,
            "cached_counts_partial": _CachedCountsPartial}
 
 
-def _failures(cls, monkeypatch):
+def _failures(cls, monkeypatch, which=None):
     monkeypatch.setattr(pins, "OracleAllocator", cls)
     failed = []
-    for pin in PREFIX_PINS:
+    for pin in (PREFIX_PINS if which is None else which):
         try:
             pin()
-        except Exception:
+        except (Exception, pytest.fail.Exception):   # pytest.raises reports through a BaseException
             failed.append(pin.__name__)
     return failed
 
@@ -92,3 +124,12 @@ def test_planted_allocator_mistakes_fail_a_pin(name, monkeypatch):
         assert failed == []
     else:
         assert failed, "mutation %s passed every prefix-cache pin" % name
+
+
+@pytest.mark.parametrize("name", sorted(BEAM_MUTANTS))
+def test_planted_beam_mistakes_fail_a_pin(name, monkeypatch):
+    failed = _failures(BEAM_MUTANTS[name], monkeypatch, BEAM_PINS)
+    if name == "none":
+        assert failed == []
+    else:
+        assert failed, "mutation %s passed every beam pin" % name

@@ -320,9 +320,10 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ the CUDA path
 
-def companion_timing(batch, stream, reps=200, num_pairs=96):
-    """Latency and GB/s of the two companions alone: the step's slot-mapped append, and a
-    copy-on-write batch of `num_pairs` whole-block copies from blocks in use to free ones.
+def companion_timing(batch, stream, reps=50, num_pairs=96):
+    """Latency and GB/s of the companions alone: the step's slot-mapped append, a
+    copy-on-write batch of `num_pairs` whole-block copies from blocks in use to free ones,
+    and a swap of up to 128 blocks out to pinned host memory and back in.
     `us` is the median of per-call CUDA-event brackets; `us_back_to_back` the mean over
     `reps` calls queued without gaps."""
     import torch
@@ -345,6 +346,23 @@ def companion_timing(batch, stream, reps=200, num_pairs=96):
         "copy_blocks": (lambda: pa.pa_copy_blocks(batch.k_cache, batch.v_cache, pairs_d, stream=stream),
                         n * 2 * (row * wl.block_size) * 2 + 16 * n, {"pairs": n}),
     }
+    # swapping: whole blocks between the device pool and a pinned host pool, both ways
+    ns = int(min(128, len(used), len(free)))
+    kh = torch.empty((ns,) + tuple(batch.k_cache.shape[1:]), dtype=batch.k_cache.dtype).pin_memory()
+    vh = torch.empty_like(kh).pin_memory()
+    out_pairs = torch.from_numpy(np.stack([rng.choice(used, ns, replace=False), np.arange(ns)], 1)
+                                 .astype(np.int64)).to(batch.device)
+    in_pairs = torch.from_numpy(np.stack([np.arange(ns), rng.choice(free, ns, replace=False)], 1)
+                                .astype(np.int64)).to(batch.device)
+    swap_bytes = ns * 2 * row * wl.block_size
+    calls["swap_out"] = (lambda: pa.pa_swap_blocks(kh, vh, batch.k_cache, batch.v_cache, out_pairs, stream=stream),
+                         swap_bytes, {"pairs": ns, "direction": "device to pinned host"})
+    calls["swap_in"] = (lambda: pa.pa_swap_blocks(batch.k_cache, batch.v_cache, kh, vh, in_pairs, stream=stream),
+                        swap_bytes, {"pairs": ns, "direction": "pinned host to device"})
+    flat_h = kh.view(-1)
+    flat_d = torch.empty_like(flat_h, device=batch.device)
+    calls["copy_engine_h2d_reference"] = (lambda: flat_d.copy_(flat_h, non_blocking=True), ns * row * wl.block_size,
+                                          {"note": "one contiguous copy of one pool's swapped bytes (PCIe ceiling)"})
     out = {}
     for name, (fn, nbytes, extra) in calls.items():
         for _ in range(5):

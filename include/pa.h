@@ -195,6 +195,24 @@ PA_API pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* blo
  */
 PA_API pa_status pa_device_status(uint32_t* flags, void* stream);
 
+/*
+ * Whole-block copies from one pool to another ([FSAH] "Engineering Limitations":
+ * CPU-GPU block swapping under memory pressure): for each (src, dst) pair in
+ * block_mapping[num_pairs][2] (int64), block src of src_k_cache / src_v_cache
+ * ([num_src_blocks][Hkv][B][D]) is copied to block dst of dst_k_cache / dst_v_cache
+ * ([num_dst_blocks][Hkv][B][D]).  Each pool, and block_mapping, may be device memory
+ * or pinned (page-locked) host memory, which the kernel reads or writes over PCIe
+ * through its device mapping; pageable host memory is refused (PA_ERR_INVALID).
+ * Pairs must not write one destination twice or read a block another pair writes.
+ * Out-of-range pairs raise PA_DEV_BAD_PAIR and are skipped.  Asynchronous on stream;
+ * the host side must stay allocated (and unread, for a swap-out) until the stream
+ * reaches the copy.
+ */
+PA_API pa_status pa_swap_blocks(void* dst_k_cache, void* dst_v_cache, const void* src_k_cache,
+                                const void* src_v_cache, const int64_t* block_mapping, int num_pairs,
+                                int num_kv_heads, int head_dim, int block_size, int num_src_blocks,
+                                int num_dst_blocks, pa_dtype dtype, void* stream);
+
 /* ------------------------------------------------------------------ block allocator */
 
 /*
@@ -224,6 +242,9 @@ typedef struct {
     int64_t waste_tokens;      /* unused slots in the sequences' last blocks */
     int64_t cached_blocks;     /* blocks in the prefix tree (referenced or not) */
     int64_t cached_free;       /* unreferenced cached blocks (reusable by eviction) */
+    int64_t host_blocks;       /* blocks of the host tier (0 without one) */
+    int64_t host_free;         /* free host blocks */
+    int64_t swapped_seqs;      /* sequences swapped out to the host tier */
 } pa_alloc_stats_t;
 
 /* Returns NULL on bad arguments (see pa_last_error_string). */
@@ -292,6 +313,33 @@ PA_API pa_status pa_alloc_beam_step(pa_allocator* a, const int64_t* beam_ids, in
 /* Drops one reference to each block of seq_id; blocks reaching zero rejoin the free
  * pool, or stay in the prefix tree as unreferenced cached blocks. */
 PA_API pa_status pa_alloc_free_seq(pa_allocator* a, int64_t seq_id);
+
+/*
+ * Host tier for swapping ([FSAH] "Engineering Limitations": CPU-GPU block swapping
+ * under memory pressure).  pa_alloc_add_host_pool gives the allocator
+ * num_host_blocks host blocks (ids 0..n-1, a FIFO free queue), once.  The caller
+ * owns the host pools themselves: pinned host memory shaped like the device pools
+ * ([num_host_blocks][Hkv][B][D] for K and for V), moved with pa_swap_blocks.
+ *
+ * pa_alloc_swap_out moves a resident sequence to the host: each of its blocks, in
+ * table order, gets a host block; (device, host) pairs go to pairs_out[2 * n] and
+ * *num_pairs_out = n; each device block loses the sequence's reference (blocks that
+ * other sequences share stay with them; cached blocks stay cached).  The caller must
+ * run pa_swap_blocks(host pools <- device pools, pairs) before any later write can
+ * reach the released device blocks, i.e. before the next append's copy in stream
+ * order.  pa_alloc_swap_in brings it back: each host block gets a device block
+ * (taken as any other), (host, device) pairs are returned, the host blocks are freed;
+ * run pa_swap_blocks(device pools <- host pools, pairs) before the sequence's next
+ * decode.  A swapped-out sequence cannot be forked, appended to, reshuffled or put in
+ * a dense table (PA_ERR_INVALID); pa_alloc_free_seq frees its host blocks;
+ * pa_alloc_block_table returns its host block ids.  Out of host or device blocks:
+ * PA_ERR_OOM, nothing changes.
+ */
+PA_API pa_status pa_alloc_add_host_pool(pa_allocator* a, int num_host_blocks);
+PA_API pa_status pa_alloc_swap_out(pa_allocator* a, int64_t seq_id, int64_t* pairs_out, int* num_pairs_out);
+PA_API pa_status pa_alloc_swap_in(pa_allocator* a, int64_t seq_id, int64_t* pairs_out, int* num_pairs_out);
+PA_API int pa_alloc_num_host_free(const pa_allocator* a);
+PA_API int pa_alloc_is_swapped(const pa_allocator* a, int64_t seq_id);  /* 1, 0, or -1 if unknown */
 
 /* Copies seq_id's block table into out[capacity]; *n_out = its length.
  * PA_ERR_INVALID if capacity is too small (nothing is written then). */

@@ -25,6 +25,13 @@ count going up by one; copy-on-write happens only on a write into a shared,
 partially filled last block; running out of blocks raises OutOfBlocks and
 changes nothing (a batch of appends included).
 
+Host tier ([fullstackaihub] "Engineering Limitations": CPU-GPU block swapping
+under memory pressure; the pages give no policy, only the mechanism).  Read as: a
+separate pool of host blocks with its own FIFO free queue; swapping a sequence out
+gives each of its blocks, in table order, a host block and drops the sequence's
+reference to the device block; swapping in takes device blocks as any allocation
+does and frees the host blocks; a swapped-out sequence is only held, never used.
+
 Prefix cache (the pages name the radix tree only).  The tree is read at block
 granularity: each node is one full physical block, labelled by the B token ids it
 holds and hanging under the node of the block before it, so the path from the root
@@ -62,6 +69,9 @@ class OracleAllocator:
         self.key_of = {}          # cached block -> its key in the tree
         self.nchildren = {}       # cached block -> number of cached children
         self.unreferenced = OrderedDict()   # cached blocks with count 0, earliest release first
+        self.host_free = deque()  # host tier: free host blocks
+        self.num_host_blocks = 0
+        self.on_host = set()      # sequences swapped out (their tables hold host blocks)
 
     # [fullstackaihub] section 2: PhysicalAddr = T[floor(i/B)]*B + (i mod B)
     def slot(self, seq_id, i):
@@ -152,7 +162,7 @@ class OracleAllocator:
 
     def fork(self, parent, child):
         """Child shares every block of the parent (each count + 1)."""
-        if parent not in self.tables or child in self.tables:
+        if parent not in self.tables or parent in self.on_host or child in self.tables:
             raise ValueError("bad fork")
         self.tables[child] = list(self.tables[parent])
         self.ntokens[child] = self.ntokens[parent]
@@ -161,8 +171,8 @@ class OracleAllocator:
 
     def append_slot(self, seq_id):
         """Slot for one new token; returns (slot, (src, dst) or None)."""
-        if seq_id not in self.tables:
-            raise ValueError("unknown sequence")
+        if seq_id not in self.tables or seq_id in self.on_host:
+            raise ValueError("unknown or swapped-out sequence")
         table = self.tables[seq_id]
         i = self.ntokens[seq_id]
         cow = None
@@ -187,7 +197,10 @@ class OracleAllocator:
 
     def append_slots(self, seq_ids):
         """One append per listed sequence in order, all or nothing: on OutOfBlocks
-        (or an unknown sequence) the allocator is left as it was."""
+        (or an unknown sequence) the allocator is left as it was.  Unknown or swapped-out
+        sequences are reported before any shortage of blocks."""
+        if any(s not in self.tables or s in self.on_host for s in seq_ids):
+            raise ValueError("unknown or swapped-out sequence")
         trial = copy.deepcopy(self)
         res = [trial.append_slot(s) for s in seq_ids]
         self.__dict__.update(trial.__dict__)
@@ -201,7 +214,7 @@ class OracleAllocator:
         Returns [(slot, (src, dst) or None)] per new beam."""
         beam_ids, new_ids = [int(b) for b in beam_ids], [int(b) for b in new_ids]
         parents = [int(p) for p in parents]
-        if len(set(beam_ids)) != len(beam_ids) or any(b not in self.tables for b in beam_ids):
+        if len(set(beam_ids)) != len(beam_ids) or any(b not in self.tables or b in self.on_host for b in beam_ids):
             raise ValueError("old beams unknown or repeated")
         if len(parents) != len(new_ids) or any(not 0 <= p < len(beam_ids) for p in parents):
             raise ValueError("bad parent index")
@@ -223,9 +236,51 @@ class OracleAllocator:
     def free_seq(self, seq_id):
         if seq_id not in self.tables:
             raise ValueError("unknown sequence")
-        for blk in self.tables.pop(seq_id):
-            self._release(blk)
+        if seq_id in self.on_host:
+            self.host_free.extend(self.tables.pop(seq_id))
+            self.on_host.discard(seq_id)
+        else:
+            for blk in self.tables.pop(seq_id):
+                self._release(blk)
         del self.ntokens[seq_id]
+
+    def add_host_pool(self, num_host_blocks):
+        if num_host_blocks <= 0 or self.num_host_blocks:
+            raise ValueError("bad host pool")
+        self.num_host_blocks = num_host_blocks
+        self.host_free = deque(range(num_host_blocks))
+
+    def swap_out(self, seq_id):
+        """Moves a resident sequence to host blocks; returns [(device, host)] in table order."""
+        if seq_id not in self.tables or seq_id in self.on_host:
+            raise ValueError("unknown or swapped-out sequence")
+        table = self.tables[seq_id]
+        if len(table) > len(self.host_free):
+            raise OutOfBlocks()
+        pairs = []
+        for i, blk in enumerate(table):
+            h = self.host_free.popleft()
+            pairs.append((blk, h))
+            self._release(blk)
+            table[i] = h
+        self.on_host.add(seq_id)
+        return pairs
+
+    def swap_in(self, seq_id):
+        """Brings a swapped-out sequence back to device blocks; returns [(host, device)]."""
+        if seq_id not in self.on_host:
+            raise ValueError("sequence is not swapped out")
+        table = self.tables[seq_id]
+        if len(table) > self.available():
+            raise OutOfBlocks()
+        pairs = []
+        for i, h in enumerate(table):
+            blk = self._take()
+            pairs.append((h, blk))
+            self.host_free.append(h)
+            table[i] = blk
+        self.on_host.discard(seq_id)
+        return pairs
 
     def block_table(self, seq_id):
         return list(self.tables[seq_id])

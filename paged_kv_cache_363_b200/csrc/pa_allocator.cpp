@@ -46,8 +46,9 @@ void set_error(const std::string& msg);
 
 struct pa_allocator {
     struct Seq {
-        std::vector<int32_t> table;
+        std::vector<int32_t> table;  // device blocks, or host blocks while swapped out
         int64_t tokens = 0;
+        bool on_host = false;
     };
     int32_t num_blocks = 0;
     int32_t block_size = 0;
@@ -63,6 +64,17 @@ struct pa_allocator {
     std::map<uint64_t, int32_t> lru;             // unreferenced cached blocks by release stamp
     std::vector<uint64_t> stamp;                 // per block: its key in lru
     uint64_t clock = 0;
+
+    // host tier for swapped-out sequences (0 blocks until pa_alloc_add_host_pool)
+    int32_t num_host_blocks = 0;
+    std::deque<int32_t> host_free;
+
+    // the sequence, if it exists and is resident on the device
+    Seq* resident(int64_t seq_id)
+    {
+        auto it = seqs.find(seq_id);
+        return it == seqs.end() || it->second.on_host ? nullptr : &it->second;
+    }
 
     bool cached(int32_t b) const { return !node_key[(size_t)b].empty(); }
     int64_t available() const { return (int64_t)free_q.size() + (int64_t)lru.size(); }
@@ -129,7 +141,7 @@ struct pa_allocator {
             auto it = st.find(seq_ids[k]);
             if (it == st.end()) {
                 auto q = seqs.find(seq_ids[k]);
-                if (q == seqs.end()) return -1;
+                if (q == seqs.end() || q->second.on_host) return -1;
                 it = st.emplace(seq_ids[k], std::make_pair(q->second.tokens,
                                                            q->second.table.empty() ? -1 : q->second.table.back()))
                          .first;
@@ -245,8 +257,8 @@ pa_status pa_alloc_fork(pa_allocator* a, int64_t parent_id, int64_t child_id)
 {
     if (!a) return PA_ERR_INVALID;
     auto it = a->seqs.find(parent_id);
-    if (it == a->seqs.end() || a->seqs.count(child_id)) {
-        pa::set_error("pa_alloc_fork: unknown parent or existing child");
+    if (it == a->seqs.end() || it->second.on_host || a->seqs.count(child_id)) {
+        pa::set_error("pa_alloc_fork: unknown or swapped-out parent, or existing child");
         return PA_ERR_INVALID;
     }
     pa_allocator::Seq child = it->second;
@@ -321,7 +333,7 @@ pa_status pa_alloc_append_slot(pa_allocator* a, int64_t seq_id, int64_t* slot_ou
     }
     const int64_t need = a->blocks_for_appends(&seq_id, 1);
     if (need < 0) {
-        pa::set_error("pa_alloc_append_slot: unknown sequence " + std::to_string(seq_id));
+        pa::set_error("pa_alloc_append_slot: unknown or swapped-out sequence " + std::to_string(seq_id));
         return PA_ERR_INVALID;
     }
     if (need > a->available()) {
@@ -346,8 +358,8 @@ pa_status pa_alloc_append_slots(pa_allocator* a, const int64_t* seq_ids, int n, 
     const int64_t need = a->blocks_for_appends(seq_ids, n);
     if (need < 0) {
         for (int k = 0; k < n; ++k)
-            if (!a->seqs.count(seq_ids[k])) {
-                pa::set_error("pa_alloc_append_slot: unknown sequence " + std::to_string(seq_ids[k]));
+            if (!a->resident(seq_ids[k])) {
+                pa::set_error("pa_alloc_append_slots: unknown or swapped-out sequence " + std::to_string(seq_ids[k]));
                 break;
             }
         return PA_ERR_INVALID;
@@ -381,8 +393,9 @@ pa_status pa_alloc_beam_step(pa_allocator* a, const int64_t* beam_ids, int num_b
     }
     std::unordered_map<int64_t, int> old_index;
     for (int i = 0; i < num_beams; ++i) {
-        if (!a->seqs.count(beam_ids[i]) || !old_index.emplace(beam_ids[i], i).second) {
-            pa::set_error("pa_alloc_beam_step: beam " + std::to_string(beam_ids[i]) + " unknown or listed twice");
+        if (!a->resident(beam_ids[i]) || !old_index.emplace(beam_ids[i], i).second) {
+            pa::set_error("pa_alloc_beam_step: beam " + std::to_string(beam_ids[i]) +
+                          " unknown, swapped out or listed twice");
             return PA_ERR_INVALID;
         }
     }
@@ -458,8 +471,87 @@ pa_status pa_alloc_free_seq(pa_allocator* a, int64_t seq_id)
         pa::set_error("pa_alloc_free_seq: unknown sequence " + std::to_string(seq_id));
         return PA_ERR_INVALID;
     }
-    for (int32_t b : it->second.table) a->drop_ref(b);
+    if (it->second.on_host) {
+        for (int32_t h : it->second.table) a->host_free.push_back(h);
+    } else {
+        for (int32_t b : it->second.table) a->drop_ref(b);
+    }
     a->seqs.erase(it);
+    return PA_OK;
+}
+
+pa_status pa_alloc_add_host_pool(pa_allocator* a, int num_host_blocks)
+{
+    if (!a || num_host_blocks <= 0 || a->num_host_blocks > 0) {
+        pa::set_error("pa_alloc_add_host_pool: bad argument or a host pool exists");
+        return PA_ERR_INVALID;
+    }
+    a->num_host_blocks = num_host_blocks;
+    for (int i = 0; i < num_host_blocks; ++i) a->host_free.push_back(i);
+    return PA_OK;
+}
+
+pa_status pa_alloc_swap_out(pa_allocator* a, int64_t seq_id, int64_t* pairs_out, int* num_pairs_out)
+{
+    if (!a || !num_pairs_out) {
+        pa::set_error("pa_alloc_swap_out: bad argument");
+        return PA_ERR_INVALID;
+    }
+    pa_allocator::Seq* q = a->resident(seq_id);
+    if (!q) {
+        pa::set_error("pa_alloc_swap_out: unknown or swapped-out sequence " + std::to_string(seq_id));
+        return PA_ERR_INVALID;
+    }
+    if (!q->table.empty() && !pairs_out) {
+        pa::set_error("pa_alloc_swap_out: pairs_out is null");
+        return PA_ERR_INVALID;
+    }
+    if (q->table.size() > a->host_free.size()) {
+        pa::set_error("pa_alloc_swap_out: out of host blocks");
+        return PA_ERR_OOM;
+    }
+    for (size_t i = 0; i < q->table.size(); ++i) {
+        const int32_t h = a->host_free.front();
+        a->host_free.pop_front();
+        pairs_out[2 * i] = q->table[i];
+        pairs_out[2 * i + 1] = h;
+        a->drop_ref(q->table[i]);
+        q->table[i] = h;
+    }
+    q->on_host = true;
+    *num_pairs_out = (int)q->table.size();
+    return PA_OK;
+}
+
+pa_status pa_alloc_swap_in(pa_allocator* a, int64_t seq_id, int64_t* pairs_out, int* num_pairs_out)
+{
+    if (!a || !num_pairs_out) {
+        pa::set_error("pa_alloc_swap_in: bad argument");
+        return PA_ERR_INVALID;
+    }
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end() || !it->second.on_host) {
+        pa::set_error("pa_alloc_swap_in: sequence " + std::to_string(seq_id) + " is not swapped out");
+        return PA_ERR_INVALID;
+    }
+    pa_allocator::Seq& q = it->second;
+    if (!q.table.empty() && !pairs_out) {
+        pa::set_error("pa_alloc_swap_in: pairs_out is null");
+        return PA_ERR_INVALID;
+    }
+    if ((int64_t)q.table.size() > a->available()) {
+        pa::set_error("pa_alloc_swap_in: out of blocks");
+        return PA_ERR_OOM;
+    }
+    for (size_t i = 0; i < q.table.size(); ++i) {
+        const int32_t b = a->take();
+        pairs_out[2 * i] = q.table[i];
+        pairs_out[2 * i + 1] = b;
+        a->host_free.push_back(q.table[i]);
+        q.table[i] = b;
+    }
+    q.on_host = false;
+    *num_pairs_out = (int)q.table.size();
     return PA_OK;
 }
 
@@ -490,8 +582,8 @@ pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq_ids, i
     }
     for (int k = 0; k < n; ++k) {
         auto it = a->seqs.find(seq_ids[k]);
-        if (it == a->seqs.end()) {
-            pa::set_error("pa_alloc_block_tables: unknown sequence " + std::to_string(seq_ids[k]));
+        if (it == a->seqs.end() || it->second.on_host) {
+            pa::set_error("pa_alloc_block_tables: unknown or swapped-out sequence " + std::to_string(seq_ids[k]));
             return PA_ERR_INVALID;
         }
         if ((int64_t)it->second.table.size() > max_blocks) {
@@ -518,6 +610,15 @@ int pa_alloc_num_free(const pa_allocator* a) { return a ? (int)a->free_q.size() 
 
 int pa_alloc_num_cached_free(const pa_allocator* a) { return a ? (int)a->lru.size() : -1; }
 
+int pa_alloc_num_host_free(const pa_allocator* a) { return a ? (int)a->host_free.size() : -1; }
+
+int pa_alloc_is_swapped(const pa_allocator* a, int64_t seq_id)
+{
+    if (!a) return -1;
+    auto it = a->seqs.find(seq_id);
+    return it == a->seqs.end() ? -1 : (it->second.on_host ? 1 : 0);
+}
+
 int pa_alloc_num_tokens(const pa_allocator* a, int64_t seq_id)
 {
     if (!a) return -1;
@@ -536,6 +637,9 @@ pa_status pa_alloc_stats(const pa_allocator* a, pa_alloc_stats_t* out)
     s.cow_copies = a->cow_copies;
     s.cached_blocks = (int64_t)a->tree.size();
     s.cached_free = (int64_t)a->lru.size();
+    s.host_blocks = a->num_host_blocks;
+    s.host_free = (int64_t)a->host_free.size();
+    for (const auto& kv : a->seqs) s.swapped_seqs += kv.second.on_host ? 1 : 0;
     for (const auto& kv : a->seqs) {
         s.tokens += kv.second.tokens;
         s.waste_tokens += (int64_t)kv.second.table.size() * a->block_size - kv.second.tokens;

@@ -284,6 +284,76 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapp
     return PA_OK;
 }
 
+// Address a kernel can use for p: device memory as is, pinned (page-locked) host
+// memory through its device mapping; anything else is refused.
+static pa_status kernel_address(const char* who, const char* what, const void* p, const void** out)
+{
+    cudaPointerAttributes at{};
+    const cudaError_t e = cudaPointerGetAttributes(&at, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        set_error(std::string(who) + ": cannot query " + what + ": " + cudaGetErrorString(e));
+        return PA_ERR_INVALID;
+    }
+    if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) {
+        *out = p;
+        return PA_OK;
+    }
+    if (at.type == cudaMemoryTypeHost && at.devicePointer) {
+        *out = at.devicePointer;
+        return PA_OK;
+    }
+    set_error(std::string(who) + ": " + what + " must be device memory or pinned host memory");
+    return PA_ERR_INVALID;
+}
+
+pa_status pa_swap_blocks(void* dst_k_cache, void* dst_v_cache, const void* src_k_cache, const void* src_v_cache,
+                         const int64_t* block_mapping, int num_pairs, int num_kv_heads, int head_dim, int block_size,
+                         int num_src_blocks, int num_dst_blocks, pa_dtype dtype, void* stream)
+{
+    pa_status st = check_common("pa_swap_blocks", num_kv_heads, head_dim, block_size, num_src_blocks, dtype);
+    if (st != PA_OK) return st;
+    if (num_dst_blocks <= 0) {
+        set_error("pa_swap_blocks: num_dst_blocks must be > 0");
+        return PA_ERR_INVALID;
+    }
+    if (num_pairs < 0 || num_pairs > 65535) {
+        set_error("pa_swap_blocks: num_pairs must be in [0, 65535]");
+        return PA_ERR_INVALID;
+    }
+    if (num_pairs == 0) return PA_OK;
+    if (!dst_k_cache || !dst_v_cache || !src_k_cache || !src_v_cache || !block_mapping) {
+        set_error("pa_swap_blocks: null pointer");
+        return PA_ERR_INVALID;
+    }
+    if (!aligned(dst_k_cache, 16) || !aligned(dst_v_cache, 16) || !aligned(src_k_cache, 16) ||
+        !aligned(src_v_cache, 16) || !aligned(block_mapping, 8)) {
+        set_error("pa_swap_blocks: misaligned pointer");
+        return PA_ERR_INVALID;
+    }
+    SwapArgs a{};
+    const void* p = nullptr;
+    if ((st = kernel_address("pa_swap_blocks", "dst_k_cache", dst_k_cache, &p)) != PA_OK) return st;
+    a.dst_k = const_cast<void*>(p);
+    if ((st = kernel_address("pa_swap_blocks", "dst_v_cache", dst_v_cache, &p)) != PA_OK) return st;
+    a.dst_v = const_cast<void*>(p);
+    if ((st = kernel_address("pa_swap_blocks", "src_k_cache", src_k_cache, &a.src_k)) != PA_OK) return st;
+    if ((st = kernel_address("pa_swap_blocks", "src_v_cache", src_v_cache, &a.src_v)) != PA_OK) return st;
+    if ((st = kernel_address("pa_swap_blocks", "block_mapping", block_mapping, &p)) != PA_OK) return st;
+    a.block_mapping = static_cast<const int64_t*>(p);
+    unsigned int* status = nullptr;
+    st = status_ptr(&status);
+    if (st != PA_OK) return st;
+    a.status = status;
+    a.num_pairs = num_pairs;
+    a.num_src_blocks = num_src_blocks;
+    a.num_dst_blocks = num_dst_blocks;
+    a.block_bytes = (size_t)num_kv_heads * block_size * head_dim * elt_bytes(dtype);
+    const cudaError_t e = launch_swap_blocks(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail("pa_swap_blocks launch", e);
+    return PA_OK;
+}
+
 pa_status pa_device_status(uint32_t* flags, void* stream)
 {
     if (!flags) return PA_ERR_INVALID;

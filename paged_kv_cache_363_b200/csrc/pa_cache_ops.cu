@@ -6,6 +6,9 @@
 // copy_blocks: the copy-on-write block copy ("PagedAttention and vLLM
 // Architecture", section 3): a shared block about to be written is duplicated
 // into a fresh block before the write.
+// swap_blocks: whole blocks between a device pool and a pinned host pool
+// ("PagedAttention Paper Breakdown", "Engineering Limitations": CPU-GPU block
+// swapping under memory pressure).
 //
 // Both are pure data movement, bounded by HBM bandwidth: every thread moves
 // 16-byte vectors, consecutive threads cover consecutive bytes of a row (or of a
@@ -80,6 +83,37 @@ __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(const CopyArg
     }
 }
 
+// Block swap between a device pool and a pinned host pool (either direction), the
+// host side reached through its device mapping over PCIe.  Same tiling as the
+// copy-on-write copy; plain loads and stores (the host side is not read-only cached).
+__global__ void __launch_bounds__(kCopyThreads) swap_blocks_kernel(const SwapArgs a)
+{
+    const int pair = blockIdx.y;
+    const int64_t src = a.block_mapping[2 * pair];
+    const int64_t dst = a.block_mapping[2 * pair + 1];
+    if (src < 0 || dst < 0 || src >= a.num_src_blocks || dst >= a.num_dst_blocks) {
+        if (blockIdx.x == 0 && blockIdx.z == 0 && threadIdx.x == 0) atomicOr(a.status, PA_DEV_BAD_PAIR);
+        return;
+    }
+    const char* sp = static_cast<const char*>(blockIdx.z == 0 ? a.src_k : a.src_v);
+    char* dp = static_cast<char*>(blockIdx.z == 0 ? a.dst_k : a.dst_v);
+    const uint4* s = reinterpret_cast<const uint4*>(sp + (size_t)src * a.block_bytes);
+    uint4* d = reinterpret_cast<uint4*>(dp + (size_t)dst * a.block_bytes);
+    const int64_t nvec = (int64_t)(a.block_bytes / 16);
+    const int64_t base = (int64_t)blockIdx.x * kCopyThreads * kCopyVec + threadIdx.x;
+    uint4 buf[kCopyVec];
+#pragma unroll
+    for (int k = 0; k < kCopyVec; ++k) {
+        const int64_t i = base + (int64_t)k * kCopyThreads;
+        if (i < nvec) buf[k] = s[i];
+    }
+#pragma unroll
+    for (int k = 0; k < kCopyVec; ++k) {
+        const int64_t i = base + (int64_t)k * kCopyThreads;
+        if (i < nvec) d[i] = buf[k];
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_reshape_and_cache(const ReshapeArgs& a, int elt_bytes, int head_dim, int block_size,
@@ -107,6 +141,16 @@ cudaError_t launch_copy_blocks(const CopyArgs& a, cudaStream_t stream)
     const int64_t per_cta = (int64_t)kCopyThreads * kCopyVec;
     dim3 grid((unsigned)((nvec + per_cta - 1) / per_cta), (unsigned)a.num_pairs, 2);
     copy_blocks_kernel<<<grid, kCopyThreads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_swap_blocks(const SwapArgs& a, cudaStream_t stream)
+{
+    if (a.num_pairs == 0) return cudaSuccess;
+    const int64_t nvec = (int64_t)(a.block_bytes / 16);
+    const int64_t per_cta = (int64_t)kCopyThreads * kCopyVec;
+    dim3 grid((unsigned)((nvec + per_cta - 1) / per_cta), (unsigned)a.num_pairs, 2);
+    swap_blocks_kernel<<<grid, kCopyThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

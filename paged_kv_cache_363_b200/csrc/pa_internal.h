@@ -100,4 +100,21 @@ struct CopyArgs {
 
 cudaError_t launch_copy_blocks(const CopyArgs& a, cudaStream_t stream);
 
+// Whole-block copies between two pools, either of which may be pinned host memory
+// (addressed through its device mapping).
+struct SwapArgs {
+    void* dst_k;
+    void* dst_v;
+    const void* src_k;
+    const void* src_v;
+    const int64_t* block_mapping;  // [num_pairs][2] (src block, dst block)
+    unsigned int* status;
+    int num_pairs;
+    int num_src_blocks;
+    int num_dst_blocks;
+    size_t block_bytes;
+};
+
+cudaError_t launch_swap_blocks(const SwapArgs& a, cudaStream_t stream);
+
 }  // namespace pa

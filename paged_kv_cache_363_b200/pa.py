@@ -28,7 +28,8 @@ _u32 = ctypes.c_uint32
 
 class pa_alloc_stats_t(ctypes.Structure):
     _fields_ = [(n, _i64) for n in ("num_blocks", "num_free", "num_seqs", "shared_blocks", "cow_copies",
-                                   "tokens", "waste_tokens", "cached_blocks", "cached_free")]
+                                   "tokens", "waste_tokens", "cached_blocks", "cached_free", "host_blocks",
+                                   "host_free", "swapped_seqs")]
 
 
 # (name, restype, argtypes) of every symbol declared in include/pa.h
@@ -39,6 +40,7 @@ SIGNATURES = [
     ("pa_decode_static_workspace", _int, [_vp, _vp, _vp, _vp, _vp, _vp] + [_int] * 8 + [_f32, _int, _int, _vp]),
     ("pa_reshape_and_cache", _int, [_vp, _vp, _vp, _vp, _vp] + [_int] * 6 + [_vp]),
     ("pa_copy_blocks", _int, [_vp, _vp, _vp] + [_int] * 6 + [_vp]),
+    ("pa_swap_blocks", _int, [_vp, _vp, _vp, _vp, _vp] + [_int] * 7 + [_vp]),
     ("pa_device_status", _int, [ctypes.POINTER(_u32), _vp]),
     ("pa_alloc_create", _vp, [_int, _int, _vp]),
     ("pa_alloc_destroy", None, [_vp]),
@@ -49,6 +51,11 @@ SIGNATURES = [
     ("pa_alloc_append_slots", _int, [_vp, _vp, _int, _vp, _vp, ctypes.POINTER(_int)]),
     ("pa_alloc_beam_step", _int, [_vp, _vp, _int, _vp, _vp, _int, _vp, _vp, ctypes.POINTER(_int)]),
     ("pa_alloc_free_seq", _int, [_vp, _i64]),
+    ("pa_alloc_add_host_pool", _int, [_vp, _int]),
+    ("pa_alloc_swap_out", _int, [_vp, _i64, _vp, ctypes.POINTER(_int)]),
+    ("pa_alloc_swap_in", _int, [_vp, _i64, _vp, ctypes.POINTER(_int)]),
+    ("pa_alloc_num_host_free", _int, [_vp]),
+    ("pa_alloc_is_swapped", _int, [_vp, _i64]),
     ("pa_alloc_block_table", _int, [_vp, _i64, _vp, _int, ctypes.POINTER(_int)]),
     ("pa_alloc_block_tables", _int, [_vp, _vp, _int, _vp, _int, _i32, _vp]),
     ("pa_alloc_ref_count", _int, [_vp, _i32]),
@@ -95,6 +102,15 @@ def _dtype_code(t):
 def _dev_ptr(t, name):
     if not t.is_cuda:
         raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    return t.data_ptr()
+
+
+def _pool_ptr(t, name):
+    """A CUDA tensor, or a pinned CPU tensor (the library maps it), contiguous."""
+    if not (t.is_cuda or t.is_pinned()):
+        raise ValueError("%s must be a CUDA tensor or pinned host memory" % name)
     if not t.is_contiguous():
         raise ValueError("%s must be contiguous" % name)
     return t.data_ptr()
@@ -190,6 +206,24 @@ def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None
                                   _dev_ptr(v_cache, "v_cache"), _dev_ptr(slot_mapping, "slot_mapping"), N, Hkv, D,
                                   B, NB, dt, _stream(stream))
     _check(st, "pa_reshape_and_cache")
+
+
+def pa_swap_blocks(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache, block_mapping, stream=None):
+    """For every (src, dst) row of block_mapping[n, 2] (int64): dst pools[dst] <- src pools[src].
+    Pools and block_mapping may be CUDA tensors or pinned CPU tensors."""
+    import torch
+    NBs, Hkv, B, D = src_k_cache.shape
+    NBd = dst_k_cache.shape[0]
+    if tuple(dst_k_cache.shape[1:]) != (Hkv, B, D) or dst_k_cache.dtype != src_k_cache.dtype:
+        raise ValueError("pools differ in block shape or dtype")
+    if block_mapping.dtype != torch.int64 or (block_mapping.numel() and block_mapping.shape[-1] != 2):
+        raise TypeError("block_mapping must be int64 [n, 2]")
+    n = block_mapping.numel() // 2
+    ptr = _pool_ptr(block_mapping, "block_mapping") if n else None
+    st = lib.pa_swap_blocks(_pool_ptr(dst_k_cache, "dst_k_cache"), _pool_ptr(dst_v_cache, "dst_v_cache"),
+                            _pool_ptr(src_k_cache, "src_k_cache"), _pool_ptr(src_v_cache, "src_v_cache"), ptr, n,
+                            Hkv, D, B, NBs, NBd, _dtype_code(src_k_cache), _stream(stream))
+    _check(st, "pa_swap_blocks")
 
 
 def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None):
@@ -295,6 +329,30 @@ class Allocator:
 
     def free_seq(self, seq_id):
         _check(lib.pa_alloc_free_seq(self._h, int(seq_id)), "pa_alloc_free_seq")
+
+    def add_host_pool(self, num_host_blocks):
+        _check(lib.pa_alloc_add_host_pool(self._h, int(num_host_blocks)), "pa_alloc_add_host_pool")
+
+    def _swap(self, fn, name, seq_id):
+        cap = max(1, len(self.block_table(seq_id)))
+        pairs = np.empty((cap, 2), np.int64)
+        n = _int(0)
+        _check(fn(self._h, int(seq_id), _np_ptr(pairs), ctypes.byref(n)), name)
+        return pairs[:n.value]
+
+    def swap_out(self, seq_id):
+        """Moves the sequence to the host tier; returns its (device, host) block pairs."""
+        return self._swap(lib.pa_alloc_swap_out, "pa_alloc_swap_out", seq_id)
+
+    def swap_in(self, seq_id):
+        """Brings the sequence back; returns its (host, device) block pairs."""
+        return self._swap(lib.pa_alloc_swap_in, "pa_alloc_swap_in", seq_id)
+
+    def num_host_free(self):
+        return int(lib.pa_alloc_num_host_free(self._h))
+
+    def is_swapped(self, seq_id):
+        return int(lib.pa_alloc_is_swapped(self._h, int(seq_id)))
 
     def block_table(self, seq_id):
         n = _int(0)

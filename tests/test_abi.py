@@ -82,10 +82,13 @@ def test_partition_and_workspace_sizes():
     assert pa.pa_decode_workspace_size(0, 32, 8, 128, 32, 32768, 512) == 0
 
 
-def _replay(ops, NB, B, order):
+def _replay(ops, NB, B, order, NH=0):
     """Run the same script on the library allocator and the oracle allocator."""
     lib_a = pa.Allocator(NB, B, order)
     ora = OracleAllocator(NB, B, order)
+    if NH:
+        lib_a.add_host_pool(NH)
+        ora.add_host_pool(NH)
     for op in ops:
         kind = op[0]
         if kind == "add":
@@ -140,18 +143,30 @@ def _replay(ops, NB, B, order):
         elif kind == "free":
             ora.free_seq(op[1])
             lib_a.free_seq(op[1])
+        elif kind in ("swapout", "swapin"):
+            fo, fl = (ora.swap_out, lib_a.swap_out) if kind == "swapout" else (ora.swap_in, lib_a.swap_in)
+            try:
+                want = fo(op[1])
+            except OracleOOM:
+                with pytest.raises(pa.OutOfBlocks):
+                    fl(op[1])
+                continue
+            assert [tuple(p) for p in fl(op[1]).tolist()] == want
         # full state comparison after every op
         assert lib_a.num_free() == ora.num_free()
         assert lib_a.num_cached_free() == ora.num_cached_free()
         for b in range(NB):
             assert lib_a.ref_count(b) == ora.ref[b]
+        assert lib_a.num_host_free() == len(ora.host_free)
         for sid in ora.tables:
             assert lib_a.block_table(sid) == ora.block_table(sid)
             assert lib_a.num_tokens(sid) == ora.ntokens[sid]
+            assert lib_a.is_swapped(sid) == (1 if sid in ora.on_host else 0)
     st = lib_a.stats()
     assert st["cow_copies"] == ora.cow_count
     assert st["cached_blocks"] == len(ora.tree) and st["cached_free"] == ora.num_cached_free()
     assert st["waste_tokens"] == sum(ora.waste_tokens(s) for s in ora.tables)
+    assert st["host_free"] == len(ora.host_free) and st["swapped_seqs"] == len(ora.on_host)
     return lib_a, ora
 
 
@@ -159,8 +174,9 @@ def _replay(ops, NB, B, order):
 def test_allocator_matches_oracle_on_random_scripts(seed):
     rng = np.random.default_rng(seed)
     NB, B = int(rng.integers(20, 80)), int(rng.choice([4, 16]))
+    NH = int(rng.integers(5, 40))
     order = rng.permutation(NB)
-    ops, live, nxt = [], [], 0
+    ops, live, nxt, swapped = [], [], 0, []
     # prompts for the prefix cache: a few shared stems over a tiny vocabulary, so that
     # full blocks repeat, prefixes diverge part-way and evictions happen
     stems = [rng.integers(0, 3, size=int(rng.integers(B, 5 * B))).tolist() for _ in range(3)]
@@ -183,6 +199,13 @@ def test_allocator_matches_oracle_on_random_scripts(seed):
             nxt += 1
         elif r < 0.7:
             ops.append(("append", int(rng.choice(live))))
+        elif r < 0.74:
+            if swapped and rng.random() < 0.5:
+                ops.append(("swapin", swapped.pop(int(rng.integers(0, len(swapped))))))
+            else:
+                sid = int(rng.choice(live))
+                ops.append(("swapout", sid))
+                swapped.append(sid)
         elif r < 0.78:
             k = int(rng.integers(1, len(live) + 1))
             ops.append(("batch", [int(x) for x in rng.choice(live, size=k, replace=False)]))
@@ -206,60 +229,26 @@ def test_allocator_matches_oracle_on_random_scripts(seed):
             sid = int(rng.choice(live))
             ops.append(("free", sid))
             live.remove(sid)
-    # failing adds never create the sequence: drop later ops on it by replaying defensively
-    lib_a, ora = None, None
-    clean, known = [], set()
+    # replay on the oracle alone: keep ops that succeed or run out of blocks, drop the
+    # ones it rejects as invalid (unknown, freed or swapped-out sequences)
+    clean = []
     sim = OracleAllocator(NB, B, order)
+    sim.add_host_pool(NH)
     for op in ops:
-        if op[0] == "add":
-            try:
-                sim.add_seq(op[1], op[2])
-                known.add(op[1])
-            except OracleOOM:
-                pass
-            clean.append(op)
-        elif op[0] == "fork":
-            if op[1] in known:
-                sim.fork(op[1], op[2])
-                known.add(op[2])
-                clean.append(op)
-        elif op[0] == "append":
-            if op[1] in known:
-                try:
-                    sim.append_slot(op[1])
-                except OracleOOM:
-                    pass
-                clean.append(op)
-        elif op[0] == "cached":
-            try:
-                sim.add_seq_cached(op[1], op[2])
-                known.add(op[1])
-            except OracleOOM:
-                pass
-            clean.append(op)
-        elif op[0] == "beam":
-            if all(b in known for b in op[1]):
-                try:
-                    sim.beam_step(op[1], op[2], op[3])
-                    known.difference_update(op[1])
-                    known.update(op[3])
-                except OracleOOM:
-                    pass
-                clean.append(op)
-        elif op[0] == "batch":
-            ids = [s for s in op[1] if s in known]
-            if ids:
-                try:
-                    sim.append_slots(ids)
-                except OracleOOM:
-                    pass
-                clean.append(("batch", ids))
-        elif op[0] == "free":
-            if op[1] in known:
-                sim.free_seq(op[1])
-                known.discard(op[1])
-                clean.append(op)
-    _replay(clean, NB, B, order)
+        kind = op[0]
+        fn = {"add": lambda: sim.add_seq(op[1], op[2]), "cached": lambda: sim.add_seq_cached(op[1], op[2]),
+              "fork": lambda: sim.fork(op[1], op[2]), "append": lambda: sim.append_slot(op[1]),
+              "batch": lambda: sim.append_slots(op[1]), "free": lambda: sim.free_seq(op[1]),
+              "beam": lambda: sim.beam_step(op[1], op[2], op[3]), "swapout": lambda: sim.swap_out(op[1]),
+              "swapin": lambda: sim.swap_in(op[1])}[kind]
+        try:
+            fn()
+        except OracleOOM:
+            pass
+        except (ValueError, KeyError):
+            continue
+        clean.append(op)
+    _replay(clean, NB, B, order, NH)
 
 
 def test_allocator_argument_errors():

@@ -369,3 +369,92 @@ def test_beam_step_out_of_blocks_changes_nothing():
         a.beam_step(beams, [0, 2], [5, 6])
     with pytest.raises(ValueError):
         a.beam_step(beams, [0, 1], [9, 6])         # 9 is held by a sequence outside the beams
+
+
+# ---------------------------------------------------------------- swapping
+# [fullstackaihub] "Engineering Limitations": CPU-GPU block swapping under memory pressure.
+
+def test_swap_out_releases_device_blocks_and_swap_in_restores_the_sequence():
+    a = OracleAllocator(16, 4)
+    a.add_host_pool(8)
+    a.add_seq(0, 10)                               # 3 blocks
+    t = a.block_table(0)
+    free0 = a.num_free()
+    pairs = a.swap_out(0)
+    assert [d for d, _ in pairs] == t and [h for _, h in pairs] == [0, 1, 2]     # host FIFO, table order
+    assert a.num_free() == free0 + 3 and all(a.ref[b] == 0 for b in t)
+    assert a.block_table(0) == [0, 1, 2] and 0 in a.on_host and len(a.host_free) == 5
+    with pytest.raises(ValueError):
+        a.append_slot(0)
+    with pytest.raises(ValueError):
+        a.fork(0, 1)
+    back = a.swap_in(0)
+    assert [h for h, _ in back] == [0, 1, 2] and len(a.host_free) == 8
+    assert a.block_table(0) == [d for _, d in back] and all(a.ref[b] == 1 for b in a.block_table(0))
+    assert a.ntokens[0] == 10 and a.append_slot(0)[1] is None
+
+
+def test_swapping_out_one_sharer_leaves_the_shared_blocks_to_the_other():
+    a = OracleAllocator(16, 4)
+    a.add_host_pool(8)
+    a.add_seq(0, 6)
+    a.fork(0, 1)
+    shared = a.block_table(0)
+    a.swap_out(1)
+    assert a.block_table(0) == shared and all(a.ref[b] == 1 for b in shared)
+    assert a.append_slot(0)[1] is None             # the remaining stream owns the block now: no copy
+
+
+def test_swap_round_trip_keeps_the_attention_output():
+    """Swap half the sequences out, let other sequences reuse the freed device blocks,
+    swap back in: decode over the returned tables equals decode before the swap."""
+    rng = np.random.default_rng(8)
+    B, Hkv, D, NB, NH = 4, 2, 8, 40, 32
+    a = OracleAllocator(NB, B, free_order=rng.permutation(NB))
+    a.add_host_pool(NH)
+    kc = rng.standard_normal((NB, Hkv, B, D)).astype(np.float32)
+    vc = rng.standard_normal((NB, Hkv, B, D)).astype(np.float32)
+    kh = np.zeros((NH, Hkv, B, D), np.float32)
+    vh = np.zeros((NH, Hkv, B, D), np.float32)
+    lens = [9, 14, 3, 11]
+    for s, L in enumerate(lens):
+        a.add_seq(s, L)
+    q = rng.standard_normal((4, Hkv, D)).astype(np.float32)
+
+    def run():
+        mb = max(len(a.block_table(s)) for s in range(4))
+        tab = np.array([a.block_table(s) + [-1] * (mb - len(a.block_table(s))) for s in range(4)], np.int32)
+        return oracle.decode(q, kc, vc, tab, np.array(lens, np.int32), 0.3)
+
+    before = run()
+    for s in (1, 3):
+        for d, h in a.swap_out(s):
+            kh[h], vh[h] = kc[d], vc[d]
+    a.add_seq(9, 4 * (a.num_free() - 3))           # another sequence takes (and overwrites) freed blocks
+    for b in a.block_table(9):
+        kc[b] = 7.0
+        vc[b] = -7.0
+    a.free_seq(9)
+    for s in (3, 1):
+        for h, d in a.swap_in(s):
+            kc[d], vc[d] = kh[h], vh[h]
+    assert np.array_equal(run(), before)
+
+
+def test_swap_out_of_blocks_changes_nothing():
+    a = OracleAllocator(8, 4)
+    a.add_host_pool(2)
+    a.add_seq(0, 12)                               # 3 blocks, host has 2
+    before = (_state(a), list(a.host_free), set(a.on_host))
+    with pytest.raises(OutOfBlocks):
+        a.swap_out(0)
+    assert (_state(a), list(a.host_free), set(a.on_host)) == before
+    b = OracleAllocator(4, 4)
+    b.add_host_pool(4)
+    b.add_seq(0, 12)
+    b.swap_out(0)
+    b.add_seq(1, 13)                               # all 4 device blocks
+    before = (_state(b), list(b.host_free), set(b.on_host))
+    with pytest.raises(OutOfBlocks):
+        b.swap_in(0)
+    assert (_state(b), list(b.host_free), set(b.on_host)) == before

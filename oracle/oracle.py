@@ -39,6 +39,9 @@ def lib():
         L.oracle_reshape_and_cache.argtypes = [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int]
         L.oracle_copy_blocks.restype = c_int
         L.oracle_copy_blocks.argtypes = [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int]
+        L.oracle_prefill.restype = c_int
+        L.oracle_prefill.argtypes = [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int,
+                                     c_int, ctypes.c_double, c_int]
         del c_i32
         _lib = L
     return _lib
@@ -138,6 +141,29 @@ def copy_blocks(k_cache, v_cache, block_mapping):
     if rc != 0:
         raise ValueError("oracle_copy_blocks: block index out of range")
     return kc, vc
+
+
+def prefill(q, k_cache, v_cache, block_tables, context_lens, q_start, scale, nthreads=1):
+    """fp64 chunked-prefill attention: query i of sequence s (row q_start[s] + i of
+    q [Nq, Hq, D]) sits at position context_lens[s] - n_s + i and attends to tokens
+    0..that position through the block table.  Returns out [Nq, Hq, D] float64."""
+    q = _c(q, np.float32)
+    k = _c(k_cache, np.float32)
+    v = _c(v_cache, np.float32)
+    T = _c(block_tables, np.int32)
+    Ls = _c(context_lens, np.int32)
+    qs = _c(q_start, np.int32)
+    Nq, Hq, D = q.shape
+    NB, Hkv, B, D2 = k.shape
+    S = Ls.shape[0]
+    assert D2 == D and v.shape == k.shape and qs.shape == (S + 1,) and int(qs[-1]) == Nq
+    MB = T.shape[1] if T.ndim == 2 else 0
+    out = np.zeros((Nq, Hq, D), np.float64)
+    rc = lib().oracle_prefill(_ptr(out), _ptr(q), _ptr(k), _ptr(v), _ptr(T), _ptr(Ls), _ptr(qs), S, Hq, Hkv, D,
+                              B, MB, float(scale), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_prefill rejected its arguments")
+    return out
 
 
 def decode_bruteforce(q, k_cache, v_cache, block_tables, context_lens, scale):

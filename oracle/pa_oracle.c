@@ -257,3 +257,101 @@ int oracle_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mappin
     }
     return 0;
 }
+
+/*
+ * Chunked prefill over the paged cache (the multi-token case of the same
+ * attention: [INIT] section 3 "When a prompt is processed" assigns the prompt's
+ * blocks; the new tokens' K/V are in the pools before the call, as for decode).
+ * Sequence s holds L_s = context_lens[s] tokens, of which the last
+ * n_s = q_start[s+1] - q_start[s] are queries: query i of s sits at position
+ * p = L_s - n_s + i and attends causally to tokens 0..p, i.e. it is the decode
+ * attention of that row with context length p + 1.  q and out are packed by
+ * q_start: row q_start[s] + i, head h.  Plain loops, fp64; nothing is shared
+ * with the decode function above except the address translation.
+ */
+struct prefill_job {
+    double* out;                 /* [Nq][Hq][D] */
+    const float* q;              /* [Nq][Hq][D] */
+    const float* k_cache;
+    const float* v_cache;
+    const int32_t* block_tables; /* [S][MB] */
+    const int32_t* context_lens; /* [S] */
+    const int32_t* q_start;      /* [S+1] */
+    int S, Hq, Hkv, D, B, MB;
+    double scale;
+    int nthreads, tid;
+};
+
+static void prefill_row(const struct prefill_job* j, int s, int i, int h)
+{
+    const int D = j->D;
+    const int kvh = h / (j->Hq / j->Hkv);
+    const int n = j->q_start[s + 1] - j->q_start[s];
+    const int64_t row = (int64_t)j->q_start[s] + i;
+    const int p = j->context_lens[s] - n + i;          /* position of this query token */
+    const float* q = j->q + ((size_t)row * j->Hq + h) * D;
+    const int32_t* T = j->block_tables + (size_t)s * j->MB;
+    double* out = j->out + ((size_t)row * j->Hq + h) * D;
+    for (int d = 0; d < D; ++d) out[d] = 0.0;
+    const int L = p + 1;                                /* tokens 0..p */
+    if (L <= 0) return;
+    double* z = (double*)malloc(sizeof(double) * (size_t)L);
+    double zmax = -INFINITY;
+    for (int t = 0; t < L; ++t) {
+        const float* k = j->k_cache + pool_row(oracle_physical_slot(T, j->B, t), kvh, j->Hkv, j->B, D);
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += (double)q[d] * (double)k[d];
+        z[t] = j->scale * dot;
+        if (z[t] > zmax) zmax = z[t];
+    }
+    double denom = 0.0;
+    for (int t = 0; t < L; ++t) denom += exp(z[t] - zmax);
+    for (int t = 0; t < L; ++t) {
+        const double w = exp(z[t] - zmax) / denom;
+        const float* v = j->v_cache + pool_row(oracle_physical_slot(T, j->B, t), kvh, j->Hkv, j->B, D);
+        for (int d = 0; d < D; ++d) out[d] += w * (double)v[d];
+    }
+    free(z);
+}
+
+static void* prefill_worker(void* arg)
+{
+    const struct prefill_job* j = (const struct prefill_job*)arg;
+    const int64_t rows = j->q_start[j->S];
+    int64_t u = 0;
+    for (int s = 0; s < j->S; ++s)
+        for (int i = 0; i < j->q_start[s + 1] - j->q_start[s]; ++i)
+            for (int h = 0; h < j->Hq; ++h, ++u)
+                if (u % j->nthreads == j->tid) prefill_row(j, s, i, h);
+    (void)rows;
+    return NULL;
+}
+
+/* Returns 0, or -1 on a bad argument (a sequence with more queries than tokens,
+ * a context beyond its table, q_start not non-decreasing). */
+int oracle_prefill(double* out, const float* q, const float* k_cache, const float* v_cache,
+                   const int32_t* block_tables, const int32_t* context_lens, const int32_t* q_start, int S, int Hq,
+                   int Hkv, int D, int B, int MB, double scale, int nthreads)
+{
+    if (S < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || D <= 0 || B <= 0 || MB < 0 || q_start[0] != 0) return -1;
+    for (int s = 0; s < S; ++s) {
+        const int n = q_start[s + 1] - q_start[s];
+        if (n < 0 || n > context_lens[s] || context_lens[s] > (int64_t)MB * B) return -1;
+    }
+    if (nthreads < 1) nthreads = 1;
+    struct prefill_job* jobs = (struct prefill_job*)calloc((size_t)nthreads, sizeof(struct prefill_job));
+    pthread_t* th = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+    for (int t = 0; t < nthreads; ++t) {
+        struct prefill_job* j = &jobs[t];
+        j->out = out; j->q = q; j->k_cache = k_cache; j->v_cache = v_cache;
+        j->block_tables = block_tables; j->context_lens = context_lens; j->q_start = q_start;
+        j->S = S; j->Hq = Hq; j->Hkv = Hkv; j->D = D; j->B = B; j->MB = MB;
+        j->scale = scale; j->nthreads = nthreads; j->tid = t;
+    }
+    for (int t = 1; t < nthreads; ++t) pthread_create(&th[t], NULL, prefill_worker, &jobs[t]);
+    prefill_worker(&jobs[0]);
+    for (int t = 1; t < nthreads; ++t) pthread_join(th[t], NULL);
+    free(jobs);
+    free(th);
+    return 0;
+}

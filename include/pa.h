@@ -196,6 +196,29 @@ PA_API pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* blo
 PA_API pa_status pa_device_status(uint32_t* flags, void* stream);
 
 /*
+ * Chunked prefill over the paged cache ([INIT] section 3: a prompt's blocks are
+ * assigned when it is processed; [FSAH] section 2: token t of a sequence lives at
+ * slot T[t / B] * B + t % B), on the tensor cores.  Sequence s holds
+ * context_lens[s] tokens in the pools, its new tokens already appended (as for
+ * pa_decode); its last n_s = q_start[s+1] - q_start[s] tokens are the queries:
+ * q rows q_start[s] .. q_start[s+1]-1 of q [num_query_tokens][num_heads][head_dim],
+ * query i at position context_lens[s] - n_s + i.  Each attends causally to tokens
+ * 0..its position: out[row][h] = softmax_t(scale * q[row][h] . K_t) . V_t over
+ * t <= position, with query head h reading kv head h / (num_heads / num_kv_heads).
+ * q_start (device, int32, S+1 entries, q_start[0] = 0, non-decreasing) and
+ * context_lens are device arrays; max_query_len bounds every n_s (it sizes the grid:
+ * larger n_s leave rows unwritten).  A sequence with n_s > context_lens[s] or a
+ * context beyond its table raises PA_DEV_BAD_CONTEXT and is skipped.  bf16 only,
+ * head_dim 128, num_heads / num_kv_heads in {1, 2, 4, 8} (else PA_ERR_UNSUPPORTED).
+ * With every n_s = 1 this is pa_decode.  No workspace.  Asynchronous on stream.
+ */
+PA_API pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, const int32_t* context_lens, const int32_t* q_start,
+                            int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                            int max_blocks_per_seq, int num_blocks, int num_query_tokens, int max_query_len,
+                            float scale, pa_dtype dtype, void* stream);
+
+/*
  * Whole-block copies from one pool to another ([FSAH] "Engineering Limitations":
  * CPU-GPU block swapping under memory pressure): for each (src, dst) pair in
  * block_mapping[num_pairs][2] (int64), block src of src_k_cache / src_v_cache

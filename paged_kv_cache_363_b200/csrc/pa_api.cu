@@ -284,6 +284,66 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapp
     return PA_OK;
 }
 
+pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                     const int32_t* context_lens, const int32_t* q_start, int num_seqs, int num_heads,
+                     int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+                     int num_query_tokens, int max_query_len, float scale, pa_dtype dtype, void* stream)
+{
+    pa_status st = check_common("pa_prefill", num_kv_heads, head_dim, block_size, num_blocks, dtype);
+    if (st != PA_OK) return st;
+    if (dtype != PA_DTYPE_BF16 || head_dim != 128) {
+        set_error("pa_prefill: bf16 with head_dim 128 only (the tensor-core tile)");
+        return PA_ERR_UNSUPPORTED;
+    }
+    if (num_seqs < 0 || num_seqs > 65535 || num_heads <= 0 || num_heads % num_kv_heads != 0 ||
+        num_query_tokens < 0 || max_query_len < 0 || max_blocks_per_seq < 0 || !(scale == scale) ||
+        scale == INFINITY || scale == -INFINITY) {
+        set_error("pa_prefill: bad sizes or scale");
+        return PA_ERR_INVALID;
+    }
+    const int group = num_heads / num_kv_heads;
+    if (group != 1 && group != 2 && group != 4 && group != 8) {
+        set_error("pa_prefill: num_heads / num_kv_heads must be 1, 2, 4 or 8");
+        return PA_ERR_UNSUPPORTED;
+    }
+    if (num_seqs == 0 || num_query_tokens == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !q_start) {
+        set_error("pa_prefill: null pointer");
+        return PA_ERR_INVALID;
+    }
+    if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16)) {
+        set_error("pa_prefill: misaligned pointer (q, out, caches need 16 bytes)");
+        return PA_ERR_INVALID;
+    }
+    if ((int64_t)num_blocks * num_kv_heads * block_size > (int64_t)INT32_MAX) {
+        set_error("pa_prefill: num_blocks * num_kv_heads * block_size must stay below 2^31 (tensor-copy row index)");
+        return PA_ERR_UNSUPPORTED;
+    }
+    unsigned int* status = nullptr;
+    st = status_ptr(&status);
+    if (st != PA_OK) return st;
+    PrefillArgs a{};
+    a.out = out;
+    a.q = q;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.q_start = q_start;
+    a.status = status;
+    a.num_seqs = num_seqs;
+    a.num_heads = num_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.num_blocks = num_blocks;
+    a.block_size = block_size;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    const cudaError_t e =
+        launch_prefill(a, group, num_query_tokens, max_query_len, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail("pa_prefill launch", e);
+    return PA_OK;
+}
+
 // Address a kernel can use for p: device memory as is, pinned (page-locked) host
 // memory through its device mapping; anything else is refused.
 static pa_status kernel_address(const char* who, const char* what, const void* p, const void** out)

@@ -50,6 +50,72 @@
 
 namespace pa {
 
+// ---------------------------------------------------------------- tensor maps
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// The pool [num_blocks][kv_heads][B][D] as a 2-D bf16 tensor of rows of D elements;
+// boxes of 64 columns x `B` rows (one stage tile), 128-byte swizzle.  A small cache avoids re-encoding
+// the maps of the same pools on every call.
+cudaError_t tensor_map(CUtensorMap* out, const void* pool, uint64_t rows, int D, int B)
+{
+    struct Entry {
+        const void* ptr;
+        uint64_t rows;
+        int d, b, dev;
+        CUtensorMap map;
+    };
+    static std::mutex mu;
+    static Entry cache[16] = {};
+    static int next = 0;
+    int dev = 0;
+    cudaError_t ce = cudaGetDevice(&dev);
+    if (ce != cudaSuccess) return ce;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        for (auto& en : cache)
+            if (en.ptr == pool && en.rows == rows && en.d == D && en.b == B && en.dev == dev) {
+                *out = en.map;
+                return cudaSuccess;
+            }
+    }
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    CUtensorMap m;
+    std::memset(&m, 0, sizeof(m));
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)B};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    std::lock_guard<std::mutex> lk(mu);
+    Entry& en = cache[next];
+    next = (next + 1) % 16;
+    en.ptr = pool;
+    en.rows = rows;
+    en.d = D;
+    en.b = B;
+    en.dev = dev;
+    en.map = m;
+    *out = m;
+    return cudaSuccess;
+}
+
 namespace {
 
 constexpr int kEndUnit = 1;    // no more work for this CTA
@@ -357,72 +423,6 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
             *abort_flag = 1;
         }
     }
-}
-
-// ---------------------------------------------------------------- tensor maps
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// The pool [num_blocks][kv_heads][B][D] as a 2-D bf16 tensor of rows of D elements;
-// boxes of 64 columns x `B` rows (one stage tile), 128-byte swizzle.  A small cache avoids re-encoding
-// the maps of the same pools on every call.
-cudaError_t tensor_map(CUtensorMap* out, const void* pool, uint64_t rows, int D, int B)
-{
-    struct Entry {
-        const void* ptr;
-        uint64_t rows;
-        int d, b, dev;
-        CUtensorMap map;
-    };
-    static std::mutex mu;
-    static Entry cache[16] = {};
-    static int next = 0;
-    int dev = 0;
-    cudaError_t ce = cudaGetDevice(&dev);
-    if (ce != cudaSuccess) return ce;
-    {
-        std::lock_guard<std::mutex> lk(mu);
-        for (auto& en : cache)
-            if (en.ptr == pool && en.rows == rows && en.d == D && en.b == B && en.dev == dev) {
-                *out = en.map;
-                return cudaSuccess;
-            }
-    }
-    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
-    if (!fn) return cudaErrorNotSupported;
-    CUtensorMap m;
-    std::memset(&m, 0, sizeof(m));
-    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)B};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool), dims, strides, box,
-                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    std::lock_guard<std::mutex> lk(mu);
-    Entry& en = cache[next];
-    next = (next + 1) % 16;
-    en.ptr = pool;
-    en.rows = rows;
-    en.d = D;
-    en.b = B;
-    en.dev = dev;
-    en.map = m;
-    *out = m;
-    return cudaSuccess;
 }
 
 // ---------------------------------------------------------------- launch

@@ -4,6 +4,8 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "pa.h"
@@ -73,6 +75,12 @@ cudaError_t launch_decode(const DecodeArgs& a, pa_dtype dtype, int head_dim, int
                           cudaStream_t stream);
 bool decode_uses_tensor_cores(pa_dtype dtype, int head_dim, int group);
 
+// Tensor maps (TMA descriptors).  The driver's encoder, looked up once, and a cached
+// 2-D bf16 map of a pool [num_blocks][kv_heads][B][D] seen as `rows` rows of D
+// elements, boxes of 64 columns x `box_rows` rows, 128-byte swizzle.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
+cudaError_t tensor_map(CUtensorMap* out, const void* pool, uint64_t rows, int D, int box_rows);
+
 struct ReshapeArgs {
     const void* key;
     const void* value;
@@ -99,6 +107,28 @@ struct CopyArgs {
 };
 
 cudaError_t launch_copy_blocks(const CopyArgs& a, cudaStream_t stream);
+
+// Chunked prefill on the tensor cores (pa_prefill.cu): bf16, head_dim 128.
+struct PrefillArgs {
+    void* out;
+    const void* q;
+    const void* k_cache;
+    const void* v_cache;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    const int32_t* q_start;    // [S + 1] query rows of each sequence
+    unsigned int* status;
+    int num_seqs;
+    int num_heads;
+    int num_kv_heads;
+    int max_blocks_per_seq;
+    int num_blocks;
+    int block_size;
+    float scale_log2;
+};
+
+cudaError_t launch_prefill(const PrefillArgs& a, int group, int num_query_tokens, int max_query_len,
+                           cudaStream_t stream);
 
 // Whole-block copies between two pools, either of which may be pinned host memory
 // (addressed through its device mapping).

@@ -1,0 +1,423 @@
+// Chunked prefill attention over the paged KV cache on the 5th-generation tensor
+// cores (tcgen05, accumulators in tensor memory), for sm_100a.
+//
+// What it computes: the multi-token case of the decode attention.  Sequence s holds
+// L_s tokens in the pools (its new tokens already appended, as for decode), of which
+// the last n_s are queries; query i sits at position p = L_s - n_s + i and attends to
+// tokens 0..p through the block table ("PagedAttention and vLLM Architecture",
+// section 3: the prompt's blocks are assigned when it is processed; "PagedAttention
+// Paper Breakdown", section 2: token t lives at slot T[t / B] * B + t % B).
+//
+// A CTA owns one (sequence, kv head, query tile).  The tile's 128 rows are T query
+// tokens x G query heads of the kv head's group (T = 128 / G), so every K/V byte the
+// CTA loads serves all G heads.  It walks the keys in tiles of 128 tokens:
+//   - warp 4 (one thread) stages Q once and each K/V tile by TMA, one 16-row box per
+//     (physical block, 64 columns), 128-byte swizzle, two stages;
+//   - warp 5 (one thread) issues S = Q K^T (M=128, N=128, K=128: 8 MMAs) into tensor
+//     memory, and O += P V (8 MMAs, B operand MN-major) once P is ready; the next
+//     tile's S is issued as soon as the softmax has read this one, so it overlaps the
+//     softmax;
+//   - warps 0-3 (a thread per row) read S from tensor memory, mask (causal and past
+//     the context), keep the running max in base-2 units, rescale O in tensor memory
+//     only when the max grows by more than 8 (2^8: exact up to rounding, fewer
+//     rescales), write P as bf16 into shared memory, and at the end normalise O and
+//     store it.
+// Every wait is bounded; on expiry the CTA raises PA_DEV_WAIT_TIMEOUT, drains its own
+// copies and MMAs, frees its tensor memory and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "pa_internal.h"
+#include "pa_ptx.cuh"
+#include "pa_tcgen05.cuh"
+
+namespace pa {
+namespace {
+
+constexpr int kM = 128;            // tile rows
+constexpr int kN = 128;            // key tokens per tile
+constexpr int kD = 128;            // head dim
+constexpr int kHalf = 128 * 128;   // bytes of a 64-column half of a 128-row bf16 tile
+constexpr int kTile = 2 * kHalf;   // 32 KB
+constexpr int kBox = 16;           // rows per TMA box of K/V (one 16-token run of a block)
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 256;  // S: columns 0..127, O: 128..255
+constexpr uint32_t kLazyRescale = 8; // base-2 units
+
+constexpr int OFF_Q = 0;
+constexpr int OFF_K = OFF_Q + kTile;
+constexpr int OFF_V = OFF_K + 2 * kTile;
+constexpr int OFF_P = OFF_V + 2 * kTile;
+constexpr int OFF_BAR = OFF_P + kTile;
+// barriers: q_full, kv_full[2], kv_empty[2], s_full, s_free, p_full, o_done, drain
+constexpr int NBAR = 10;
+constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
+constexpr int OFF_ABORT = OFF_TMEM + 8;
+constexpr int kSmem = OFF_ABORT + 8 + 1024;  // + slack to align the base to 1024 bytes
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tmap_q,
+                      const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v)
+{
+    constexpr int T = kM / G;  // query tokens per tile
+    const int tile = (int)gridDim.x - 1 - (int)blockIdx.x;  // the tiles with the most keys start first
+    const int kvh = blockIdx.y;
+    const int s = blockIdx.z;
+    const int q0 = __ldg(a.q_start + s);
+    const int n = __ldg(a.q_start + s + 1) - q0;
+    int L = __ldg(a.context_lens + s);
+    const int Lcap = a.max_blocks_per_seq * a.block_size;
+    if (n < 0 || L < n || L > Lcap) {
+        if (threadIdx.x == 0 && tile == 0 && kvh == 0) atomicOr(a.status, PA_DEV_BAD_CONTEXT);
+        return;
+    }
+    const int t_lo = tile * T;
+    if (t_lo >= n) return;  // whole CTA, before any shared state exists
+    const int t_hi = min(n, t_lo + T);
+    const int p_max = L - n + t_hi - 1;  // last query position of the tile
+    const int ntiles = p_max / kN + 1;
+
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+    uint64_t* q_full = bars + 0;
+    uint64_t* kv_full = bars + 1;   // [2]
+    uint64_t* kv_empty = bars + 3;  // [2]
+    uint64_t* s_full = bars + 5;
+    uint64_t* s_free = bars + 6;
+    uint64_t* p_full = bars + 7;
+    uint64_t* o_done = bars + 8;
+    uint64_t* drain = bars + 9;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&kv_full[i], 1);
+            mbar_init(&kv_empty[i], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(s_free, 4);
+        mbar_init(p_full, 4);
+        mbar_init(o_done, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 5) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem_s = tmem;
+    const uint32_t tmem_o = tmem + 128;
+
+    if (warp == 4) {
+        // ---------------- producer: Q once, then K/V tiles
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_normal();
+            mbar_arrive_expect_tx(q_full, kTile);
+            for (int h = 0; h < 2; ++h)
+                tma_load_3d(smem_u32(smem + OFF_Q + h * kHalf), &tmap_q, h * 64, kvh * G, q0 + t_lo, q_full, pol);
+            const int32_t* table = a.block_tables + (size_t)s * a.max_blocks_per_seq;
+            bool ok = true;
+            for (int j = 0; j < ntiles && ok; ++j) {
+                const int st = j & 1;
+                if (j >= 2 && !mbar_wait_bounded(&kv_empty[st], ((j >> 1) & 1) ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const int tok0 = j * kN;
+                const int nbox = min(kN / kBox, (L - tok0 + kBox - 1) / kBox);
+                mbar_arrive_expect_tx(&kv_full[st], (uint32_t)nbox * kBox * 128 * 4);
+                for (int i = 0; i < nbox; ++i) {
+                    const int tok = tok0 + i * kBox;
+                    int phys = __ldg(table + tok / a.block_size);
+                    if ((unsigned)phys >= (unsigned)a.num_blocks) {
+                        atomicOr(a.status, PA_DEV_BAD_BLOCK);
+                        phys = 0;
+                    }
+                    const int row = (phys * a.num_kv_heads + kvh) * a.block_size + tok % a.block_size;
+                    for (int h = 0; h < 2; ++h) {
+                        const int off = st * kTile + h * kHalf + i * kBox * 128;
+                        tma_load_2d(smem_u32(smem + OFF_K + off), &tmap_k, h * 64, row, &kv_full[st], pol);
+                        tma_load_2d(smem_u32(smem + OFF_V + off), &tmap_v, h * 64, row, &kv_full[st], pol);
+                    }
+                }
+            }
+            if (!ok) {
+                atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+                *abort_flag = 1;
+            }
+            // no copy may still be landing in shared memory at exit
+            volatile int never = 0;
+            if (!mbar_wait_bounded(q_full, 0, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+            for (int j = max(0, ntiles - 2); j < ntiles; ++j)
+                if (!mbar_wait_bounded(&kv_full[j & 1], (j >> 1) & 1, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+        }
+    } else if (warp == 5) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = umma_idesc_bf16(kM, kN, false);
+            constexpr uint32_t idesc_pv = umma_idesc_bf16(kM, kD, true);
+            const uint32_t sq = smem_u32(smem + OFF_Q), sk = smem_u32(smem + OFF_K), sv = smem_u32(smem + OFF_V),
+                           sp = smem_u32(smem + OFF_P);
+            bool ok = mbar_wait_bounded(q_full, 0, abort_flag) && mbar_wait_bounded(&kv_full[0], 0, abort_flag);
+            auto issue_qk = [&](int j) {
+                const uint32_t kb = sk + (j & 1) * kTile;
+#pragma unroll
+                for (int k = 0; k < kD / 16; ++k) {
+                    const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
+                    umma_bf16_ss(tmem_s, umma_desc_sw128(sq + off, 16, 1024), umma_desc_sw128(kb + off, 16, 1024),
+                                 idesc_qk, k > 0 ? 1u : 0u);
+                }
+                umma_commit(s_full);
+            };
+            if (ok) {
+                tc_fence_after_sync();
+                issue_qk(0);
+            }
+            for (int j = 0; j < ntiles && ok; ++j) {
+                if (j + 1 < ntiles) {
+                    if (!mbar_wait_bounded(&kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag) ||
+                        !mbar_wait_bounded(s_free, j & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    issue_qk(j + 1);
+                }
+                if (!mbar_wait_bounded(p_full, j & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t vb = sv + (j & 1) * kTile;
+#pragma unroll
+                for (int k = 0; k < kN / 16; ++k) {
+                    const uint32_t aoff = (k >> 2) * kHalf + (k & 3) * 32;
+                    umma_bf16_ss(tmem_o, umma_desc_sw128(sp + aoff, 16, 1024),
+                                 umma_desc_sw128(vb + k * 16 * 128, kHalf, 1024), idesc_pv,
+                                 (j > 0 || k > 0) ? 1u : 0u);
+                }
+                umma_commit(o_done);
+                umma_commit(&kv_empty[j & 1]);
+            }
+            if (!ok) {
+                atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+                *abort_flag = 1;
+            }
+            // every MMA issued here has completed before tensor memory is freed
+            umma_commit(drain);
+            volatile int never = 0;
+            if (!mbar_wait_bounded(drain, 0, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+        }
+    } else {
+        // ---------------- softmax warps: thread r owns tile row r (TMEM lane r)
+        const int r = threadIdx.x;
+        const int t_local = r / G;
+        const int g = r % G;
+        const int tq = t_lo + t_local;
+        const bool valid_row = t_local < T && tq < n;
+        const int lim = valid_row ? (L - n + tq) : -1;  // last key this row may see
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const float sl = a.scale_log2;
+        float m_used = -INFINITY, l = 0.f;
+        bool ok = true;
+        unsigned char* pbase = smem + OFF_P;
+        for (int j = 0; j < ntiles; ++j) {
+            if (!mbar_wait_bounded(s_full, j & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after_sync();
+            uint32_t sr[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tmem_s + lane_base + c * 32, sr[c]);
+            tmem_wait_ld();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_free);
+            const int kv0 = j * kN;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int kv = kv0 + c * 32 + e;
+                    const float x = kv <= lim ? __uint_as_float(sr[c][e]) * sl : -INFINITY;
+                    sr[c][e] = __float_as_uint(x);
+                    mx = fmaxf(mx, x);
+                }
+            const float m_new = fmaxf(m_used, mx);
+            const bool rescale = m_used != -INFINITY && m_new > m_used + (float)kLazyRescale;
+            // the previous tile's P.V has finished: P may be overwritten and O is stable
+            if (j > 0 && !mbar_wait_bounded(o_done, (j - 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after_sync();
+            if (rescale) {
+                const float alpha = exp2f(m_used - m_new);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem_o + lane_base + c * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(tmem_o + lane_base + c * 32, o);
+                }
+                tmem_wait_st();
+                l *= alpha;
+            }
+            if (rescale || m_used == -INFINITY) m_used = m_new;
+            // P = 2^(s - m), bf16, into the swizzled P tile (row r: 128 bytes per 64-column half)
+            float rowsum = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e2 = 0; e2 < 4; ++e2) {
+                        const float x0 = __uint_as_float(sr[c][q8 * 8 + e2 * 2]);
+                        const float x1 = __uint_as_float(sr[c][q8 * 8 + e2 * 2 + 1]);
+                        const float p0 = m_used == -INFINITY ? 0.f : exp2f(x0 - m_used);
+                        const float p1 = m_used == -INFINITY ? 0.f : exp2f(x1 - m_used);
+                        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                        rowsum += __low2float(pb) + __high2float(pb);
+                        w[e2] = *reinterpret_cast<const uint32_t*>(&pb);
+                    }
+                    const int chunk = c * 4 + q8;  // 16-byte chunk of the row, 0..15
+                    const int h = chunk >> 3;
+                    const int cc = chunk & 7;
+                    *reinterpret_cast<uint4*>(pbase + h * kHalf + r * 128 + ((cc ^ (r & 7)) << 4)) =
+                        make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            l += rowsum;
+            // keys past the context in this tile: zero their V rows (0-weights must meet finite values)
+            if (kv0 + kN > L) {
+                unsigned char* vb = smem + OFF_V + (j & 1) * kTile;
+                const int first = max(0, L - kv0);
+                const int chunks = (kN - first) * 16;  // 16-byte chunks over both halves
+                for (int i = r; i < chunks; i += 128) {
+                    const int row = first + (i >> 4);
+                    const int h = (i >> 3) & 1;
+                    *reinterpret_cast<uint4*>(vb + h * kHalf + row * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            fence_async_smem();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+        }
+        if (ok && mbar_wait_bounded(o_done, (ntiles - 1) & 1, abort_flag)) {
+            tc_fence_after_sync();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) +
+                                 ((size_t)(q0 + tq) * a.num_heads + (size_t)kvh * G + g) * kD;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tmem_o + lane_base + c * 32, o);
+                tmem_wait_ld();
+                if (valid_row) {
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        uint4 pk;
+                        pk.x = pack_bf16(__uint_as_float(o[v4 * 8 + 0]) * inv, __uint_as_float(o[v4 * 8 + 1]) * inv);
+                        pk.y = pack_bf16(__uint_as_float(o[v4 * 8 + 2]) * inv, __uint_as_float(o[v4 * 8 + 3]) * inv);
+                        pk.z = pack_bf16(__uint_as_float(o[v4 * 8 + 4]) * inv, __uint_as_float(o[v4 * 8 + 5]) * inv);
+                        pk.w = pack_bf16(__uint_as_float(o[v4 * 8 + 6]) * inv, __uint_as_float(o[v4 * 8 + 7]) * inv);
+                        *reinterpret_cast<uint4*>(out + c * 32 + v4 * 8) = pk;
+                    }
+                }
+            }
+        } else {
+            ok = false;
+        }
+        if (!ok) {
+            if (lane == 0) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+            *abort_flag = 1;
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == 5) tmem_dealloc(tmem, kTmemCols);
+}
+
+// q [Nq][Hq][D] as a 3-D bf16 tensor (D, Hq, Nq); boxes of 64 columns x G heads x
+// 128/G tokens, 128-byte swizzle: one box fills a 64-column half of the Q tile with
+// rows ordered (token, head).
+cudaError_t q_tensor_map(CUtensorMap* out, const void* q, int num_tokens, int num_heads, int G)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    std::memset(out, 0, sizeof(*out));
+    const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)num_heads, (cuuint64_t)num_tokens};
+    const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)num_heads * kD * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)(kM / G)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int G>
+cudaError_t launch_g(const PrefillArgs& a, int num_query_tokens, int max_query_len, cudaStream_t stream)
+{
+    CUtensorMap tq, tk, tv;
+    cudaError_t e = q_tensor_map(&tq, a.q, num_query_tokens, a.num_heads, G);
+    if (e != cudaSuccess) return e;
+    const uint64_t rows = (uint64_t)a.num_blocks * a.num_kv_heads * a.block_size;
+    if ((e = tensor_map(&tk, a.k_cache, rows, kD, kBox)) != cudaSuccess) return e;
+    if ((e = tensor_map(&tv, a.v_cache, rows, kD, kBox)) != cudaSuccess) return e;
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_done[dev & 63]) {
+        e = cudaFuncSetAttribute(prefill_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+        if (e != cudaSuccess) return e;
+        attr_done[dev & 63] = true;
+    }
+    constexpr int T = kM / G;
+    const dim3 grid((unsigned)((max_query_len + T - 1) / T), (unsigned)a.num_kv_heads, (unsigned)a.num_seqs);
+    prefill_tc_kernel<G><<<grid, kThreads, kSmem, stream>>>(a, tq, tk, tv);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const PrefillArgs& a, int group, int num_query_tokens, int max_query_len,
+                           cudaStream_t stream)
+{
+    if (a.num_seqs == 0 || max_query_len == 0 || num_query_tokens == 0) return cudaSuccess;
+    switch (group) {
+        case 1: return launch_g<1>(a, num_query_tokens, max_query_len, stream);
+        case 2: return launch_g<2>(a, num_query_tokens, max_query_len, stream);
+        case 4: return launch_g<4>(a, num_query_tokens, max_query_len, stream);
+        case 8: return launch_g<8>(a, num_query_tokens, max_query_len, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace pa

@@ -39,6 +39,7 @@ SIGNATURES = [
     ("pa_decode", _int, [_vp, _vp, _vp, _vp, _vp, _vp] + [_int] * 8 + [_f32, _int, _vp, _sz, _int, _vp]),
     ("pa_decode_static_workspace", _int, [_vp, _vp, _vp, _vp, _vp, _vp] + [_int] * 8 + [_f32, _int, _int, _vp]),
     ("pa_reshape_and_cache", _int, [_vp, _vp, _vp, _vp, _vp] + [_int] * 6 + [_vp]),
+    ("pa_prefill", _int, [_vp] * 7 + [_int] * 9 + [_f32, _int, _vp]),
     ("pa_copy_blocks", _int, [_vp, _vp, _vp] + [_int] * 6 + [_vp]),
     ("pa_swap_blocks", _int, [_vp, _vp, _vp, _vp, _vp] + [_int] * 7 + [_vp]),
     ("pa_device_status", _int, [ctypes.POINTER(_u32), _vp]),
@@ -206,6 +207,29 @@ def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None
                                   _dev_ptr(v_cache, "v_cache"), _dev_ptr(slot_mapping, "slot_mapping"), N, Hkv, D,
                                   B, NB, dt, _stream(stream))
     _check(st, "pa_reshape_and_cache")
+
+
+def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, q_start, max_query_len, scale, stream=None):
+    """out[Nq,Hq,D] <- causal attention of the packed query rows q[Nq,Hq,D] (rows q_start[s]..q_start[s+1]-1
+    are the last tokens of sequence s) over k/v_cache[NB,Hkv,B,D] through block_tables."""
+    import torch
+    Nq, Hq, D = q.shape
+    NB, Hkv, B, D2 = k_cache.shape
+    S = context_lens.shape[0]
+    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or tuple(q_start.shape) != (S + 1,):
+        raise ValueError("block_tables must be [S, max_blocks] and q_start [S + 1]")
+    if any(t.dtype != torch.int32 for t in (block_tables, context_lens, q_start)):
+        raise TypeError("block_tables, context_lens and q_start must be int32")
+    dt = _dtype_code(q)
+    if any(_dtype_code(t) != dt for t in (out, k_cache, v_cache)):
+        raise TypeError("q, out and the caches must share a dtype")
+    st = lib.pa_prefill(_dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
+                        _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables"),
+                        _dev_ptr(context_lens, "context_lens"), _dev_ptr(q_start, "q_start"), S, Hq, Hkv, D, B,
+                        block_tables.shape[1], NB, Nq, int(max_query_len), float(scale), dt, _stream(stream))
+    _check(st, "pa_prefill")
 
 
 def pa_swap_blocks(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache, block_mapping, stream=None):

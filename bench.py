@@ -416,6 +416,73 @@ def e2e_leg(stepper, args, world, dev):
     return {"ms": ms, "h2d": stepper.h2d_bytes, "d2h": stepper.d2h_bytes, "host_us": 1e6 * host_s / args.steps}
 
 
+def run_prefill(args, wl, batch, dev, stream, world):
+    """Chunked prefill: TFLOP/s of pa_prefill (causal FLOPs only) against the tensor peak."""
+    import torch
+    from paged_kv_cache_363_b200 import pa
+
+    flops = wl.flops()
+    for _ in range(args.warmup):
+        batch.step(stream)
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        t0.record(stream)
+        for a, b in evs:
+            a.record(stream)
+            batch.step(stream)
+            b.record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = reduce_max(t0.elapsed_time(t1), dev)
+    per = [a.elapsed_time(b) for a, b in evs]
+    avg = reduce_max(statistics.mean(per), dev)
+    # end to end: each step uploads its query rows from pinned memory and reads the output back
+    qh = batch.q.cpu().pin_memory()
+    oh = torch.empty(batch.out.shape, dtype=batch.out.dtype).pin_memory()
+    e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for k in range(args.warmup + args.steps):
+        if k == args.warmup:
+            e_s.record(stream)
+        batch.q.copy_(qh, non_blocking=True)
+        batch.step(stream)
+        oh.copy_(batch.out, non_blocking=True)
+    e_e.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = reduce_max(e_s.elapsed_time(e_e), dev)
+    peak = None
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, kind = float(json.load(f)["bf16_tflops"]), "measured (cuBLAS bf16 burst)"
+    except Exception:
+        peak, kind = 1590.0, "fallback"
+    achieved = flops / (avg * 1e-3) / 1e12
+    out_ok = bool(torch.isfinite(batch.out.float()).all().item())
+    line = {
+        "metric": "chunked prefill attention TFLOP/s over the paged KV cache (causal FLOPs)",
+        "value": round(world * flops * args.steps / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload=wl.name, num_seqs=wl.num_seqs, num_heads=wl.num_heads, num_kv_heads=wl.num_kv_heads,
+                       head_dim=wl.head_dim, block_size=wl.block_size, query_tokens=int(wl.query_lens.sum()),
+                       context_tokens=int(wl.context_lens.sum()), seed=wl.seed,
+                       l2="compute-bound; %.0f MB of KV read per step" % (
+                           wl.context_lens.sum() * 2 * wl.num_kv_heads * wl.head_dim * 2 / 1e6),
+                       parallelism="replicas: one batch per GPU (dp%d)" % world),
+        "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel", "achieved": round(achieved, 2),
+                     "peak": peak, "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": None, "algorithmic_flops_per_launch": flops, "avg_launch_us": round(avg * 1e3, 3)},
+        "e2e": {"value": round(world * flops * args.steps / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": qh.numel() * qh.element_size(),
+                "d2h_bytes_per_step": oh.numel() * oh.element_size(), "ms_per_step": round(e2e_ms / args.steps, 5)},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+        "device_status": pa.pa_device_status(), "output_finite": out_ok,
+    }
+    return line
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -444,10 +511,20 @@ def run_gpu(args):
         values = W.prefix_values(wl, dev)
     elif isinstance(wl, W.BeamWorkload):
         values = W.beam_values(wl, dev)
+    elif isinstance(wl, W.PrefillWorkload):
+        values = W.prefill_values(wl, dev)
     else:
         values = W.decode_values(wl, dev)
     batch = runner.make_batch(wl, dev, values=values)
     from paged_kv_cache_363_b200 import pa
+    if isinstance(wl, W.PrefillWorkload):
+        stream = torch.cuda.current_stream(dev)
+        line = run_prefill(args, wl, batch, dev, stream, world)
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line))
+        return 0
     part = pa.pa_decode_partition_size(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size,
                                        batch.max_context_len, batch.partition_size)
     n_part = -(-batch.max_context_len // part)

@@ -11,8 +11,9 @@
 // A CTA owns one (sequence, kv head, query tile).  The tile's 128 rows are T query
 // tokens x G query heads of the kv head's group (T = 128 / G), so every K/V byte the
 // CTA loads serves all G heads.  It walks the keys in tiles of 128 tokens:
-//   - warp 4 (one thread) stages Q once and each K/V tile by TMA, one 16-row box per
-//     (physical block, 64 columns), 128-byte swizzle, two stages;
+//   - warp 4 stages Q once and each K/V tile by TMA, one 16-row box per (16-token run
+//     of a physical block, 64 columns), 128-byte swizzle, two stages; lane i looks up
+//     and issues box i of the tile;
 //   - warp 5 (one thread) issues S = Q K^T (M=128, N=128, K=128: 8 MMAs) into tensor
 //     memory, and O += P V (8 MMAs, B operand MN-major) once P is ready; the next
 //     tile's S is issued as soon as the softmax has read this one, so it overlaps the
@@ -59,6 +60,14 @@ constexpr int NBAR = 10;
 constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
 constexpr int OFF_ABORT = OFF_TMEM + 8;
 constexpr int kSmem = OFF_ABORT + 8 + 1024;  // + slack to align the base to 1024 bytes
+
+// 2^x by the hardware approximation (ex2.approx, relative error about 2^-22; 2^-inf = 0).
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 {
@@ -128,38 +137,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_o = tmem + 128;
 
     if (warp == 4) {
-        // ---------------- producer: Q once, then K/V tiles
+        // ---------------- producer: Q once, then K/V tiles.  Lane i looks up the
+        // physical block of the tile's i-th 16-token box and issues its copies, so
+        // the table reads of a tile overlap instead of queueing behind each other.
+        const uint64_t pol = policy_evict_normal();
         if (lane == 0) {
-            const uint64_t pol = policy_evict_normal();
             mbar_arrive_expect_tx(q_full, kTile);
             for (int h = 0; h < 2; ++h)
                 tma_load_3d(smem_u32(smem + OFF_Q + h * kHalf), &tmap_q, h * 64, kvh * G, q0 + t_lo, q_full, pol);
-            const int32_t* table = a.block_tables + (size_t)s * a.max_blocks_per_seq;
-            bool ok = true;
-            for (int j = 0; j < ntiles && ok; ++j) {
-                const int st = j & 1;
-                if (j >= 2 && !mbar_wait_bounded(&kv_empty[st], ((j >> 1) & 1) ^ 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                const int tok0 = j * kN;
-                const int nbox = min(kN / kBox, (L - tok0 + kBox - 1) / kBox);
-                mbar_arrive_expect_tx(&kv_full[st], (uint32_t)nbox * kBox * 128 * 4);
-                for (int i = 0; i < nbox; ++i) {
-                    const int tok = tok0 + i * kBox;
-                    int phys = __ldg(table + tok / a.block_size);
-                    if ((unsigned)phys >= (unsigned)a.num_blocks) {
-                        atomicOr(a.status, PA_DEV_BAD_BLOCK);
-                        phys = 0;
-                    }
-                    const int row = (phys * a.num_kv_heads + kvh) * a.block_size + tok % a.block_size;
-                    for (int h = 0; h < 2; ++h) {
-                        const int off = st * kTile + h * kHalf + i * kBox * 128;
-                        tma_load_2d(smem_u32(smem + OFF_K + off), &tmap_k, h * 64, row, &kv_full[st], pol);
-                        tma_load_2d(smem_u32(smem + OFF_V + off), &tmap_v, h * 64, row, &kv_full[st], pol);
-                    }
+        }
+        const int32_t* table = a.block_tables + (size_t)s * a.max_blocks_per_seq;
+        bool ok = true;
+        for (int j = 0; j < ntiles && ok; ++j) {
+            const int st = j & 1;
+            const int tok0 = j * kN;
+            const int nbox = min(kN / kBox, (L - tok0 + kBox - 1) / kBox);
+            const int tok = tok0 + lane * kBox;
+            int phys = 0;
+            if (lane < nbox) {
+                phys = __ldg(table + tok / a.block_size);
+                if ((unsigned)phys >= (unsigned)a.num_blocks) {
+                    atomicOr(a.status, PA_DEV_BAD_BLOCK);
+                    phys = 0;
                 }
             }
+            if (lane == 0) {
+                if (j >= 2 && !mbar_wait_bounded(&kv_empty[st], ((j >> 1) & 1) ^ 1, abort_flag)) ok = false;
+                if (ok) mbar_arrive_expect_tx(&kv_full[st], (uint32_t)nbox * kBox * 128 * 4);
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            if (lane < nbox) {
+                const int row = (phys * a.num_kv_heads + kvh) * a.block_size + tok % a.block_size;
+                for (int h = 0; h < 2; ++h) {
+                    const int off = st * kTile + h * kHalf + lane * kBox * 128;
+                    tma_load_2d(smem_u32(smem + OFF_K + off), &tmap_k, h * 64, row, &kv_full[st], pol);
+                    tma_load_2d(smem_u32(smem + OFF_V + off), &tmap_v, h * 64, row, &kv_full[st], pol);
+                }
+            }
+        }
+        if (lane == 0) {
             if (!ok) {
                 atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
                 *abort_flag = 1;
@@ -273,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after_sync();
             if (rescale) {
-                const float alpha = exp2f(m_used - m_new);
+                const float alpha = fast_exp2(m_used - m_new);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t o[32];
@@ -287,6 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 l *= alpha;
             }
             if (rescale || m_used == -INFINITY) m_used = m_new;
+            const float mref = m_used == -INFINITY ? 0.f : m_used;  // a row with no key yet: every x is -inf
             // P = 2^(s - m), bf16, into the swizzled P tile (row r: 128 bytes per 64-column half)
             float rowsum = 0.f;
 #pragma unroll
@@ -298,8 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int e2 = 0; e2 < 4; ++e2) {
                         const float x0 = __uint_as_float(sr[c][q8 * 8 + e2 * 2]);
                         const float x1 = __uint_as_float(sr[c][q8 * 8 + e2 * 2 + 1]);
-                        const float p0 = m_used == -INFINITY ? 0.f : exp2f(x0 - m_used);
-                        const float p1 = m_used == -INFINITY ? 0.f : exp2f(x1 - m_used);
+                        const float p0 = fast_exp2(x0 - mref);
+                        const float p1 = fast_exp2(x1 - mref);
                         const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
                         rowsum += __low2float(pb) + __high2float(pb);
                         w[e2] = *reinterpret_cast<const uint32_t*>(&pb);

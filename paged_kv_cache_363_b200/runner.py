@@ -378,6 +378,42 @@ class BeamBatch:
         return wl.num_seqs * (2 * row * 2 + 8) + int(self.cow_pairs.shape[0]) * 2 * (row * wl.block_size) * 2
 
 
+class PrefillBatch:
+    """Chunked prefill: every sequence's prefix and chunk placed by the allocator and
+    written with pa_reshape_and_cache; the step is one pa_prefill over all chunks."""
+
+    def __init__(self, wl, device="cuda", values=None, fill=float("nan"), partition_size=None):
+        self.wl = wl
+        self.device = torch.device(device)
+        S, Hq, Hkv, D, B, NB = (wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size,
+                                wl.num_blocks)
+        dt = W.torch_dtype(wl.dtype)
+        if values is None:
+            values = W.prefill_values(wl, self.device)
+        q, keys, vals = values
+        self.k_cache = torch.full((NB, Hkv, B, D), fill, dtype=dt, device=self.device)
+        self.v_cache = torch.full((NB, Hkv, B, D), fill, dtype=dt, device=self.device)
+        self.alloc = pa.Allocator(NB, B, wl.free_order)
+        L = wl.context_lens
+        slots = np.concatenate([self.alloc.add_seq(s, int(L[s])) for s in range(S)])
+        pa.pa_reshape_and_cache(keys.to(self.device).contiguous(), vals.to(self.device).contiguous(), self.k_cache,
+                                self.v_cache, torch.from_numpy(slots).to(self.device))
+        tables, ctx = DecodeBatch.tables_now(self)
+        self.block_tables = torch.from_numpy(tables).to(self.device)
+        self.context_lens = torch.from_numpy(ctx).to(self.device)
+        qs = np.concatenate([[0], np.cumsum(wl.query_lens)]).astype(np.int32)
+        self.q_start_np = qs
+        self.q_start = torch.from_numpy(qs).to(self.device)
+        self.max_query_len = int(wl.query_lens.max()) if S else 0
+        self.q = q.to(self.device).contiguous()
+        self.out = torch.empty_like(self.q)
+
+    def step(self, stream=None):
+        pa.pa_prefill(self.out, self.q, self.k_cache, self.v_cache, self.block_tables, self.context_lens,
+                      self.q_start, self.max_query_len, self.wl.scale, stream=stream)
+        return self.out
+
+
 def make_batch(wl, device="cuda", values=None, fill=float("nan"), partition_size=None):
     if isinstance(wl, W.CowWorkload):
         cls = CowBatch
@@ -385,6 +421,8 @@ def make_batch(wl, device="cuda", values=None, fill=float("nan"), partition_size
         cls = PrefixBatch
     elif isinstance(wl, W.BeamWorkload):
         cls = BeamBatch
+    elif isinstance(wl, W.PrefillWorkload):
+        cls = PrefillBatch
     else:
         cls = DecodeBatch
     return cls(wl, device=device, values=values, fill=fill, partition_size=partition_size)

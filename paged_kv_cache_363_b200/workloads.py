@@ -42,6 +42,8 @@ WORKLOADS = {
     6: dict(name="prefix-cache-bf16", num_prompts=8, requests_per_prompt=16, num_heads=32, num_kv_heads=8,
             head_dim=128, block_size=16, dtype="bf16", stem_lens=(512, 1536), suffix_lens=(16, 256),
             vocab=32000, num_blocks=20000, partition_size=0),
+    8: dict(name="prefill-chunk-bf16", num_seqs=16, num_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+            dtype="bf16", prefix_lens=(0, 2048), chunk=1024, num_blocks=20000, partition_size=0),
     7: dict(name="beam-search-bf16", num_requests=16, beam_width=4, num_heads=32, num_kv_heads=8, head_dim=128,
             block_size=16, dtype="bf16", prompt_lens=(256, 1024), beam_steps=24, num_blocks=20000,
             partition_size=0),
@@ -177,6 +179,39 @@ class BeamWorkload:
         return np.repeat(self.prompt_lens, self.beam_width) + self.beam_steps
 
 
+@dataclass
+class PrefillWorkload:
+    """Chunked prefill: sequence s already holds prefix_lens[s] tokens and appends a
+    chunk of `chunk` tokens, which are its queries (causal over prefix + chunk)."""
+    wid: int
+    name: str
+    seed: int
+    num_seqs: int
+    num_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    dtype: str
+    num_blocks: int
+    partition_size: int
+    prefix_lens: np.ndarray             # int32 [S]
+    query_lens: np.ndarray              # int32 [S]
+    free_order: np.ndarray
+    scale: float = field(default=0.0)
+
+    @property
+    def context_lens(self):
+        return (self.prefix_lens + self.query_lens).astype(np.int32)
+
+    def flops(self):
+        """Causal attention FLOPs: 4 * D per (query, visible key, query head)."""
+        tot = 0
+        for P, n in zip(self.prefix_lens, self.query_lens):
+            keys = int(n) * int(P) + int(n) * (int(n) + 1) // 2
+            tot += 4 * self.head_dim * self.num_heads * keys
+        return tot
+
+
 def _rng(seed, salt):
     return np.random.default_rng([int(seed), int(salt)])
 
@@ -210,6 +245,18 @@ def make_workload(wid, seed=0, **overrides):
                          head_dim=spec["head_dim"], block_size=spec["block_size"], dtype=spec["dtype"],
                          num_blocks=spec["num_blocks"], partition_size=spec["partition_size"],
                          prompt_lens=prompt_lens, private_tokens=private, free_order=free_order)
+    elif wid == 8:
+        S = spec["num_seqs"]
+        plo, phi = spec["prefix_lens"]
+        prefix = rng.integers(plo, phi + 1, size=S).astype(np.int32)
+        qlen = np.full(S, spec["chunk"], np.int32) if "query_lens" not in spec else np.asarray(spec["query_lens"],
+                                                                                             np.int32)
+        free_order = rng.permutation(spec["num_blocks"]).astype(np.int32)
+        wl = PrefillWorkload(wid=wid, name=spec["name"], seed=seed, num_seqs=S, num_heads=spec["num_heads"],
+                             num_kv_heads=spec["num_kv_heads"], head_dim=spec["head_dim"],
+                             block_size=spec["block_size"], dtype=spec["dtype"], num_blocks=spec["num_blocks"],
+                             partition_size=spec["partition_size"], prefix_lens=prefix, query_lens=qlen,
+                             free_order=free_order)
     elif wid == 7:
         R, Wd, T = spec["num_requests"], spec["beam_width"], spec["beam_steps"]
         plo, phi = spec["prompt_lens"]
@@ -315,6 +362,17 @@ def prefix_values(wl, device="cpu"):
     xoff = np.zeros(wl.num_seqs + 1, np.int64)
     xoff[1:] = np.cumsum(wl.suffix_lens)
     return q, sk, sv, soff, xk, xv, xoff
+
+
+def prefill_values(wl, device="cpu"):
+    """q rows of every chunk [sum query_lens, Hq, D] (packed by sequence) and the K/V
+    rows of every context token [sum context_lens, Hkv, D] (packed by sequence)."""
+    Hq, Hkv, D = wl.num_heads, wl.num_kv_heads, wl.head_dim
+    total = int(wl.context_lens.sum())
+    q = normal((int(wl.query_lens.sum()), Hq, D), wl.dtype, device, wl.seed, 1)
+    keys = normal((total, Hkv, D), wl.dtype, device, wl.seed, 2)
+    vals = normal((total, Hkv, D), wl.dtype, device, wl.seed, 3)
+    return q, keys, vals
 
 
 def beam_values(wl, device="cpu"):

@@ -128,3 +128,29 @@ def test_unsupported_shapes_are_refused(pa):
         pa.pa_prefill(torch.empty_like(q), q, k, k, t, torch.tensor([4], dtype=torch.int32, device="cuda"),
                       torch.tensor([0, 4], dtype=torch.int32, device="cuda"), 4, 1.0)
     assert e.value.status == pa.PA_ERR_UNSUPPORTED
+
+
+def test_prefill_workload_full_size_sampled(pa):
+    from paged_kv_cache_363_b200 import runner
+    from paged_kv_cache_363_b200 import workloads as W
+    from pa_testlib import oracle_logical
+    wl = W.make_workload(8, seed=0)
+    vals = W.prefill_values(wl, "cpu")
+    batch = runner.PrefillBatch(wl, "cuda", values=vals)
+    out = batch.step()
+    torch.cuda.synchronize()
+    assert pa.pa_device_status() == 0
+    got = out.float().cpu().numpy()
+    assert np.isfinite(got).all()
+    q, keys, values = vals
+    koff = np.concatenate([[0], np.cumsum(wl.context_lens)])
+    qs = batch.q_start_np
+    rows, ks, vs = [], [], []
+    for s in (0, 5, wl.num_seqs - 1):
+        for i in (0, 1, 511, int(wl.query_lens[s]) - 1):
+            pos = int(wl.prefix_lens[s]) + i
+            rows.append(int(qs[s]) + i)
+            ks.append(keys[koff[s]:koff[s] + pos + 1].float().numpy())
+            vs.append(values[koff[s]:koff[s] + pos + 1].float().numpy())
+    ref = oracle_logical(q[rows].float().numpy(), ks, vs, wl.block_size, wl.scale)
+    assert max_abs(got[rows], ref) <= TOL["bf16"]

@@ -10,19 +10,22 @@
 //
 // A CTA owns one (sequence, kv head, query tile).  The tile's 128 rows are T query
 // tokens x G query heads of the kv head's group (T = 128 / G), so every K/V byte the
-// CTA loads serves all G heads.  It walks the keys in tiles of 128 tokens:
+// CTA loads serves all G heads.  It walks the keys in tiles of 64 tokens:
 //   - warp 4 stages Q once and each K/V tile by TMA, one 16-row box per (16-token run
 //     of a physical block, 64 columns), 128-byte swizzle, two stages; lane i looks up
 //     and issues box i of the tile;
-//   - warp 5 (one thread) issues S = Q K^T (M=128, N=128, K=128: 8 MMAs) into tensor
-//     memory, and O += P V (8 MMAs, B operand MN-major) once P is ready; the next
+//   - warp 5 (one thread) issues S = Q K^T (M=128, N=64, K=128: 8 MMAs) into tensor
+//     memory, and O += P V (N=128, K=64: 4 MMAs, A = P from tensor memory, B operand
+//     MN-major) once P is ready; the next
 //     tile's S is issued as soon as the softmax has read this one, so it overlaps the
 //     softmax;
 //   - warps 0-3 (a thread per row) read S from tensor memory, mask (causal and past
 //     the context), keep the running max in base-2 units, rescale O in tensor memory
 //     only when the max grows by more than 8 (2^8: exact up to rounding, fewer
-//     rescales), write P as bf16 into shared memory, and at the end normalise O and
-//     store it.
+//     rescales), write P as bf16 into tensor memory (two buffers, so the next tile's
+//     P is written while this tile's P.V runs), and at the end normalise O and store it.
+// Two CTAs share an SM (97 KB of shared memory and 256 tensor-memory columns each),
+// so one CTA's softmax overlaps the other's matrix multiplies.
 // Every wait is bounded; on expiry the CTA raises PA_DEV_WAIT_TIMEOUT, drains its own
 // copies and MMAs, frees its tensor memory and returns.
 #include <cuda.h>
@@ -41,25 +44,29 @@ namespace pa {
 namespace {
 
 constexpr int kM = 128;            // tile rows
-constexpr int kN = 128;            // key tokens per tile
+constexpr int kN = 64;             // key tokens per tile
 constexpr int kD = 128;            // head dim
-constexpr int kHalf = 128 * 128;   // bytes of a 64-column half of a 128-row bf16 tile
-constexpr int kTile = 2 * kHalf;   // 32 KB
+constexpr int kQHalf = kM * 128;   // bytes of a 64-column half of the Q tile (16 KB)
+constexpr int kKVHalf = kN * 128;  // bytes of a 64-column half of a K or V tile (8 KB)
 constexpr int kBox = 16;           // rows per TMA box of K/V (one 16-token run of a block)
 constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 256;  // S: columns 0..127, O: 128..255
+constexpr uint32_t kTmemCols = 256;  // S: 0..63, P: 64..95 and 96..127, O: 128..255 (two CTAs fill the 512)
 constexpr uint32_t kLazyRescale = 8; // base-2 units
 
+// Tiles, from a 1024-byte aligned base: Q (32 KB), K and V in two stages (16 KB
+// each): 96 KB.  P lives in tensor memory (two buffers, the A operand of P.V).  The
+// barriers go in the alignment slack when it has room, else after the tiles; two
+// CTAs share an SM.
 constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + kTile;
-constexpr int OFF_V = OFF_K + 2 * kTile;
-constexpr int OFF_P = OFF_V + 2 * kTile;
-constexpr int OFF_BAR = OFF_P + kTile;
-// barriers: q_full, kv_full[2], kv_empty[2], s_full, s_free, p_full, o_done, drain
-constexpr int NBAR = 10;
-constexpr int OFF_TMEM = OFF_BAR + NBAR * 8;
-constexpr int OFF_ABORT = OFF_TMEM + 8;
-constexpr int kSmem = OFF_ABORT + 8 + 1024;  // + slack to align the base to 1024 bytes
+constexpr int OFF_K = OFF_Q + 2 * kQHalf;
+constexpr int OFF_V = OFF_K + 2 * 2 * kKVHalf;
+constexpr int kTiles = OFF_V + 2 * 2 * kKVHalf;
+// barriers: q_full, kv_full[2], kv_empty[2], s_full, s_free, p_full, o_done[2], drain
+constexpr int NBAR = 11;
+constexpr int kMisc = 128;          // barriers, TMEM base, abort flag
+constexpr int kSmem = kTiles + 1024 + kMisc;
+static_assert(kTiles + 1023 <= kSmem, "tiles fit with any base alignment");
+static_assert(NBAR * 8 + 16 <= kMisc, "misc area");
 
 // 2^x by the hardware approximation (ex2.approx, relative error about 2^-22; 2^-inf = 0).
 __device__ __forceinline__ float fast_exp2(float x)
@@ -69,6 +76,15 @@ __device__ __forceinline__ float fast_exp2(float x)
     return y;
 }
 
+// A bounded mbarrier wait taken by every lane of a warp, with one answer for the
+// whole warp: the tcgen05.ld / tcgen05.st that follow are .sync.aligned and must be
+// reached by all lanes together or by none.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
+{
+    const bool ok = mbar_wait_bounded(bar, parity, abort_flag);
+    return __all_sync(0xffffffffu, ok) != 0;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -76,7 +92,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 }
 
 template <int G>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v)
 {
@@ -99,18 +115,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ntiles = p_max / kN + 1;
 
     extern __shared__ unsigned char smem_raw[];
-    unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+    const uint32_t slack = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    unsigned char* smem = smem_raw + slack;
+    unsigned char* misc = slack >= (uint32_t)kMisc ? smem_raw : smem + kTiles;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(misc);
     uint64_t* q_full = bars + 0;
     uint64_t* kv_full = bars + 1;   // [2]
     uint64_t* kv_empty = bars + 3;  // [2]
     uint64_t* s_full = bars + 5;
     uint64_t* s_free = bars + 6;
     uint64_t* p_full = bars + 7;
-    uint64_t* o_done = bars + 8;
-    uint64_t* drain = bars + 9;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_TMEM);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
+    uint64_t* o_done = bars + 8;    // [2]: P.V of the tiles using P buffer 0 / 1
+    uint64_t* drain = bars + 10;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + NBAR * 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + NBAR * 8 + 8);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
@@ -123,7 +141,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(s_full, 1);
         mbar_init(s_free, 4);
         mbar_init(p_full, 4);
-        mbar_init(o_done, 1);
+        mbar_init(&o_done[0], 1);
+        mbar_init(&o_done[1], 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -134,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tmem_s = tmem;
+    const uint32_t tmem_p = tmem + 64;  // + 32 * buffer
     const uint32_t tmem_o = tmem + 128;
 
     if (warp == 4) {
@@ -142,9 +162,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the table reads of a tile overlap instead of queueing behind each other.
         const uint64_t pol = policy_evict_normal();
         if (lane == 0) {
-            mbar_arrive_expect_tx(q_full, kTile);
+            mbar_arrive_expect_tx(q_full, 2 * kQHalf);
             for (int h = 0; h < 2; ++h)
-                tma_load_3d(smem_u32(smem + OFF_Q + h * kHalf), &tmap_q, h * 64, kvh * G, q0 + t_lo, q_full, pol);
+                tma_load_3d(smem_u32(smem + OFF_Q + h * kQHalf), &tmap_q, h * 64, kvh * G, q0 + t_lo, q_full, pol);
         }
         const int32_t* table = a.block_tables + (size_t)s * a.max_blocks_per_seq;
         bool ok = true;
@@ -170,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane < nbox) {
                 const int row = (phys * a.num_kv_heads + kvh) * a.block_size + tok % a.block_size;
                 for (int h = 0; h < 2; ++h) {
-                    const int off = st * kTile + h * kHalf + lane * kBox * 128;
+                    const int off = st * 2 * kKVHalf + h * kKVHalf + lane * kBox * 128;
                     tma_load_2d(smem_u32(smem + OFF_K + off), &tmap_k, h * 64, row, &kv_full[st], pol);
                     tma_load_2d(smem_u32(smem + OFF_V + off), &tmap_v, h * 64, row, &kv_full[st], pol);
                 }
@@ -192,16 +212,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = umma_idesc_bf16(kM, kN, false);
             constexpr uint32_t idesc_pv = umma_idesc_bf16(kM, kD, true);
-            const uint32_t sq = smem_u32(smem + OFF_Q), sk = smem_u32(smem + OFF_K), sv = smem_u32(smem + OFF_V),
-                           sp = smem_u32(smem + OFF_P);
+            const uint32_t sq = smem_u32(smem + OFF_Q), sk = smem_u32(smem + OFF_K), sv = smem_u32(smem + OFF_V);
             bool ok = mbar_wait_bounded(q_full, 0, abort_flag) && mbar_wait_bounded(&kv_full[0], 0, abort_flag);
             auto issue_qk = [&](int j) {
-                const uint32_t kb = sk + (j & 1) * kTile;
+                const uint32_t kb = sk + (j & 1) * 2 * kKVHalf;
 #pragma unroll
                 for (int k = 0; k < kD / 16; ++k) {
-                    const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
-                    umma_bf16_ss(tmem_s, umma_desc_sw128(sq + off, 16, 1024), umma_desc_sw128(kb + off, 16, 1024),
-                                 idesc_qk, k > 0 ? 1u : 0u);
+                    const uint32_t kk = (k & 3) * 32;
+                    umma_bf16_ss(tmem_s, umma_desc_sw128(sq + (k >> 2) * kQHalf + kk, 16, 1024),
+                                 umma_desc_sw128(kb + (k >> 2) * kKVHalf + kk, 16, 1024), idesc_qk, k > 0 ? 1u : 0u);
                 }
                 umma_commit(s_full);
             };
@@ -224,15 +243,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc_fence_after_sync();
-                const uint32_t vb = sv + (j & 1) * kTile;
+                const uint32_t vb = sv + (j & 1) * 2 * kKVHalf;
 #pragma unroll
                 for (int k = 0; k < kN / 16; ++k) {
-                    const uint32_t aoff = (k >> 2) * kHalf + (k & 3) * 32;
-                    umma_bf16_ss(tmem_o, umma_desc_sw128(sp + aoff, 16, 1024),
-                                 umma_desc_sw128(vb + k * 16 * 128, kHalf, 1024), idesc_pv,
+                    umma_bf16_ts(tmem_o, tmem_p + (j & 1) * 32 + k * 8,
+                                 umma_desc_sw128(vb + k * 16 * 128, kKVHalf, 1024), idesc_pv,
                                  (j > 0 || k > 0) ? 1u : 0u);
                 }
-                umma_commit(o_done);
+                umma_commit(&o_done[j & 1]);
                 umma_commit(&kv_empty[j & 1]);
             }
             if (!ok) {
@@ -256,41 +274,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float sl = a.scale_log2;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
-        unsigned char* pbase = smem + OFF_P;
         for (int j = 0; j < ntiles; ++j) {
-            if (!mbar_wait_bounded(s_full, j & 1, abort_flag)) {
+            if (!warp_wait(s_full, j & 1, abort_flag)) {
                 ok = false;
                 break;
             }
             tc_fence_after_sync();
-            uint32_t sr[4][32];
+            constexpr int NC = kN / 32;  // 32-column chunks of the S row
+            uint32_t sr[NC][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tmem_s + lane_base + c * 32, sr[c]);
+            for (int c = 0; c < NC; ++c) tmem_ld32(tmem_s + lane_base + c * 32, sr[c]);
             tmem_wait_ld();
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(s_free);
             const int kv0 = j * kN;
-            float mx = -INFINITY;
+            // Work on the raw logits: the scale and the max subtraction fold into one FMA
+            // below.  Keys past a row's limit become the value that scales to -inf; only
+            // tiles that cross some row's limit in this warp pay for the mask.
+            const float masked = sl >= 0.f ? -INFINITY : INFINITY;
+            const bool mask_tile = __any_sync(0xffffffffu, kv0 + kN - 1 > lim);
+            if (mask_tile) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+                for (int c = 0; c < NC; ++c)
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int kv = kv0 + c * 32 + e;
-                    const float x = kv <= lim ? __uint_as_float(sr[c][e]) * sl : -INFINITY;
-                    sr[c][e] = __float_as_uint(x);
-                    mx = fmaxf(mx, x);
-                }
+                    for (int e = 0; e < 32; ++e)
+                        if (kv0 + c * 32 + e > lim) sr[c][e] = __float_as_uint(masked);
+            }
+            float mraw = __uint_as_float(sr[0][0]);
+            if (sl >= 0.f) {
+#pragma unroll
+                for (int c = 0; c < NC; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) mraw = fmaxf(mraw, __uint_as_float(sr[c][e]));
+            } else {
+#pragma unroll
+                for (int c = 0; c < NC; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) mraw = fminf(mraw, __uint_as_float(sr[c][e]));
+            }
+            const float mx = mraw == masked ? -INFINITY : mraw * sl;  // the row's max in base-2 units
             const float m_new = fmaxf(m_used, mx);
             const bool rescale = m_used != -INFINITY && m_new > m_used + (float)kLazyRescale;
-            // the previous tile's P.V has finished: P may be overwritten and O is stable
-            if (j > 0 && !mbar_wait_bounded(o_done, (j - 1) & 1, abort_flag)) {
+            // the whole warp takes the O round trip when any of its rows needs it
+            const bool rescale_warp = __any_sync(0xffffffffu, rescale) != 0;
+            // P buffer j & 1 is free once the P.V of tile j - 2 has finished; O is stable
+            // for a rescale once the P.V of tile j - 1 has (each buffer has its own
+            // barrier, whose next phase is never more than one ahead of the wait)
+            if (j >= 2 && !warp_wait(&o_done[j & 1], ((j - 2) >> 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            if (rescale_warp && j >= 1 && !warp_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)) {
                 ok = false;
                 break;
             }
             tc_fence_after_sync();
-            if (rescale) {
-                const float alpha = fast_exp2(m_used - m_new);
+            if (rescale_warp) {
+                const float alpha = rescale ? fast_exp2(m_used - m_new) : 1.f;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t o[32];
@@ -305,40 +346,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (rescale || m_used == -INFINITY) m_used = m_new;
             const float mref = m_used == -INFINITY ? 0.f : m_used;  // a row with no key yet: every x is -inf
-            // P = 2^(s - m), bf16, into the swizzled P tile (row r: 128 bytes per 64-column half)
-            float rowsum = 0.f;
+            // P = 2^(raw * scale - m) as bf16 pairs into this lane of P buffer j & 1 (32 columns);
+            // the row sum takes P before rounding (two partial sums for more parallel adds)
+            float rs0 = 0.f, rs1 = 0.f;
+            uint32_t w[32];
+            if (!mask_tile) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < NC; ++c)
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e2 = 0; e2 < 4; ++e2) {
-                        const float x0 = __uint_as_float(sr[c][q8 * 8 + e2 * 2]);
-                        const float x1 = __uint_as_float(sr[c][q8 * 8 + e2 * 2 + 1]);
-                        const float p0 = fast_exp2(x0 - mref);
-                        const float p1 = fast_exp2(x1 - mref);
-                        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                        rowsum += __low2float(pb) + __high2float(pb);
-                        w[e2] = *reinterpret_cast<const uint32_t*>(&pb);
+                    for (int e2 = 0; e2 < 16; ++e2) {
+                        const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c][2 * e2]), sl, -mref));
+                        const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c][2 * e2 + 1]), sl, -mref));
+                        rs0 += p0;
+                        rs1 += p1;
+                        w[c * 16 + e2] = pack_bf16(p0, p1);
                     }
-                    const int chunk = c * 4 + q8;  // 16-byte chunk of the row, 0..15
-                    const int h = chunk >> 3;
-                    const int cc = chunk & 7;
-                    *reinterpret_cast<uint4*>(pbase + h * kHalf + r * 128 + ((cc ^ (r & 7)) << 4)) =
-                        make_uint4(w[0], w[1], w[2], w[3]);
-                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < NC; ++c)
+#pragma unroll
+                    for (int e2 = 0; e2 < 16; ++e2) {
+                        const int kv = kv0 + c * 32 + 2 * e2;
+                        const float p0 = kv <= lim ? fast_exp2(fmaf(__uint_as_float(sr[c][2 * e2]), sl, -mref)) : 0.f;
+                        const float p1 =
+                            kv + 1 <= lim ? fast_exp2(fmaf(__uint_as_float(sr[c][2 * e2 + 1]), sl, -mref)) : 0.f;
+                        rs0 += p0;
+                        rs1 += p1;
+                        w[c * 16 + e2] = pack_bf16(p0, p1);
+                    }
             }
+            const float rowsum = rs0 + rs1;
+            tmem_st32(tmem_p + (j & 1) * 32 + lane_base, w);
+            tmem_wait_st();
             l += rowsum;
             // keys past the context in this tile: zero their V rows (0-weights must meet finite values)
             if (kv0 + kN > L) {
-                unsigned char* vb = smem + OFF_V + (j & 1) * kTile;
+                unsigned char* vb = smem + OFF_V + (j & 1) * 2 * kKVHalf;
                 const int first = max(0, L - kv0);
                 const int chunks = (kN - first) * 16;  // 16-byte chunks over both halves
                 for (int i = r; i < chunks; i += 128) {
                     const int row = first + (i >> 4);
                     const int h = (i >> 3) & 1;
-                    *reinterpret_cast<uint4*>(vb + h * kHalf + row * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(vb + h * kKVHalf + row * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
                 }
             }
             fence_async_smem();
@@ -346,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full);
         }
-        if (ok && mbar_wait_bounded(o_done, (ntiles - 1) & 1, abort_flag)) {
+        if (ok && warp_wait(&o_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort_flag)) {
             tc_fence_after_sync();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) +
@@ -414,6 +463,8 @@ cudaError_t launch_g(const PrefillArgs& a, int num_query_tokens, int max_query_l
     cudaGetDevice(&dev);
     if (!attr_done[dev & 63]) {
         e = cudaFuncSetAttribute(prefill_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(prefill_tc_kernel<G>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (e != cudaSuccess) return e;
         attr_done[dev & 63] = true;
     }

@@ -154,3 +154,12 @@ def test_prefill_workload_full_size_sampled(pa):
             vs.append(values[koff[s]:koff[s] + pos + 1].float().numpy())
     ref = oracle_logical(q[rows].float().numpy(), ks, vs, wl.block_size, wl.scale)
     assert max_abs(got[rows], ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.06, 0.3])
+def test_any_finite_scale(pa, scale):
+    lens, nq = [130, 70], [130, 20]
+    q, k, v, tables, L, qs = _case(21, lens, nq, 8, 2, 16)
+    got = _run(pa, q, k, v, tables, L, qs, scale)
+    assert np.isfinite(got).all()
+    assert max_abs(got, _oracle(q, k, v, tables, L, qs, scale)) <= TOL["bf16"]

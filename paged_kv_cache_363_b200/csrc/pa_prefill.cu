@@ -11,9 +11,9 @@
 // A CTA owns one (sequence, kv head, query tile).  The tile's 128 rows are T query
 // tokens x G query heads of the kv head's group (T = 128 / G), so every K/V byte the
 // CTA loads serves all G heads.  It walks the keys in tiles of 64 tokens:
-//   - warp 4 stages Q once and each K/V tile by TMA, one 16-row box per (16-token run
-//     of a physical block, 64 columns), 128-byte swizzle, two stages; lane i looks up
-//     and issues box i of the tile;
+//   - warp 4 stages Q once and each K and V tile by TMA, one 16-row box per (16-token
+//     run of a physical block, 64 columns), 128-byte swizzle, K in three stages and V
+//     in two; lane i looks up and issues box i of the tile;
 //   - warp 5 (one thread) issues S = Q K^T (M=128, N=64, K=128: 8 MMAs) into tensor
 //     memory, and O += P V (N=128, K=64: 4 MMAs, A = P from tensor memory, B operand
 //     MN-major) once P is ready; the next
@@ -53,19 +53,24 @@ constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 256;  // S: 0..63, P: 64..95 and 96..127, O: 128..255 (two CTAs fill the 512)
 constexpr uint32_t kLazyRescale = 8; // base-2 units
 
-// Tiles, from a 1024-byte aligned base: Q (32 KB), K and V in two stages (16 KB
-// each): 96 KB.  P lives in tensor memory (two buffers, the A operand of P.V).  The
-// barriers go in the alignment slack when it has room, else after the tiles; two
-// CTAs share an SM.
+// Tiles, from a 1024-byte aligned base: Q (32 KB), K in three stages and V in two
+// (16 KB each): 112 KB.  K and V have rings of their own: a K stage is free again as
+// soon as its S = Q K^T has run, so the next K tiles load a whole softmax earlier than
+// a shared K/V stage (freed only by P.V) would allow.  P lives in tensor memory (two
+// buffers, the A operand of P.V).  The barriers go in the alignment slack when it has
+// room, else after the tiles, so the request fits two CTAs per SM
+// (2 x (113 KB + 1 KB reserved) = 228 KB).
+constexpr int KST = 3, VST = 2;
 constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + 2 * kQHalf;
-constexpr int OFF_V = OFF_K + 2 * 2 * kKVHalf;
-constexpr int kTiles = OFF_V + 2 * 2 * kKVHalf;
-// barriers: q_full, kv_full[2], kv_empty[2], s_full, s_free, p_full, o_done[2], drain
-constexpr int NBAR = 11;
-constexpr int kMisc = 128;          // barriers, TMEM base, abort flag
-constexpr int kSmem = kTiles + 1024 + kMisc;
+constexpr int OFF_V = OFF_K + KST * 2 * kKVHalf;
+constexpr int kTiles = OFF_V + VST * 2 * kKVHalf;
+// barriers: q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full, s_free, p_full, o_done[2], drain
+constexpr int NBAR = 17;
+constexpr int kMisc = 160;          // barriers, TMEM base, abort flag
+constexpr int kSmem = 113 * 1024;
 static_assert(kTiles + 1023 <= kSmem, "tiles fit with any base alignment");
+static_assert((kMisc - 1) + kTiles + kMisc <= kSmem, "misc after the tiles when the slack is short");
 static_assert(NBAR * 8 + 16 <= kMisc, "misc area");
 
 // 2^x by the hardware approximation (ex2.approx, relative error about 2^-22; 2^-inf = 0).
@@ -120,13 +125,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     unsigned char* misc = slack >= (uint32_t)kMisc ? smem_raw : smem + kTiles;
     uint64_t* bars = reinterpret_cast<uint64_t*>(misc);
     uint64_t* q_full = bars + 0;
-    uint64_t* kv_full = bars + 1;   // [2]
-    uint64_t* kv_empty = bars + 3;  // [2]
-    uint64_t* s_full = bars + 5;
-    uint64_t* s_free = bars + 6;
-    uint64_t* p_full = bars + 7;
-    uint64_t* o_done = bars + 8;    // [2]: P.V of the tiles using P buffer 0 / 1
-    uint64_t* drain = bars + 10;
+    uint64_t* k_full = bars + 1;    // [KST]
+    uint64_t* k_empty = bars + 4;   // [KST]
+    uint64_t* v_full = bars + 7;    // [VST]
+    uint64_t* v_empty = bars + 9;   // [VST]
+    uint64_t* s_full = bars + 11;
+    uint64_t* s_free = bars + 12;
+    uint64_t* p_full = bars + 13;
+    uint64_t* o_done = bars + 14;   // [2]: P.V of the tiles using P buffer 0 / 1
+    uint64_t* drain = bars + 16;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + NBAR * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + NBAR * 8 + 8);
     const int warp = threadIdx.x >> 5;
@@ -134,9 +141,13 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&kv_full[i], 1);
-            mbar_init(&kv_empty[i], 1);
+        for (int i = 0; i < KST; ++i) {
+            mbar_init(&k_full[i], 1);
+            mbar_init(&k_empty[i], 1);
+        }
+        for (int i = 0; i < VST; ++i) {
+            mbar_init(&v_full[i], 1);
+            mbar_init(&v_empty[i], 1);
         }
         mbar_init(s_full, 1);
         mbar_init(s_free, 4);
@@ -169,7 +180,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int32_t* table = a.block_tables + (size_t)s * a.max_blocks_per_seq;
         bool ok = true;
         for (int j = 0; j < ntiles && ok; ++j) {
-            const int st = j & 1;
             const int tok0 = j * kN;
             const int nbox = min(kN / kBox, (L - tok0 + kBox - 1) / kBox);
             const int tok = tok0 + lane * kBox;
@@ -181,20 +191,32 @@ __global__ void __launch_bounds__(kThreads, 2)
                     phys = 0;
                 }
             }
+            const int row = (phys * a.num_kv_heads + kvh) * a.block_size + tok % a.block_size;
+            const uint32_t tx = (uint32_t)nbox * kBox * 128 * 2;  // both halves of the boxes
+            // K tile j into K stage j % KST, free once S of tile j - KST has run
+            const int ks = j % KST;
             if (lane == 0) {
-                if (j >= 2 && !mbar_wait_bounded(&kv_empty[st], ((j >> 1) & 1) ^ 1, abort_flag)) ok = false;
-                if (ok) mbar_arrive_expect_tx(&kv_full[st], (uint32_t)nbox * kBox * 128 * 4);
+                if (j >= KST && !mbar_wait_bounded(&k_empty[ks], ((j / KST) & 1) ^ 1, abort_flag)) ok = false;
+                if (ok) mbar_arrive_expect_tx(&k_full[ks], tx);
             }
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (!ok) break;
-            if (lane < nbox) {
-                const int row = (phys * a.num_kv_heads + kvh) * a.block_size + tok % a.block_size;
-                for (int h = 0; h < 2; ++h) {
-                    const int off = st * 2 * kKVHalf + h * kKVHalf + lane * kBox * 128;
-                    tma_load_2d(smem_u32(smem + OFF_K + off), &tmap_k, h * 64, row, &kv_full[st], pol);
-                    tma_load_2d(smem_u32(smem + OFF_V + off), &tmap_v, h * 64, row, &kv_full[st], pol);
-                }
+            if (lane < nbox)
+                for (int h = 0; h < 2; ++h)
+                    tma_load_2d(smem_u32(smem + OFF_K + ks * 2 * kKVHalf + h * kKVHalf + lane * kBox * 128), &tmap_k,
+                                h * 64, row, &k_full[ks], pol);
+            // V tile j into V stage j % VST, free once P.V of tile j - VST has run
+            const int vs = j % VST;
+            if (lane == 0) {
+                if (j >= VST && !mbar_wait_bounded(&v_empty[vs], ((j / VST) & 1) ^ 1, abort_flag)) ok = false;
+                if (ok) mbar_arrive_expect_tx(&v_full[vs], tx);
             }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            if (lane < nbox)
+                for (int h = 0; h < 2; ++h)
+                    tma_load_2d(smem_u32(smem + OFF_V + vs * 2 * kKVHalf + h * kKVHalf + lane * kBox * 128), &tmap_v,
+                                h * 64, row, &v_full[vs], pol);
         }
         if (lane == 0) {
             if (!ok) {
@@ -204,8 +226,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             // no copy may still be landing in shared memory at exit
             volatile int never = 0;
             if (!mbar_wait_bounded(q_full, 0, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
-            for (int j = max(0, ntiles - 2); j < ntiles; ++j)
-                if (!mbar_wait_bounded(&kv_full[j & 1], (j >> 1) & 1, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+            for (int j = max(0, ntiles - KST); j < ntiles; ++j)
+                if (!mbar_wait_bounded(&k_full[j % KST], (j / KST) & 1, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+            for (int j = max(0, ntiles - VST); j < ntiles; ++j)
+                if (!mbar_wait_bounded(&v_full[j % VST], (j / VST) & 1, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
         }
     } else if (warp == 5) {
         // ---------------- MMA issuer
@@ -213,9 +237,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             constexpr uint32_t idesc_qk = umma_idesc_bf16(kM, kN, false);
             constexpr uint32_t idesc_pv = umma_idesc_bf16(kM, kD, true);
             const uint32_t sq = smem_u32(smem + OFF_Q), sk = smem_u32(smem + OFF_K), sv = smem_u32(smem + OFF_V);
-            bool ok = mbar_wait_bounded(q_full, 0, abort_flag) && mbar_wait_bounded(&kv_full[0], 0, abort_flag);
+            bool ok = mbar_wait_bounded(q_full, 0, abort_flag) && mbar_wait_bounded(&k_full[0], 0, abort_flag);
             auto issue_qk = [&](int j) {
-                const uint32_t kb = sk + (j & 1) * 2 * kKVHalf;
+                const uint32_t kb = sk + (j % KST) * 2 * kKVHalf;
 #pragma unroll
                 for (int k = 0; k < kD / 16; ++k) {
                     const uint32_t kk = (k & 3) * 32;
@@ -223,6 +247,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                                  umma_desc_sw128(kb + (k >> 2) * kKVHalf + kk, 16, 1024), idesc_qk, k > 0 ? 1u : 0u);
                 }
                 umma_commit(s_full);
+                umma_commit(&k_empty[j % KST]);
             };
             if (ok) {
                 tc_fence_after_sync();
@@ -230,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             for (int j = 0; j < ntiles && ok; ++j) {
                 if (j + 1 < ntiles) {
-                    if (!mbar_wait_bounded(&kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag) ||
+                    if (!mbar_wait_bounded(&k_full[(j + 1) % KST], ((j + 1) / KST) & 1, abort_flag) ||
                         !mbar_wait_bounded(s_free, j & 1, abort_flag)) {
                         ok = false;
                         break;
@@ -238,12 +263,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                     tc_fence_after_sync();
                     issue_qk(j + 1);
                 }
-                if (!mbar_wait_bounded(p_full, j & 1, abort_flag)) {
+                if (!mbar_wait_bounded(p_full, j & 1, abort_flag) ||
+                    !mbar_wait_bounded(&v_full[j % VST], (j / VST) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after_sync();
-                const uint32_t vb = sv + (j & 1) * 2 * kKVHalf;
+                const uint32_t vb = sv + (j % VST) * 2 * kKVHalf;
 #pragma unroll
                 for (int k = 0; k < kN / 16; ++k) {
                     umma_bf16_ts(tmem_o, tmem_p + (j & 1) * 32 + k * 8,
@@ -251,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                                  (j > 0 || k > 0) ? 1u : 0u);
                 }
                 umma_commit(&o_done[j & 1]);
-                umma_commit(&kv_empty[j & 1]);
+                umma_commit(&v_empty[j % VST]);
             }
             if (!ok) {
                 atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
@@ -381,7 +407,12 @@ __global__ void __launch_bounds__(kThreads, 2)
             l += rowsum;
             // keys past the context in this tile: zero their V rows (0-weights must meet finite values)
             if (kv0 + kN > L) {
-                unsigned char* vb = smem + OFF_V + (j & 1) * 2 * kKVHalf;
+                // the tile's V copies (boxes with tokens past the context included) have landed
+                if (!warp_wait(&v_full[j % VST], (j / VST) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                unsigned char* vb = smem + OFF_V + (j % VST) * 2 * kKVHalf;
                 const int first = max(0, L - kv0);
                 const int chunks = (kN - first) * 16;  // 16-byte chunks over both halves
                 for (int i = r; i < chunks; i += 128) {

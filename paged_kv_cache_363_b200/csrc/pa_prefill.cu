@@ -327,18 +327,41 @@ __global__ void __launch_bounds__(kThreads, 2)
                     for (int e = 0; e < 32; ++e)
                         if (kv0 + c * 32 + e > lim) sr[c][e] = __float_as_uint(masked);
             }
-            float mraw = __uint_as_float(sr[0][0]);
+            // eight independent partial maxima (short dependency chains), then a tree
+            float m0 = masked, m1 = masked, m2 = masked, m3 = masked, m4 = masked, m5 = masked, m6 = masked,
+                  m7 = masked;
             if (sl >= 0.f) {
 #pragma unroll
                 for (int c = 0; c < NC; ++c)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) mraw = fmaxf(mraw, __uint_as_float(sr[c][e]));
+                    for (int e = 0; e < 32; e += 8) {
+                        m0 = fmaxf(m0, __uint_as_float(sr[c][e + 0]));
+                        m1 = fmaxf(m1, __uint_as_float(sr[c][e + 1]));
+                        m2 = fmaxf(m2, __uint_as_float(sr[c][e + 2]));
+                        m3 = fmaxf(m3, __uint_as_float(sr[c][e + 3]));
+                        m4 = fmaxf(m4, __uint_as_float(sr[c][e + 4]));
+                        m5 = fmaxf(m5, __uint_as_float(sr[c][e + 5]));
+                        m6 = fmaxf(m6, __uint_as_float(sr[c][e + 6]));
+                        m7 = fmaxf(m7, __uint_as_float(sr[c][e + 7]));
+                    }
+                m0 = fmaxf(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)), fmaxf(fmaxf(m4, m5), fmaxf(m6, m7)));
             } else {
 #pragma unroll
                 for (int c = 0; c < NC; ++c)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) mraw = fminf(mraw, __uint_as_float(sr[c][e]));
+                    for (int e = 0; e < 32; e += 8) {
+                        m0 = fminf(m0, __uint_as_float(sr[c][e + 0]));
+                        m1 = fminf(m1, __uint_as_float(sr[c][e + 1]));
+                        m2 = fminf(m2, __uint_as_float(sr[c][e + 2]));
+                        m3 = fminf(m3, __uint_as_float(sr[c][e + 3]));
+                        m4 = fminf(m4, __uint_as_float(sr[c][e + 4]));
+                        m5 = fminf(m5, __uint_as_float(sr[c][e + 5]));
+                        m6 = fminf(m6, __uint_as_float(sr[c][e + 6]));
+                        m7 = fminf(m7, __uint_as_float(sr[c][e + 7]));
+                    }
+                m0 = fminf(fminf(fminf(m0, m1), fminf(m2, m3)), fminf(fminf(m4, m5), fminf(m6, m7)));
             }
+            const float mraw = m0;
             const float mx = mraw == masked ? -INFINITY : mraw * sl;  // the row's max in base-2 units
             const float m_new = fmaxf(m_used, mx);
             const bool rescale = m_used != -INFINITY && m_new > m_used + (float)kLazyRescale;
@@ -374,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const float mref = m_used == -INFINITY ? 0.f : m_used;  // a row with no key yet: every x is -inf
             // P = 2^(raw * scale - m) as bf16 pairs into this lane of P buffer j & 1 (32 columns);
             // the row sum takes P before rounding (two partial sums for more parallel adds)
-            float rs0 = 0.f, rs1 = 0.f;
+            float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;  // independent partial sums
             uint32_t w[32];
             if (!mask_tile) {
 #pragma unroll
@@ -383,8 +406,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                     for (int e2 = 0; e2 < 16; ++e2) {
                         const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c][2 * e2]), sl, -mref));
                         const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c][2 * e2 + 1]), sl, -mref));
-                        rs0 += p0;
-                        rs1 += p1;
+                        if (e2 & 1) {
+                            rs2 += p0;
+                            rs3 += p1;
+                        } else {
+                            rs0 += p0;
+                            rs1 += p1;
+                        }
                         w[c * 16 + e2] = pack_bf16(p0, p1);
                     }
             } else {
@@ -396,12 +424,17 @@ __global__ void __launch_bounds__(kThreads, 2)
                         const float p0 = kv <= lim ? fast_exp2(fmaf(__uint_as_float(sr[c][2 * e2]), sl, -mref)) : 0.f;
                         const float p1 =
                             kv + 1 <= lim ? fast_exp2(fmaf(__uint_as_float(sr[c][2 * e2 + 1]), sl, -mref)) : 0.f;
-                        rs0 += p0;
-                        rs1 += p1;
+                        if (e2 & 1) {
+                            rs2 += p0;
+                            rs3 += p1;
+                        } else {
+                            rs0 += p0;
+                            rs1 += p1;
+                        }
                         w[c * 16 + e2] = pack_bf16(p0, p1);
                     }
             }
-            const float rowsum = rs0 + rs1;
+            const float rowsum = (rs0 + rs1) + (rs2 + rs3);
             tmem_st32(tmem_p + (j & 1) * 32 + lane_base, w);
             tmem_wait_st();
             l += rowsum;

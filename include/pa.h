@@ -196,6 +196,17 @@ PA_API pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* blo
 PA_API pa_status pa_device_status(uint32_t* flags, void* stream);
 
 /*
+ * Failure-path self-test (no counterpart in the pages; it exercises the library's
+ * own failure detection).  Launches one thread that waits, with the kernels' bounded
+ * wait and time limit (2 s), on an mbarrier nothing ever arrives at.  The wait gives
+ * up, PA_DEV_WAIT_TIMEOUT is raised in the status word (read it with
+ * pa_device_status) and the kernel returns; nothing faults or hangs, and the context
+ * stays usable.  Blocks until done; *waited_ns (nullable, host) receives how long the
+ * wait lasted on the device clock.
+ */
+PA_API pa_status pa_selftest_bounded_wait(uint64_t* waited_ns, void* stream);
+
+/*
  * Chunked prefill over the paged cache ([INIT] section 3: a prompt's blocks are
  * assigned when it is processed; [FSAH] section 2: token t of a sequence lives at
  * slot T[t / B] * B + t % B), on the tensor cores.  Sequence s holds

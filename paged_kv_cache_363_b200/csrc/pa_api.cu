@@ -414,6 +414,18 @@ pa_status pa_swap_blocks(void* dst_k_cache, void* dst_v_cache, const void* src_k
     return PA_OK;
 }
 
+pa_status pa_selftest_bounded_wait(uint64_t* waited_ns, void* stream)
+{
+    unsigned int* status = nullptr;
+    pa_status st = status_ptr(&status);
+    if (st != PA_OK) return st;
+    unsigned long long ns = 0;
+    const cudaError_t e = launch_wait_selftest(status, &ns, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail("pa_selftest_bounded_wait", e);
+    if (waited_ns) *waited_ns = (uint64_t)ns;
+    return PA_OK;
+}
+
 pa_status pa_device_status(uint32_t* flags, void* stream)
 {
     if (!flags) return PA_ERR_INVALID;

@@ -147,4 +147,7 @@ struct SwapArgs {
 
 cudaError_t launch_swap_blocks(const SwapArgs& a, cudaStream_t stream);
 
+// One bounded wait on an mbarrier nothing arrives at (pa_selftest.cu); blocks until done.
+cudaError_t launch_wait_selftest(unsigned int* status, unsigned long long* waited_ns, cudaStream_t stream);
+
 }  // namespace pa

@@ -43,6 +43,7 @@ SIGNATURES = [
     ("pa_copy_blocks", _int, [_vp, _vp, _vp] + [_int] * 6 + [_vp]),
     ("pa_swap_blocks", _int, [_vp, _vp, _vp, _vp, _vp] + [_int] * 7 + [_vp]),
     ("pa_device_status", _int, [ctypes.POINTER(_u32), _vp]),
+    ("pa_selftest_bounded_wait", _int, [ctypes.POINTER(ctypes.c_uint64), _vp]),
     ("pa_alloc_create", _vp, [_int, _int, _vp]),
     ("pa_alloc_destroy", None, [_vp]),
     ("pa_alloc_add_seq", _int, [_vp, _i64, _int, _vp]),
@@ -261,6 +262,14 @@ def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None):
     st = lib.pa_copy_blocks(_dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"), ptr, n, Hkv, D, B, NB,
                             _dtype_code(k_cache), _stream(stream))
     _check(st, "pa_copy_blocks")
+
+
+def pa_selftest_bounded_wait(stream=None):
+    """Makes one bounded device wait run out (nothing arrives); returns the nanoseconds it
+    waited.  PA_DEV_WAIT_TIMEOUT is then set in the status word."""
+    ns = ctypes.c_uint64(0)
+    _check(lib.pa_selftest_bounded_wait(ctypes.byref(ns), _stream(stream)), "pa_selftest_bounded_wait")
+    return int(ns.value)
 
 
 def pa_device_status(stream=None):

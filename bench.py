@@ -70,21 +70,23 @@ def measured_hbm_peak():
 
 
 DECODE_SOURCES = ("pa_decode.cu", "pa_decode_common.cuh", "pa_decode_fma.cuh", "pa_decode_mma.cuh", "pa_ptx.cuh")
+PREFILL_SOURCES = ("pa_prefill.cu", "pa_tcgen05.cuh", "pa_ptx.cuh")
 
 
-def decode_source_hash():
-    """Hash of the decode kernel sources (ties a committed profile to the code it measured)."""
+def decode_source_hash(sources=None):
+    """Hash of a kernel's sources (ties a committed profile to the code it measured);
+    the decode kernel's by default."""
     import hashlib
     h = hashlib.sha256()
-    for name in DECODE_SOURCES:
+    for name in (DECODE_SOURCES if sources is None else sources):
         with open(os.path.join(ROOT, "paged_kv_cache_363_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profile_traffic(kernel, workload):
+def profile_traffic(kernel, workload, sources=None):
     """dram bytes per launch from the committed ncu summary for this kernel and workload,
-    if its recorded source hash still matches the decode sources; else None."""
+    if its recorded source hash still matches the kernel's sources; else None."""
     path = os.path.join(ROOT, "profiles", "%s_%s.md" % (kernel, workload))
     try:
         fields = {}
@@ -93,7 +95,7 @@ def profile_traffic(kernel, workload):
                 if ":" in line and line.startswith("- "):
                     k, v = line[2:].split(":", 1)
                     fields[k.strip()] = v.strip().strip("`")
-        if fields.get("source_sha256_16") != decode_source_hash():
+        if fields.get("source_sha256_16") != decode_source_hash(sources):
             return None
         return float(fields["traffic_bytes_per_launch"])
     except Exception:
@@ -472,7 +474,8 @@ def run_prefill(args, wl, batch, dev, stream, world):
                        parallelism="replicas: one batch per GPU (dp%d)" % world),
         "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel", "achieved": round(achieved, 2),
                      "peak": peak, "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "traffic": None, "algorithmic_flops_per_launch": flops, "avg_launch_us": round(avg * 1e3, 3)},
+                     "traffic": profile_traffic("prefill_tc_kernel", wl.name, PREFILL_SOURCES),
+                     "algorithmic_flops_per_launch": flops, "avg_launch_us": round(avg * 1e3, 3)},
         "e2e": {"value": round(world * flops * args.steps / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": qh.numel() * qh.element_size(),
                 "d2h_bytes_per_step": oh.numel() * oh.element_size(), "ms_per_step": round(e2e_ms / args.steps, 5)},

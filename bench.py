@@ -23,6 +23,7 @@ only), on a bounded sample of sequences of the same workload per step.
 import argparse
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -74,13 +75,19 @@ PREFILL_SOURCES = ("pa_prefill.cu", "pa_tcgen05.cuh", "pa_ptx.cuh")
 
 
 def decode_source_hash(sources=None):
-    """Hash of a kernel's sources (ties a committed profile to the code it measured);
-    the decode kernel's by default."""
+    """Hash of a kernel's code (ties a committed profile to the code it measured); the
+    decode kernel's by default.  Comments and whitespace are left out, so rewording a
+    comment keeps a profile valid; any change to the code does not."""
     import hashlib
     h = hashlib.sha256()
     for name in (DECODE_SOURCES if sources is None else sources):
-        with open(os.path.join(ROOT, "paged_kv_cache_363_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "paged_kv_cache_363_b200", "csrc", name)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        for line in text.splitlines():
+            code = re.sub(r"//.*", "", line).split()
+            if code:
+                h.update((" ".join(code) + "\n").encode())
     return h.hexdigest()[:16]
 
 
@@ -95,7 +102,7 @@ def profile_traffic(kernel, workload, sources=None):
                 if ":" in line and line.startswith("- "):
                     k, v = line[2:].split(":", 1)
                     fields[k.strip()] = v.strip().strip("`")
-        if fields.get("source_sha256_16") != decode_source_hash(sources):
+        if (fields.get("source_sha256_16") or "").split(" ")[0] != decode_source_hash(sources):
             return None
         return float(fields["traffic_bytes_per_launch"])
     except Exception:

@@ -17,8 +17,8 @@
 //  * In each CTA one warp fetches units ahead of use (block-table slice and q into a
 //    small shared ring), one thread streams the units' K/V tiles into a ring of
 //    shared-memory stages with the TMA engine (1-D bulk copies of whole tiles, or 2-D
-//    tensor boxes with the 128-byte swizzle for the tensor-core consumer; never
-//    multicast) and four consumer warps take alternate blocks.  The stream of tiles
+//    tensor boxes with the 128-byte swizzle for the tensor-core consumer; each CTA
+//    loads its own tiles) and four consumer warps take alternate blocks.  The stream of tiles
 //    runs across unit boundaries, so the pipeline does not drain between units.
 //  * Consumers: CUDA cores (fp32; bf16 with one query head per kv head) or tensor
 //    cores (bf16 with 2, 4 or 8 query heads per kv head); see the two policy headers.

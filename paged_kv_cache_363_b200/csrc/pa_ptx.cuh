@@ -1,5 +1,5 @@
 // Inline-PTX helpers for sm_100a: mbarriers, 1-D bulk global->shared copies (the
-// TMA engine's untiled form; no tensor map, no multicast), bounded waits, and
+// TMA engine's untiled form; no tensor map, one CTA's own copy), bounded waits, and
 // programmatic-dependent-launch controls.
 #pragma once
 

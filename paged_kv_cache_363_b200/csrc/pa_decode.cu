@@ -22,9 +22,10 @@
 //    runs across unit boundaries, so the pipeline does not drain between units.
 //  * Consumers: CUDA cores (fp32; bf16 with one query head per kv head) or tensor
 //    cores (bf16 with 2, 4 or 8 query heads per kv head); see the two policy headers.
-//  * At the end of a unit the four warps' softmax states are merged; a sequence
-//    longer than one partition leaves (max, sum, unnormalised output) per partition in
-//    the workspace and a log-sum-exp merge kernel combines them.  Plan, persistent and
+//  * At the end of a unit each warp leaves its softmax state in shared memory and goes
+//    on with the next unit; the warp that consumed the unit's last tile merges the four
+//    states.  A sequence longer than one partition leaves (max, sum, unnormalised
+//    output) per partition in the workspace and a log-sum-exp merge kernel combines them.  Plan, persistent and
 //    merge kernels are chained with programmatic dependent launch.
 //  * Logits are kept in base-2 units (q pre-scaled by scale*log2 e) and exponentials
 //    use exp2f, the reformulation of online softmax by Milakov & Gimelshein (2018).

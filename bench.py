@@ -395,6 +395,40 @@ def companion_timing(batch, stream, reps=50, num_pairs=96):
     return out
 
 
+def plan_once_timing(batch, stream, dec_bytes, args):
+    """A serving step runs decode attention once per layer over the same sequences: plan
+    once (pa_decode_plan), then one pa_decode_run per layer.  Times the run alone, and
+    the plan alone, with CUDA events; GB/s of the run over the same algorithmic bytes."""
+    import torch
+    from paged_kv_cache_363_b200 import pa
+
+    wl = batch.wl
+    part = batch.partition_size
+    ws = batch.workspace_for(part)
+    out = torch.empty_like(batch.q)
+    plan = lambda: pa.pa_decode_plan(batch.block_tables, batch.context_lens, batch.max_context_len, wl.num_heads,
+                                     batch.k_cache, ws, part, stream=stream)
+    run = lambda: pa.pa_decode_run(out, batch.q, batch.k_cache, batch.v_cache, batch.block_tables,
+                                   batch.context_lens, batch.max_context_len, wl.scale, ws, part, stream=stream)
+    plan()
+    for _ in range(max(3, args.warmup)):
+        run()
+    res = {}
+    for name, fn in (("run", run), ("plan", plan)):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(100)]
+        for a, b in ev:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize(batch.device)
+        res[name] = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    plan()   # leave a fresh plan
+    torch.cuda.synchronize(batch.device)
+    return {"run_us": round(res["run"] * 1e3, 3), "run_gbs": round(dec_bytes / (res["run"] * 1e-3) / 1e9, 1),
+            "plan_us": round(res["plan"] * 1e3, 3),
+            "note": "one plan per step, one run per layer; the run is the persistent decode kernel and the merge"}
+
+
 def e2e_leg(stepper, args, world, dev):
     """Device time of `args.steps` host-fed steps (upload, kernels, read-back), max over ranks."""
     import torch
@@ -596,6 +630,7 @@ def run_gpu(args):
                           "buffers": 1, "cuda_graph": False}}
 
     companions = companion_timing(batch, stream) if not args.skip_e2e else None
+    plan_once = plan_once_timing(batch, stream, dec_bytes, args) if not args.skip_e2e else None
 
     peak, peak_kind = measured_hbm_peak()
     achieved = dec_bytes / (dec_avg_max * 1e-3) / 1e9
@@ -615,6 +650,7 @@ def run_gpu(args):
                      "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_us": round(dec_avg_max * 1e3, 3),
                      "launch_us_p10_p50_p90": [round(float(np.percentile(dec_ms, q)) * 1e3, 3) for q in (10, 50, 90)]},
         "companions": companions,
+        "plan_once": plan_once,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),

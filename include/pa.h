@@ -125,6 +125,27 @@ PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const 
                     size_t workspace_bytes, pa_dtype dtype, void* stream);
 
 /*
+ * pa_decode in two parts, for a decode step that runs the attention of many layers
+ * over the same sequences (the same block_tables, context_lens and sizes; other q,
+ * out and caches per layer).  pa_decode_plan writes the work plan into the workspace
+ * (the plan kernel only; no q, out or caches); pa_decode_run then runs the decode
+ * from that plan and may be called any number of times: the last CTA of each run
+ * resets the plan's work counter.  A run must use the workspace, block_tables,
+ * context_lens and every size argument of its plan (the caller's promise; nothing
+ * checks it), and follow it in stream order.  pa_decode is the plan followed by one
+ * run.  Errors as for pa_decode.
+ */
+PA_API pa_status pa_decode_plan(const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                                int num_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                                int num_blocks, int max_context_len, int partition_size, void* workspace,
+                                size_t workspace_bytes, pa_dtype dtype, void* stream);
+PA_API pa_status pa_decode_run(void* out, const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_heads,
+                               int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+                               int max_context_len, float scale, int partition_size, void* workspace,
+                               size_t workspace_bytes, pa_dtype dtype, void* stream);
+
+/*
  * Fixed size of the library's own decode workspace used by
  * pa_decode_static_workspace: 16 MiB of device memory on every GPU that loads
  * the library, held until the process exits.

@@ -138,41 +138,51 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, i
     return decode_workspace((size_t)num_seqs, (size_t)num_heads, (size_t)head_dim, np).total;
 }
 
-pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
-                    const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_heads,
-                    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
-                    int max_context_len, float scale, int partition_size, void* workspace,
-                    size_t workspace_bytes, pa_dtype dtype, void* stream)
+}  // extern "C"
+
+namespace pa {
+namespace {
+
+// pa_decode, pa_decode_plan and pa_decode_run: the same checks and arguments, then the
+// plan kernel, the persistent kernel and merge, or both.  The plan phase does not
+// touch out, q or the caches (they may be null).
+pa_status decode_call(const char* fn, int phases, void* out, const void* q, const void* k_cache,
+                      const void* v_cache, const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                      int num_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                      int num_blocks, int max_context_len, float scale, int partition_size, void* workspace,
+                      size_t workspace_bytes, pa_dtype dtype, void* stream)
 {
-    pa_status st = check_common("pa_decode", num_kv_heads, head_dim, block_size, num_blocks, dtype);
+    const std::string name(fn);
+    pa_status st = check_common(fn, num_kv_heads, head_dim, block_size, num_blocks, dtype);
     if (st != PA_OK) return st;
     if (num_seqs < 0 || num_seqs > 65535 || num_heads <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 ||
         partition_size < 0 || !std::isfinite(scale)) {
-        set_error("pa_decode: bad size or scale");
+        set_error(name + ": bad size or scale");
         return PA_ERR_INVALID;
     }
     if (num_heads % num_kv_heads != 0) {
-        set_error("pa_decode: num_heads must be a multiple of num_kv_heads");
+        set_error(name + ": num_heads must be a multiple of num_kv_heads");
         return PA_ERR_INVALID;
     }
     const int group = num_heads / num_kv_heads;
     if (group != 1 && group != 2 && group != 4 && group != 8) {
-        set_error("pa_decode: num_heads / num_kv_heads must be 1, 2, 4 or 8");
+        set_error(name + ": num_heads / num_kv_heads must be 1, 2, 4 or 8");
         return PA_ERR_UNSUPPORTED;
     }
     if (num_seqs == 0) return PA_OK;
-    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) {
-        set_error("pa_decode: null pointer");
+    const bool run = (phases & kDecodeRun) != 0;
+    if ((run && (!out || !q || !k_cache || !v_cache)) || !block_tables || !context_lens) {
+        set_error(name + ": null pointer");
         return PA_ERR_INVALID;
     }
-    if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+    if ((run && (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))) ||
         !aligned(block_tables, 4) || !aligned(context_lens, 4)) {
-        set_error("pa_decode: misaligned pointer (q, out, caches need 16 bytes)");
+        set_error(name + ": misaligned pointer (q, out, caches need 16 bytes)");
         return PA_ERR_INVALID;
     }
     if (decode_uses_tensor_cores(dtype, head_dim, group) &&
         (int64_t)num_blocks * num_kv_heads * block_size > (int64_t)INT32_MAX) {
-        set_error("pa_decode: num_blocks * num_kv_heads * block_size must stay below 2^31 (tensor-copy row index)");
+        set_error(name + ": num_blocks * num_kv_heads * block_size must stay below 2^31 (tensor-copy row index)");
         return PA_ERR_UNSUPPORTED;
     }
     const int p = resolve_partition(block_size, max_context_len, partition_size);
@@ -180,7 +190,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     const int np = max_context_len > 0 ? (max_context_len + p - 1) / p : 1;
     const DecodeWorkspace wl = decode_workspace((size_t)num_seqs, (size_t)num_heads, (size_t)head_dim, (size_t)np);
     if (!workspace || workspace_bytes < wl.total || !aligned(workspace, 16)) {
-        set_error("pa_decode: workspace missing, too small (need " + std::to_string(wl.total) +
+        set_error(name + ": workspace missing, too small (need " + std::to_string(wl.total) +
                   " bytes) or not 16-byte aligned");
         return PA_ERR_INVALID;
     }
@@ -213,10 +223,48 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     a.adaptive = partition_size == 0 ? 1 : 0;
     a.num_partitions = np;
     a.scale_log2 = scale * 1.4426950408889634f;
+    a.phases = phases;
     const cudaError_t e =
         launch_decode(a, dtype, head_dim, block_size, group, static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail("pa_decode launch", e);
+    if (e != cudaSuccess) return cuda_fail((name + " launch").c_str(), e);
     return PA_OK;
+}
+
+}  // namespace
+}  // namespace pa
+
+extern "C" {
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_heads,
+                    int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+                    int max_context_len, float scale, int partition_size, void* workspace,
+                    size_t workspace_bytes, pa_dtype dtype, void* stream)
+{
+    return decode_call("pa_decode", kDecodePlan | kDecodeRun, out, q, k_cache, v_cache, block_tables, context_lens,
+                       num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                       max_context_len, scale, partition_size, workspace, workspace_bytes, dtype, stream);
+}
+
+pa_status pa_decode_plan(const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_heads,
+                         int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+                         int max_context_len, int partition_size, void* workspace, size_t workspace_bytes,
+                         pa_dtype dtype, void* stream)
+{
+    return decode_call("pa_decode_plan", kDecodePlan, nullptr, nullptr, nullptr, nullptr, block_tables, context_lens,
+                       num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                       max_context_len, 1.0f, partition_size, workspace, workspace_bytes, dtype, stream);
+}
+
+pa_status pa_decode_run(void* out, const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int num_heads,
+                        int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+                        int max_context_len, float scale, int partition_size, void* workspace,
+                        size_t workspace_bytes, pa_dtype dtype, void* stream)
+{
+    return decode_call("pa_decode_run", kDecodeRun, out, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                       num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                       max_context_len, scale, partition_size, workspace, workspace_bytes, dtype, stream);
 }
 
 pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,

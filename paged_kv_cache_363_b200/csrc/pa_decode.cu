@@ -273,6 +273,14 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
                     info->flags = kEndUnit;
                     mbar_arrive(&utab[k % UR]);
                     mbar_arrive(&ufull[k % UR]);
+                    // This CTA takes no more units.  The last CTA to get here resets the
+                    // work counter, so the plan in the workspace serves the next run as it
+                    // is (one plan per decode step, one run per layer); it happens while the
+                    // CTAs still finish their last units, off the kernel's critical path.
+                    if (atomicAdd(a.plan + 4, 1u) == gridDim.x - 1) {
+                        a.plan[0] = 0u;
+                        a.plan[4] = 0u;
+                    }
                 }
                 ended = true;
                 break;
@@ -464,11 +472,13 @@ cudaError_t launch_persistent(const DecodeArgs& a, cudaStream_t stream)
     std::memset(&tk, 0, sizeof(tk));
     std::memset(&tv, 0, sizeof(tv));
     if constexpr (Cons::kTensorLoads) {
-        const uint64_t rows = (uint64_t)a.num_blocks * a.num_kv_heads * BS;
-        cudaError_t e = tensor_map(&tk, a.k_cache, rows, P::D, P::TR);
-        if (e != cudaSuccess) return e;
-        e = tensor_map(&tv, a.v_cache, rows, P::D, P::TR);
-        if (e != cudaSuccess) return e;
+        if (a.phases & kDecodeRun) {
+            const uint64_t rows = (uint64_t)a.num_blocks * a.num_kv_heads * BS;
+            cudaError_t e = tensor_map(&tk, a.k_cache, rows, P::D, P::TR);
+            if (e != cudaSuccess) return e;
+            e = tensor_map(&tv, a.v_cache, rows, P::D, P::TR);
+            if (e != cudaSuccess) return e;
+        }
     }
     int ctas = 0;
     cudaError_t e = resident_ctas<Cons, BS>(&ctas);
@@ -478,11 +488,14 @@ cudaError_t launch_persistent(const DecodeArgs& a, cudaStream_t stream)
     DecodeArgs args = a;
     args.num_ctas = (int)grid;
 
-    // one CTA; fewer threads for small batches keep its barriers short
-    const int plan_threads = a.num_seqs <= 256 ? 256 : (a.num_seqs <= 512 ? 512 : 1024);
-    decode_plan_kernel<<<1, plan_threads, 0, stream>>>(args, BS);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    if (a.phases & kDecodePlan) {
+        // one CTA; fewer threads for small batches keep its barriers short
+        const int plan_threads = a.num_seqs <= 256 ? 256 : (a.num_seqs <= 512 ? 512 : 1024);
+        decode_plan_kernel<<<1, plan_threads, 0, stream>>>(args, BS);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (!(a.phases & kDecodeRun)) return cudaSuccess;
     e = launch_pdl(decode_persistent_kernel<Cons, BS>, dim3(grid), dim3(P::THREADS), (size_t)P::SMEM, stream, args,
                    tk, tv);
     if (e != cudaSuccess || a.num_partitions <= 1) return e;

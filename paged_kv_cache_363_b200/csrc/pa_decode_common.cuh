@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeArgs a, i
         }
         if (lane == 0) {
             a.plan[0] = 0u;                 // work counter
+            a.plan[4] = 0u;                 // CTAs that finished a run (the last one resets both)
             a.plan[1] = (unsigned)running;  // number of (sequence, partition) pairs
             a.plan[3] = (unsigned)s_nsplit; // sequences that need the merge
         }

@@ -24,7 +24,8 @@ struct DecodeArgs {
     const int32_t* block_tables;
     const int32_t* context_lens;
     unsigned int* plan;        // [0] work counter, [1] (sequence, partition) pairs, [2] blocks per
-                               // partition, [3] sequences split into several partitions
+                               // partition, [3] sequences split into several partitions, [4] CTAs
+                               // that finished the current run
     uint2* plan_list;          // [S * NP] longest first: {sequence << 11 | partition, context length}
     unsigned int* split_list;  // [S] the sequences split into several partitions (plan[3] of them)
     float* ws_acc;             // [S][Hq][NP][D] unnormalised partition outputs (NP > 1)
@@ -41,12 +42,16 @@ struct DecodeArgs {
     int num_ctas;              // CTAs of the persistent kernel
     int num_partitions;        // NP = ceil(max_context_len / smallest partition tokens)
     float scale_log2;          // scale * log2(e): logits are kept in base-2 units
+    int phases;                // host side: kDecodePlan and/or kDecodeRun
 };
+
+constexpr int kDecodePlan = 1;  // the plan kernel: work list into the workspace
+constexpr int kDecodeRun = 2;   // the persistent kernel and the merge, from that work list
 
 // Byte layout of the decode workspace: the work plan, then (when a sequence may
 // span several partitions) the partition states.
 struct DecodeWorkspace {
-    size_t plan;       // 16 bytes: counter, pair count, blocks per partition, split count
+    size_t plan;       // 32 bytes: counter, pair count, blocks per partition, split count, exit count
     size_t list;       // 8 * S * NP bytes
     size_t splits;     // 4 * S bytes
     size_t acc;        // 4 * S * Hq * NP * D bytes (0 bytes when NP == 1)
@@ -60,7 +65,7 @@ inline DecodeWorkspace decode_workspace(size_t S, size_t Hq, size_t D, size_t NP
     const bool split = NP > 1;
     DecodeWorkspace w{};
     w.plan = 0;
-    w.list = 16;
+    w.list = 32;
     w.splits = up(w.list + 8 * S * NP);
     w.acc = up(w.splits + 4 * S);
     w.ml = up(w.acc + (split ? 4 * S * Hq * NP * D : 0));

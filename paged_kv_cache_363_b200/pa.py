@@ -37,6 +37,8 @@ SIGNATURES = [
     ("pa_decode_partition_size", _int, [_int] * 7),
     ("pa_decode_workspace_size", _sz, [_int] * 7),
     ("pa_decode", _int, [_vp, _vp, _vp, _vp, _vp, _vp] + [_int] * 8 + [_f32, _int, _vp, _sz, _int, _vp]),
+    ("pa_decode_plan", _int, [_vp, _vp] + [_int] * 9 + [_vp, _sz, _int, _vp]),
+    ("pa_decode_run", _int, [_vp, _vp, _vp, _vp, _vp, _vp] + [_int] * 8 + [_f32, _int, _vp, _sz, _int, _vp]),
     ("pa_decode_static_workspace", _int, [_vp, _vp, _vp, _vp, _vp, _vp] + [_int] * 8 + [_f32, _int, _int, _vp]),
     ("pa_reshape_and_cache", _int, [_vp, _vp, _vp, _vp, _vp] + [_int] * 6 + [_vp]),
     ("pa_prefill", _int, [_vp] * 7 + [_int] * 9 + [_f32, _int, _vp]),
@@ -171,6 +173,34 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
 
 
 PA_STATIC_WORKSPACE_BYTES = 16 * 1024 * 1024
+
+
+def pa_decode_plan(block_tables, context_lens, max_context_len, num_heads, k_cache, workspace, partition_size=0,
+                   dtype=None, stream=None):
+    """The work plan of a decode step into `workspace` (run it with pa_decode_run, once per layer).
+    k_cache gives the pool's shape and dtype (its data is not read)."""
+    NB, Hkv, B, D = k_cache.shape
+    S = context_lens.shape[0]
+    st = lib.pa_decode_plan(_dev_ptr(block_tables, "block_tables"), _dev_ptr(context_lens, "context_lens"), S,
+                            int(num_heads), Hkv, D, B, block_tables.shape[1], NB, int(max_context_len),
+                            int(partition_size), _dev_ptr(workspace, "workspace"),
+                            workspace.numel() * workspace.element_size(), _dtype_code(k_cache), _stream(stream))
+    _check(st, "pa_decode_plan")
+
+
+def pa_decode_run(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale, workspace,
+                  partition_size=0, stream=None):
+    """Decode attention from the plan pa_decode_plan left in `workspace`."""
+    S, Hq, D = q.shape
+    NB, Hkv, B, D2 = k_cache.shape
+    if D2 != D or tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("shape mismatch")
+    st = lib.pa_decode_run(_dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
+                           _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables"),
+                           _dev_ptr(context_lens, "context_lens"), S, Hq, Hkv, D, B, block_tables.shape[1], NB,
+                           int(max_context_len), float(scale), int(partition_size), _dev_ptr(workspace, "workspace"),
+                           workspace.numel() * workspace.element_size(), _dtype_code(q), _stream(stream))
+    _check(st, "pa_decode_run")
 
 
 def pa_decode_static_workspace(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,

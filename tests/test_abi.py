@@ -64,6 +64,31 @@ def test_host_validation_rejects_before_any_device_work():
     assert L.pa_copy_blocks(None, None, None, 0, 4, 128, 16, 8, 1, None) == pa.PA_OK
 
 
+def test_binding_argument_counts_match_the_header():
+    with open(os.path.join(ROOT, "include", "pa.h")) as f:
+        text = f.read()
+    decls = {m.group(1): m.group(2) for m in re.finditer(r"^PA_API [^(]*?\b(pa_\w+)\(([^)]*)\);", text, flags=re.M)}
+    for name, _, argtypes in pa.SIGNATURES:
+        params = decls[name].strip()
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        assert n == len(argtypes), "%s: header has %d parameters, binding %d" % (name, n, len(argtypes))
+
+
+def test_decode_plan_and_run_validate_on_the_host():
+    """Both halves of pa_decode reach their host-side checks (and the binding's argument
+    lists match the C signatures): bad sizes are refused before any device work."""
+    L = pa.lib
+    assert L.pa_decode_plan(None, None, 1, 4, 2, 128, 24, 4, 8, 64, 0, None, 0, pa.PA_DTYPE_BF16,
+                            None) == pa.PA_ERR_UNSUPPORTED                      # block size 24
+    assert L.pa_decode_plan(None, None, 1, 4, 3, 128, 16, 4, 8, 64, 0, None, 0, pa.PA_DTYPE_BF16,
+                            None) == pa.PA_ERR_INVALID                          # 4 heads over 3 kv heads
+    assert L.pa_decode_plan(None, None, 0, 4, 2, 128, 16, 4, 8, 64, 0, None, 0, pa.PA_DTYPE_BF16, None) == pa.PA_OK
+    assert L.pa_decode_run(None, None, None, None, None, None, 1, 4, 2, 96, 16, 4, 8, 64, 1.0, 0, None, 0,
+                           pa.PA_DTYPE_BF16, None) == pa.PA_ERR_UNSUPPORTED     # head_dim 96
+    assert L.pa_decode_run(None, None, None, None, None, None, 1, 4, 2, 128, 16, 4, 8, 64, float("nan"), 0, None,
+                           0, pa.PA_DTYPE_BF16, None) == pa.PA_ERR_INVALID      # non-finite scale
+
+
 def test_partition_and_workspace_sizes():
     assert pa.pa_decode_partition_size(8, 32, 8, 128, 32, 32768, 512) == 512
     assert pa.pa_decode_partition_size(8, 32, 8, 128, 32, 32768, 0) % 32 == 0
@@ -73,10 +98,10 @@ def test_partition_and_workspace_sizes():
         pa.pa_decode_partition_size(8, 32, 8, 128, 16, 10 ** 7, 16)      # too many partitions
     up = lambda x: (x + 255) // 256 * 256
     # one partition: only the work plan (16-byte header, one 8-byte entry and a split slot per sequence)
-    assert pa.pa_decode_workspace_size(4, 4, 4, 64, 16, 100, 512) == up(up(16 + 8 * 4) + 4 * 4)
+    assert pa.pa_decode_workspace_size(4, 4, 4, 64, 16, 100, 512) == up(up(32 + 8 * 4) + 4 * 4)
     # plan (S * NP entries, S split slots), then S * Hq * NP * D floats and S * Hq * NP (max, sum) pairs
     S, Hq, Hkv, D, NP = 8, 32, 8, 128, 64
-    acc = up(up(16 + 8 * S * NP) + 4 * S)
+    acc = up(up(32 + 8 * S * NP) + 4 * S)
     ml = up(acc + 4 * S * Hq * NP * D)
     assert pa.pa_decode_workspace_size(S, Hq, Hkv, D, 32, 32768, 512) == up(ml + 8 * S * Hq * NP)
     assert pa.pa_decode_workspace_size(0, 32, 8, 128, 32, 32768, 512) == 0

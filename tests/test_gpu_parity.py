@@ -370,3 +370,37 @@ def test_cow_small_pool_bit_exact(pa, runner):
     out = batch.step()
     assert max_abs(out.float().cpu().numpy(), ref) <= TOL["bf16"]
     _status_clean(pa)
+
+
+@pytest.mark.parametrize("wid,part", [(3, 0), (2, 256), (5, 512), (1, 0)])
+def test_plan_once_then_run_per_layer(pa, runner, wid, part):
+    """One plan per step, one run per layer: each run equals a whole pa_decode of the
+    same layer bit for bit (the runs reuse the plan; the last CTA of each resets its
+    work counter, or the next run would skip units)."""
+    over = {"num_seqs": 40, "num_blocks": 6000} if wid in (2, 3) else {}
+    wl = W.make_workload(wid, seed=2, **over)
+    wl.partition_size = part
+    batch = runner.DecodeBatch(wl, "cuda")
+    batch.append()
+    ws = torch.empty(pa.pa_decode_workspace_size(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim,
+                                                 wl.block_size, batch.max_context_len, part) + 16,
+                     dtype=torch.uint8, device="cuda")
+    pa.pa_decode_plan(batch.block_tables, batch.context_lens, batch.max_context_len, wl.num_heads, batch.k_cache, ws,
+                      part)
+    g = torch.Generator(device="cuda").manual_seed(wid)
+    for layer in range(4):
+        q = torch.randn(batch.q.shape, generator=g, device="cuda").to(batch.q.dtype)
+        kL = (batch.k_cache * (1.0 + 0.25 * layer)).contiguous()
+        vL = (batch.v_cache * (1.0 - 0.125 * layer)).contiguous()
+        got = torch.empty_like(q)
+        pa.pa_decode_run(got, q, kL, vL, batch.block_tables, batch.context_lens, batch.max_context_len, wl.scale, ws,
+                         part)
+        ref = torch.empty_like(q)
+        pa.pa_decode(ref, q, kL, vL, batch.block_tables, batch.context_lens, batch.max_context_len, wl.scale, part)
+        torch.cuda.synchronize()
+        assert torch.equal(bits_t(got), bits_t(ref)), "layer %d" % layer
+    _status_clean(pa)
+
+
+def bits_t(t):
+    return t.view(torch.int32) if t.dtype == torch.float32 else t.view(torch.int16)

@@ -198,7 +198,7 @@ pa_status decode_call(const char* fn, int phases, void* out, const void* q, cons
     unsigned char* ws = static_cast<unsigned char*>(workspace);
     a.plan = reinterpret_cast<unsigned int*>(ws + wl.plan);
     a.plan_list = reinterpret_cast<uint2*>(ws + wl.list);
-    a.split_list = reinterpret_cast<unsigned int*>(ws + wl.splits);
+    a.split_list = reinterpret_cast<uint2*>(ws + wl.splits);
     if (np > 1) {
         a.ws_acc = reinterpret_cast<float*>(ws + wl.acc);
         a.ws_ml = reinterpret_cast<float*>(ws + wl.ml);

@@ -25,8 +25,9 @@
 //  * At the end of a unit each warp leaves its softmax state in shared memory and goes
 //    on with the next unit; the warp that consumed the unit's last tile merges the four
 //    states.  A sequence longer than one partition leaves (max, sum, unnormalised
-//    output) per partition in the workspace and a log-sum-exp merge kernel combines them.  Plan, persistent and
-//    merge kernels are chained with programmatic dependent launch.
+//    output) per partition in the workspace and a log-sum-exp merge kernel combines
+//    them.  Plan, persistent and merge kernels are chained with programmatic dependent
+//    launch.
 //  * Logits are kept in base-2 units (q pre-scaled by scale*log2 e) and exponentials
 //    use exp2f, the reformulation of online softmax by Milakov & Gimelshein (2018).
 //  * Every wait is bounded: a wait that runs out raises PA_DEV_WAIT_TIMEOUT and the
@@ -248,15 +249,17 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
 
     if (warp == NCW + 1) {
         // ---------------- unit producer: takes units from the plan, fills the unit ring
-        unsigned npairs = 0;
-        if (lane == 0) npairs = *reinterpret_cast<volatile unsigned*>(a.plan + 1);
-        npairs = __shfl_sync(0xffffffffu, npairs, 0);
+        // The first unit's list entry is requested together with the pair count, not
+        // after it: its index is inside the list whatever the count (the grid has at
+        // most one CTA per unit the list can hold).
+        const unsigned npairs = __ldcg(a.plan + 1);
+        const uint2 e_first = __ldcg(a.plan_list + blockIdx.x / (unsigned)a.num_kv_heads);
         const unsigned nunits = npairs * (unsigned)a.num_kv_heads;
         int first = 0;
         int k = 0;
         bool ended = false;
         for (;; ++k) {
-            if (k >= UR && !mbar_wait_bounded(&uempty[k % UR], ((k / UR) & 1) ^ 1, abort_flag)) {
+            if (k >= UR && !mbar_wait_warp(&uempty[k % UR], ((k / UR) & 1) ^ 1, abort_flag)) {
                 if (lane == 0) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
                 *abort_flag = 1;
                 break;
@@ -285,7 +288,7 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
                 ended = true;
                 break;
             }
-            const uint2 e = a.plan_list[u / (unsigned)a.num_kv_heads];
+            const uint2 e = k == 0 ? e_first : a.plan_list[u / (unsigned)a.num_kv_heads];
             const int kvh = (int)(u % (unsigned)a.num_kv_heads);
             const int s = (int)(e.x >> 11);
             const int part = (int)(e.x & 2047u);

@@ -79,7 +79,8 @@ __device__ __forceinline__ int clamped_context(const DecodeArgs& a, int s, int b
 // With `adaptive` set the partition may grow (doubling from partition_blocks, up to
 // the longest context) while the largest unit stays within a quarter of one CTA's
 // share of all the work: fewer sequences are split, yet every CTA still gets
-// several units to balance with.  The choice is written to plan[2].
+// several units to balance with.  The choice is written to plan[2].  The split
+// sequences are listed with their context lengths for the merge kernel.
 __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeArgs a, int block_size)
 {
     __shared__ int bucket[kMaxPartitionTokens / 16 + 1];
@@ -138,7 +139,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeArgs a, i
         const int last = L > 0 ? (L - (np - 1) * P + block_size - 1) / block_size : 0;
         if (np > 1) {
             atomicAdd(&bucket[pb], np - 1);
-            a.split_list[atomicAdd(&s_nsplit, 1)] = (unsigned)s;
+            a.split_list[atomicAdd(&s_nsplit, 1)] = make_uint2((unsigned)s, (unsigned)L);
         }
         atomicAdd(&bucket[last], 1);
     }
@@ -251,77 +252,112 @@ __device__ __forceinline__ void finish_unit_warp(const DecodeArgs& a, const floa
     }
 }
 
-// Log-sum-exp merge of the partitions of the split sequences the plan listed, one
-// (sequence, query head) row per warp, warps striding over the rows:
-// M = max_p m_p, out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p.  A lane owns
-// D/32 consecutive columns (16-byte loads for D = 128); the weights of 32 partitions
-// are computed at once (one per lane) and broadcast, and the column loads of eight
-// partitions are in flight together.
+// Log-sum-exp merge of the partitions of the split sequences the plan listed:
+// M = max_p m_p, out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p, per
+// (sequence, query head) row.  `nwr` warps share a row (1, 2 or 4; a CTA of four
+// warps holds 4 / nwr rows at a time, CTAs striding over the rows).  A lane owns
+// D/32 consecutive columns.  The partitions go in chunks of 8, chunk c to warp
+// c % nwr of the row, whose eight column loads are all in flight together.  The
+// warps' sums are added in warp order, so a row's bits do not depend on the CTA that
+// merges it.
+//
+// The kernel is latency-bound, so its loads are arranged to wait on as little as
+// possible.  The plan lists each split sequence together with its context length,
+// and the first chunk's columns are requested together with the partition maxima.
+// A row then costs two dependent round trips to memory: the list entry, then the
+// partition states.
 template <typename T, int D>
-__global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeArgs a, int block_size)
+__global__ void __launch_bounds__(128, 8) decode_merge_kernel(const DecodeArgs a, int block_size, int nwr)
 {
     constexpr int EPL = D / 32;
-    constexpr int U = 8;
+    constexpr int CH = 8;
+    __shared__ __align__(16) float s_num[4][D];
+    __shared__ float s_den[4];
     pdl_wait_primary();
-    const int lane = threadIdx.x & 31;
-    const int P = (int)a.plan[2] * block_size;
-    const int rows = (int)a.plan[3] * a.num_heads;
-    const int nwarps = gridDim.x * (blockDim.x >> 5);
-    for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += nwarps) {
-        const int s = (int)a.split_list[r / a.num_heads];
-        const int row = s * a.num_heads + r % a.num_heads;
-        const int L = clamped_context(a, s, block_size, false);
-        const int np = (L + P - 1) / P;
-        const size_t row0 = (size_t)row * a.num_partitions;
-        const float2* ml = reinterpret_cast<const float2*>(a.ws_ml) + row0;
-
-        float M = -INFINITY;
-        for (int p = lane; p < np; p += 32) M = fmaxf(M, ml[p].x);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int rpc = 4 / nwr;  // rows per CTA at a time
+    const int slot = warp / nwr, sub = warp % nwr;
+    const int H = a.num_heads;
+    const unsigned* plan = a.plan;
+    const int P = (int)__ldg(plan + 2) * block_size;
+    const int rows = (int)__ldg(plan + 3) * H;
+    // the first row's list entry, requested with the counts above (the index stays
+    // inside the list, which has a slot per sequence, whatever the count turns out to be)
+    uint2 e = __ldg(a.split_list + min((int)blockIdx.x * rpc + slot, a.num_seqs * H - 1) / H);
+    for (int r0 = blockIdx.x * rpc; r0 < rows; r0 += gridDim.x * rpc) {
+        const int r = r0 + slot;
         float num[EPL];
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) num[e] = 0.f;
+        for (int k = 0; k < EPL; ++k) num[k] = 0.f;
         float den = 0.f;
-        const float* acc = a.ws_acc + row0 * D + lane * EPL;
-        for (int pc = 0; pc < np; pc += 32) {
-            float w = 0.f;
-            if (pc + lane < np) {
-                const float2 v = ml[pc + lane];
-                w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
-                den = fmaf(w, v.y, den);
-            }
-            const int cnt = min(32, np - pc);
-            for (int j = 0; j < cnt; j += U) {
-                float x[U][EPL];
+        if (r < rows) {
+            if (r0 != (int)blockIdx.x * rpc) e = __ldg(a.split_list + r / H);
+            const int L = (int)e.y;
+            const int np = (L + P - 1) / P;
+            const size_t row0 = ((size_t)e.x * H + r % H) * a.num_partitions;
+            const float2* ml = reinterpret_cast<const float2*>(a.ws_ml) + row0;
+            const float* acc = a.ws_acc + row0 * D + lane * EPL;
+            float x[CH][EPL];
+            auto load_chunk = [&](int c) {
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const float* src = acc + (size_t)(pc + min(j + u, cnt - 1)) * D;
+                for (int u = 0; u < CH; ++u) {
+                    // partitions past np repeat the last one; their weight is 0
+                    const float* src = acc + (size_t)min(c * CH + u, np - 1) * D;
                     if constexpr (EPL == 4) {
-                        const float4 v = *reinterpret_cast<const float4*>(src);
+                        const float4 v = __ldg(reinterpret_cast<const float4*>(src));
                         x[u][0] = v.x; x[u][1] = v.y; x[u][2] = v.z; x[u][3] = v.w;
                     } else {
-                        const float2 v = *reinterpret_cast<const float2*>(src);
+                        const float2 v = __ldg(reinterpret_cast<const float2*>(src));
                         x[u][0] = v.x; x[u][1] = v.y;
                     }
                 }
+            };
+            int c = sub;
+            if (c * CH < np) load_chunk(c);
+            float M = -INFINITY;
+            for (int p = lane; p < np; p += 32) M = fmaxf(M, __ldg(&ml[p].x));
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    // lanes past the partition count hold weight 0, so the clamped
-                    // (repeated) loads above add nothing
-                    const float wj = __shfl_sync(0xffffffffu, w, min(j + u, 31));
-                    const float wu = j + u < cnt ? wj : 0.f;
+            for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+            for (; c * CH < np; c += nwr) {
+                if (c != sub) load_chunk(c);
+                // lane u < 8 holds the weight of partition c * 8 + u
+                const int pw = c * CH + (lane & (CH - 1));
+                float w = 0.f;
+                if (lane < CH && pw < np) {
+                    const float2 v = __ldg(ml + pw);
+                    w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
+                    den = fmaf(w, v.y, den);
+                }
 #pragma unroll
-                    for (int e = 0; e < EPL; ++e) num[e] = fmaf(wu, x[u][e], num[e]);
+                for (int u = 0; u < CH; ++u) {
+                    const float wu = __shfl_sync(0xffffffffu, w, u);
+#pragma unroll
+                    for (int k = 0; k < EPL; ++k) num[k] = fmaf(wu, x[u][k], num[k]);
                 }
             }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
         }
+        if (nwr > 1) {
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-        const float inv = den > 0.f ? 1.f / den : 0.f;
-        T* o = static_cast<T*>(a.out) + (size_t)row * D + lane * EPL;
+            for (int k = 0; k < EPL; ++k) s_num[warp][lane * EPL + k] = num[k];
+            if (lane == 0) s_den[warp] = den;
+            __syncthreads();
+            if (sub == 0) {
+                for (int j = 1; j < nwr; ++j) {
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) o[e] = from_f32<T>(num[e] * inv);
+                    for (int k = 0; k < EPL; ++k) num[k] += s_num[warp + j][lane * EPL + k];
+                    den += s_den[warp + j];
+                }
+            }
+            __syncthreads();
+        }
+        if (r < rows && sub == 0) {
+            const float inv = den > 0.f ? 1.f / den : 0.f;
+            T* o = static_cast<T*>(a.out) + ((size_t)e.x * H + r % H) * D + lane * EPL;
+#pragma unroll
+            for (int k = 0; k < EPL; ++k) o[k] = from_f32<T>(num[k] * inv);
+        }
     }
 }
 
@@ -348,12 +384,15 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 template <typename T, int D>
 cudaError_t launch_merge(const DecodeArgs& a, int block_size, cudaStream_t stream)
 {
-    // up to eight CTAs (32 warps) per SM; the warps loop over the rows of the split sequences
+    // one warp per row while a row has at most one chunk of 8 partitions, two for two
+    // chunks, else four; up to eight CTAs per SM, striding over the rows of the split sequences
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const long ctas = ((long)a.num_seqs * a.num_heads + 3) / 4;
+    const int nwr = a.num_partitions <= 8 ? 1 : (a.num_partitions <= 16 ? 2 : 4);
+    const long rpc = 4 / nwr;
+    const long ctas = ((long)a.num_seqs * a.num_heads + rpc - 1) / rpc;
     const unsigned grid = (unsigned)(ctas < 8L * sms ? ctas : 8L * sms);
-    return launch_pdl(decode_merge_kernel<T, D>, dim3(grid), dim3(128), 0, stream, a, block_size);
+    return launch_pdl(decode_merge_kernel<T, D>, dim3(grid), dim3(128), 0, stream, a, block_size, nwr);
 }
 
 }  // namespace

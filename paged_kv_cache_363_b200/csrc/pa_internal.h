@@ -27,7 +27,8 @@ struct DecodeArgs {
                                // partition, [3] sequences split into several partitions, [4] CTAs
                                // that finished the current run
     uint2* plan_list;          // [S * NP] longest first: {sequence << 11 | partition, context length}
-    unsigned int* split_list;  // [S] the sequences split into several partitions (plan[3] of them)
+    uint2* split_list;         // [S] the sequences split into several partitions (plan[3] of them):
+                               // {sequence, context length}
     float* ws_acc;             // [S][Hq][NP][D] unnormalised partition outputs (NP > 1)
     float* ws_ml;              // [S][Hq][NP][2] (running max in log2 units, softmax sum)
     unsigned int* status;      // device status word (PA_DEV_* bits)
@@ -53,7 +54,7 @@ constexpr int kDecodeRun = 2;   // the persistent kernel and the merge, from tha
 struct DecodeWorkspace {
     size_t plan;       // 32 bytes: counter, pair count, blocks per partition, split count, exit count
     size_t list;       // 8 * S * NP bytes
-    size_t splits;     // 4 * S bytes
+    size_t splits;     // 8 * S bytes
     size_t acc;        // 4 * S * Hq * NP * D bytes (0 bytes when NP == 1)
     size_t ml;         // 8 * S * Hq * NP bytes (0 bytes when NP == 1)
     size_t total;
@@ -67,7 +68,7 @@ inline DecodeWorkspace decode_workspace(size_t S, size_t Hq, size_t D, size_t NP
     w.plan = 0;
     w.list = 32;
     w.splits = up(w.list + 8 * S * NP);
-    w.acc = up(w.splits + 4 * S);
+    w.acc = up(w.splits + 8 * S);
     w.ml = up(w.acc + (split ? 4 * S * Hq * NP * D : 0));
     w.total = up(w.ml + (split ? 8 * S * Hq * NP : 0));
     return w;

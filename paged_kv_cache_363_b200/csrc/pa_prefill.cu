@@ -81,15 +81,6 @@ __device__ __forceinline__ float fast_exp2(float x)
     return y;
 }
 
-// A bounded mbarrier wait taken by every lane of a warp, with one answer for the
-// whole warp: the tcgen05.ld / tcgen05.st that follow are .sync.aligned and must be
-// reached by all lanes together or by none.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
-{
-    const bool ok = mbar_wait_bounded(bar, parity, abort_flag);
-    return __all_sync(0xffffffffu, ok) != 0;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -301,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < ntiles; ++j) {
-            if (!warp_wait(s_full, j & 1, abort_flag)) {
+            if (!mbar_wait_warp(s_full, j & 1, abort_flag)) {
                 ok = false;
                 break;
             }
@@ -370,11 +361,11 @@ __global__ void __launch_bounds__(kThreads, 2)
             // P buffer j & 1 is free once the P.V of tile j - 2 has finished; O is stable
             // for a rescale once the P.V of tile j - 1 has (each buffer has its own
             // barrier, whose next phase is never more than one ahead of the wait)
-            if (j >= 2 && !warp_wait(&o_done[j & 1], ((j - 2) >> 1) & 1, abort_flag)) {
+            if (j >= 2 && !mbar_wait_warp(&o_done[j & 1], ((j - 2) >> 1) & 1, abort_flag)) {
                 ok = false;
                 break;
             }
-            if (rescale_warp && j >= 1 && !warp_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)) {
+            if (rescale_warp && j >= 1 && !mbar_wait_warp(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)) {
                 ok = false;
                 break;
             }
@@ -441,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             // keys past the context in this tile: zero their V rows (0-weights must meet finite values)
             if (kv0 + kN > L) {
                 // the tile's V copies (boxes with tokens past the context included) have landed
-                if (!warp_wait(&v_full[j % VST], (j / VST) & 1, abort_flag)) {
+                if (!mbar_wait_warp(&v_full[j % VST], (j / VST) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -459,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full);
         }
-        if (ok && warp_wait(&o_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort_flag)) {
+        if (ok && mbar_wait_warp(&o_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort_flag)) {
             tc_fence_after_sync();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) +

@@ -73,6 +73,16 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// The same wait taken by every lane of a warp, with one answer for the whole warp.
+// Lanes could otherwise see the time limit or the abort flag at different moments and
+// leave a later warp-wide shuffle, or a .sync.aligned instruction (tcgen05.ld/st), short
+// of a lane.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort)
+{
+    const bool ok = mbar_wait_bounded(bar, parity, abort);
+    return __all_sync(0xffffffffu, ok) != 0;
+}
+
 // 1-D bulk copy global -> shared, completion signalled on `bar` as tx bytes.
 // dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar)

@@ -74,6 +74,17 @@ def test_binding_argument_counts_match_the_header():
         assert n == len(argtypes), "%s: header has %d parameters, binding %d" % (name, n, len(argtypes))
 
 
+def test_binding_constants_match_the_header():
+    with open(os.path.join(ROOT, "include", "pa.h")) as f:
+        text = f.read()
+    defines = dict(re.findall(r"^#define (PA_\w+) \(?([0-9u *]+)\)?", text, flags=re.M))
+    for name in ("PA_STATIC_WORKSPACE_BYTES",):
+        value = 1
+        for factor in defines[name].replace("u", "").split("*"):
+            value *= int(factor)
+        assert value == getattr(pa, name), name
+
+
 def test_decode_plan_and_run_validate_on_the_host():
     """Both halves of pa_decode reach their host-side checks (and the binding's argument
     lists match the C signatures): bad sizes are refused before any device work."""
@@ -97,11 +108,11 @@ def test_partition_and_workspace_sizes():
     with pytest.raises(pa.PAError):
         pa.pa_decode_partition_size(8, 32, 8, 128, 16, 10 ** 7, 16)      # too many partitions
     up = lambda x: (x + 255) // 256 * 256
-    # one partition: only the work plan (16-byte header, one 8-byte entry and a split slot per sequence)
-    assert pa.pa_decode_workspace_size(4, 4, 4, 64, 16, 100, 512) == up(up(32 + 8 * 4) + 4 * 4)
+    # one partition: only the work plan (32-byte header, one 8-byte entry and an 8-byte split slot per sequence)
+    assert pa.pa_decode_workspace_size(4, 4, 4, 64, 16, 100, 512) == up(up(32 + 8 * 4) + 8 * 4)
     # plan (S * NP entries, S split slots), then S * Hq * NP * D floats and S * Hq * NP (max, sum) pairs
     S, Hq, Hkv, D, NP = 8, 32, 8, 128, 64
-    acc = up(up(32 + 8 * S * NP) + 4 * S)
+    acc = up(up(32 + 8 * S * NP) + 8 * S)
     ml = up(acc + 4 * S * Hq * NP * D)
     assert pa.pa_decode_workspace_size(S, Hq, Hkv, D, 32, 32768, 512) == up(ml + 8 * S * Hq * NP)
     assert pa.pa_decode_workspace_size(0, 32, 8, 128, 32, 32768, 512) == 0

@@ -33,6 +33,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
@@ -513,15 +514,17 @@ cudaError_t launch_g(const PrefillArgs& a, int num_query_tokens, int max_query_l
     const uint64_t rows = (uint64_t)a.num_blocks * a.num_kv_heads * a.block_size;
     if ((e = tensor_map(&tk, a.k_cache, rows, kD, kBox)) != cudaSuccess) return e;
     if ((e = tensor_map(&tv, a.v_cache, rows, kD, kBox)) != cudaSuccess) return e;
-    static bool attr_done[64] = {};
+    // the kernel's attributes, set once per device (setting them twice is harmless, so
+    // two threads racing to the first call need no lock)
+    static std::atomic<bool> attr_done[64] = {};
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (!attr_done[dev & 63]) {
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if (!attr_done[dev & 63].load()) {
         e = cudaFuncSetAttribute(prefill_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(prefill_tc_kernel<G>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (e != cudaSuccess) return e;
-        attr_done[dev & 63] = true;
+        attr_done[dev & 63].store(true);
     }
     constexpr int T = kM / G;
     const dim3 grid((unsigned)((max_query_len + T - 1) / T), (unsigned)a.num_kv_heads, (unsigned)a.num_seqs);

@@ -24,7 +24,7 @@
 //     only when the max grows by more than 8 (2^8: exact up to rounding, fewer
 //     rescales), write P as bf16 into tensor memory (two buffers, so the next tile's
 //     P is written while this tile's P.V runs), and at the end normalise O and store it.
-// Two CTAs share an SM (97 KB of shared memory and 256 tensor-memory columns each),
+// Two CTAs share an SM (113 KB of shared memory and 256 tensor-memory columns each),
 // so one CTA's softmax overlaps the other's matrix multiplies.
 // Every wait is bounded; on expiry the CTA raises PA_DEV_WAIT_TIMEOUT, drains its own
 // copies and MMAs, frees its tensor memory and returns.

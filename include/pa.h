@@ -207,6 +207,23 @@ PA_API pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* blo
                          int num_kv_heads, int head_dim, int block_size, int num_blocks, pa_dtype dtype,
                          void* stream);
 
+/*
+ * Optional host-side checks of the two mappings whose misuse the kernels cannot make
+ * safe: pairs and slots are handled concurrently, so a repeated destination (or a
+ * destination that is also a source) leaves a result that depends on thread order.
+ * Both take HOST arrays, touch no device, change nothing and return PA_OK or
+ * PA_ERR_INVALID (the first offending index in pa_last_error_string()).
+ *   pa_check_block_mapping: block_mapping [num_pairs][2] int64 (src, dst) as for
+ *     pa_copy_blocks; invalid if an entry is outside [0, num_blocks), a destination
+ *     appears twice, or a destination is also a source.
+ *   pa_check_slot_mapping: slot_mapping [num_tokens] int64 as for
+ *     pa_reshape_and_cache; invalid if a slot >= 0 appears twice or is past the pool
+ *     (num_blocks * block_size); negative slots (padding) are ignored.
+ * A null array with a count of 0 is valid.
+ */
+PA_API pa_status pa_check_block_mapping(const int64_t* block_mapping, int num_pairs, int num_blocks);
+PA_API pa_status pa_check_slot_mapping(const int64_t* slot_mapping, int num_tokens, int num_blocks, int block_size);
+
 /* ------------------------------------------------------------------ device status */
 
 /*

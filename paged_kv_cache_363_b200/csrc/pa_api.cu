@@ -2,12 +2,15 @@
 // the kernels, the device status word, and the per-thread error message.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <mutex>
 #include <string>
+#include <utility>
+#include <vector>
 
 #include "pa.h"
 #include "pa_internal.h"
@@ -294,6 +297,73 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache
     const cudaError_t e =
         launch_reshape_and_cache(a, elt_bytes(dtype), head_dim, block_size, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail("pa_reshape_and_cache launch", e);
+    return PA_OK;
+}
+
+pa_status pa_check_block_mapping(const int64_t* block_mapping, int num_pairs, int num_blocks)
+{
+    if (num_pairs < 0 || num_blocks <= 0 || (num_pairs > 0 && !block_mapping)) {
+        set_error("pa_check_block_mapping: bad count or null array");
+        return PA_ERR_INVALID;
+    }
+    // (block, pair index) of every destination, then of every source, sorted by block
+    std::vector<std::pair<int64_t, int>> dst, src;
+    dst.reserve(num_pairs);
+    src.reserve(num_pairs);
+    for (int i = 0; i < num_pairs; ++i) {
+        const int64_t s = block_mapping[2 * i], d = block_mapping[2 * i + 1];
+        if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks) {
+            set_error("pa_check_block_mapping: pair " + std::to_string(i) + " names a block outside [0, num_blocks)");
+            return PA_ERR_INVALID;
+        }
+        dst.emplace_back(d, i);
+        src.emplace_back(s, i);
+    }
+    std::sort(dst.begin(), dst.end());
+    std::sort(src.begin(), src.end());
+    for (size_t k = 1; k < dst.size(); ++k)
+        if (dst[k].first == dst[k - 1].first) {
+            set_error("pa_check_block_mapping: pairs " + std::to_string(dst[k - 1].second) + " and " +
+                      std::to_string(dst[k].second) + " write the same block " + std::to_string(dst[k].first));
+            return PA_ERR_INVALID;
+        }
+    for (size_t k = 0, m = 0; k < dst.size(); ++k) {
+        while (m < src.size() && src[m].first < dst[k].first) ++m;
+        if (m < src.size() && src[m].first == dst[k].first) {
+            set_error("pa_check_block_mapping: block " + std::to_string(dst[k].first) + " is written by pair " +
+                      std::to_string(dst[k].second) + " and read by pair " + std::to_string(src[m].second));
+            return PA_ERR_INVALID;
+        }
+    }
+    return PA_OK;
+}
+
+pa_status pa_check_slot_mapping(const int64_t* slot_mapping, int num_tokens, int num_blocks, int block_size)
+{
+    if (num_tokens < 0 || num_blocks <= 0 || block_size <= 0 || (num_tokens > 0 && !slot_mapping)) {
+        set_error("pa_check_slot_mapping: bad count or size, or null array");
+        return PA_ERR_INVALID;
+    }
+    const int64_t nslots = (int64_t)num_blocks * block_size;
+    std::vector<std::pair<int64_t, int>> slots;
+    slots.reserve(num_tokens);
+    for (int t = 0; t < num_tokens; ++t) {
+        const int64_t s = slot_mapping[t];
+        if (s < 0) continue;  // padding
+        if (s >= nslots) {
+            set_error("pa_check_slot_mapping: token " + std::to_string(t) + " has slot " + std::to_string(s) +
+                      ", past the pool's " + std::to_string(nslots) + " slots");
+            return PA_ERR_INVALID;
+        }
+        slots.emplace_back(s, t);
+    }
+    std::sort(slots.begin(), slots.end());
+    for (size_t k = 1; k < slots.size(); ++k)
+        if (slots[k].first == slots[k - 1].first) {
+            set_error("pa_check_slot_mapping: tokens " + std::to_string(slots[k - 1].second) + " and " +
+                      std::to_string(slots[k].second) + " share slot " + std::to_string(slots[k].first));
+            return PA_ERR_INVALID;
+        }
     return PA_OK;
 }
 

@@ -43,6 +43,8 @@ SIGNATURES = [
     ("pa_reshape_and_cache", _int, [_vp, _vp, _vp, _vp, _vp] + [_int] * 6 + [_vp]),
     ("pa_prefill", _int, [_vp] * 7 + [_int] * 9 + [_f32, _int, _vp]),
     ("pa_copy_blocks", _int, [_vp, _vp, _vp] + [_int] * 6 + [_vp]),
+    ("pa_check_block_mapping", _int, [_vp, _int, _int]),
+    ("pa_check_slot_mapping", _int, [_vp, _int, _int, _int]),
     ("pa_swap_blocks", _int, [_vp, _vp, _vp, _vp, _vp] + [_int] * 7 + [_vp]),
     ("pa_device_status", _int, [ctypes.POINTER(_u32), _vp]),
     ("pa_selftest_bounded_wait", _int, [ctypes.POINTER(ctypes.c_uint64), _vp]),
@@ -224,8 +226,35 @@ def pa_decode_static_workspace(out, q, k_cache, v_cache, block_tables, context_l
     return out
 
 
-def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None):
-    """k/v_cache[slot // B, :, slot % B, :] <- key/value[t] for every slot >= 0."""
+def _host_int64(a):
+    """A C-contiguous int64 numpy copy of a host or device array (for the host-side checks)."""
+    import numpy as np
+    if hasattr(a, "detach"):
+        a = a.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(a), dtype=np.int64)
+
+
+def pa_check_block_mapping(block_mapping, num_blocks):
+    """Host-side check of copy pairs [n, 2] (any array; copied to host): raises PAError if an
+    entry is out of range, a destination repeats, or a destination is also a source."""
+    m = _host_int64(block_mapping).reshape(-1)
+    if m.size % 2:
+        raise ValueError("block_mapping must be [n, 2]")
+    n = m.size // 2
+    _check(lib.pa_check_block_mapping(m.ctypes.data if n else None, n, int(num_blocks)), "pa_check_block_mapping")
+
+
+def pa_check_slot_mapping(slot_mapping, num_blocks, block_size):
+    """Host-side check of append slots (any array; copied to host): raises PAError if a slot
+    >= 0 repeats or lies past the pool."""
+    m = _host_int64(slot_mapping).reshape(-1)
+    _check(lib.pa_check_slot_mapping(m.ctypes.data if m.size else None, m.size, int(num_blocks), int(block_size)),
+           "pa_check_slot_mapping")
+
+
+def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None, check=False):
+    """k/v_cache[slot // B, :, slot % B, :] <- key/value[t] for every slot >= 0.  With check=True
+    the slots are first copied to the host and checked (pa_check_slot_mapping; synchronising)."""
     N, Hkv, D = key.shape
     NB, Hkv2, B, D2 = k_cache.shape
     if (Hkv2, D2) != (Hkv, D) or tuple(value.shape) != tuple(key.shape) or tuple(slot_mapping.shape) != (N,):
@@ -233,6 +262,8 @@ def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None
     import torch
     if slot_mapping.dtype != torch.int64:
         raise TypeError("slot_mapping must be int64")
+    if check:
+        pa_check_slot_mapping(slot_mapping, NB, B)
     dt = _dtype_code(key)
     st = lib.pa_reshape_and_cache(_dev_ptr(key, "key"), _dev_ptr(value, "value"), _dev_ptr(k_cache, "k_cache"),
                                   _dev_ptr(v_cache, "v_cache"), _dev_ptr(slot_mapping, "slot_mapping"), N, Hkv, D,
@@ -281,13 +312,17 @@ def pa_swap_blocks(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache, block_map
     _check(st, "pa_swap_blocks")
 
 
-def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None):
-    """For every (src, dst) row of block_mapping[n, 2] (int64): block dst <- block src, both pools."""
+def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None, check=False):
+    """For every (src, dst) row of block_mapping[n, 2] (int64): block dst <- block src, both pools.
+    With check=True the pairs are first copied to the host and checked (pa_check_block_mapping;
+    synchronising)."""
     NB, Hkv, B, D = k_cache.shape
     import torch
     if block_mapping.dtype != torch.int64 or (block_mapping.numel() and block_mapping.shape[-1] != 2):
         raise TypeError("block_mapping must be int64 [n, 2]")
     n = block_mapping.numel() // 2
+    if check:
+        pa_check_block_mapping(block_mapping, NB)
     ptr = _dev_ptr(block_mapping, "block_mapping") if n else None
     st = lib.pa_copy_blocks(_dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"), ptr, n, Hkv, D, B, NB,
                             _dtype_code(k_cache), _stream(stream))

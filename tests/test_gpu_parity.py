@@ -227,6 +227,29 @@ def test_copy_blocks_bit_exact(pa, dtype, D, B, Hkv):
     _status_clean(pa)
 
 
+def test_checked_copy_and_append_refuse_racing_mappings_before_any_write(pa):
+    """check=True runs the host-side checks first: a racing mapping is refused and the
+    pools stay as they were; a sound one goes through bit-exact."""
+    NB, Hkv, B, D = 16, 2, 16, 64
+    pool_k = torch.randn(NB, Hkv, B, D, generator=torch.Generator().manual_seed(3))
+    pool_v = torch.randn(NB, Hkv, B, D, generator=torch.Generator().manual_seed(4))
+    kc, vc = pool_k.clone().cuda(), pool_v.clone().cuda()
+    for bad in ([[0, 3], [1, 3]], [[0, 3], [3, 5]]):
+        with pytest.raises(pa.PAError):
+            pa.pa_copy_blocks(kc, vc, torch.tensor(bad, dtype=torch.int64, device="cuda"), check=True)
+    key = torch.ones(3, Hkv, D, device="cuda")
+    with pytest.raises(pa.PAError):
+        pa.pa_reshape_and_cache(key, key, kc, vc, torch.tensor([5, 40, 5], dtype=torch.int64, device="cuda"),
+                                check=True)
+    torch.cuda.synchronize()
+    assert torch.equal(kc.cpu(), pool_k) and torch.equal(vc.cpu(), pool_v)
+    good = np.array([[0, 3], [0, 4], [1, 5]], np.int64)
+    pa.pa_copy_blocks(kc, vc, torch.from_numpy(good).cuda(), check=True)
+    rk, rv = oracle.copy_blocks(bits(pool_k), bits(pool_v), good)
+    assert np.array_equal(bits(kc), rk) and np.array_equal(bits(vc), rv)
+    _status_clean(pa)
+
+
 # ------------------------------------------------------------------ device-side checks
 
 def test_device_checks_flag_bad_inputs_without_touching_memory(pa):

@@ -107,3 +107,62 @@ def test_planted_mistakes_fail_a_pin(mut):
         assert passed
     else:
         assert not passed
+
+
+# ---------------------------------------------------------------- split-K merge
+
+MERGE_MUTATIONS = ["none", "den_without_l", "num_unweighted", "last_partition_dropped",
+                   "partition_end_off_by_one"]
+
+
+def _split_merge(q_row, k, v, table, kvh, cuts, scale, mut):
+    """Partition states (m, l, acc) over [t0, t1) and their log-sum-exp merge, restated
+    with a switch for one planted mistake."""
+    B = k.shape[2]
+    states = []
+    for t0, t1 in zip(cuts[:-1], cuts[1:]):
+        t1 = max(t0, t1 - 1) if mut == "partition_end_off_by_one" else t1
+        z = [scale * float(np.dot(q_row.astype(np.float64), k[table[i // B], kvh, i % B].astype(np.float64)))
+             for i in range(t0, t1)]
+        if not z:
+            states.append((-math.inf, 0.0, np.zeros(k.shape[3])))
+            continue
+        m = max(z)
+        e = [math.exp(x - m) for x in z]
+        acc = sum(w * v[table[i // B], kvh, i % B].astype(np.float64) for w, i in zip(e, range(t0, t1)))
+        states.append((m, sum(e), acc))
+    if mut == "last_partition_dropped":
+        states = states[:-1]
+    M = max(m for m, _, _ in states)
+    num, den = 0.0, 0.0
+    for m, l, acc in states:
+        w = 0.0 if m == -math.inf else math.exp(m - M)
+        num = num + (acc if mut == "num_unweighted" else w * acc)
+        den += w if mut == "den_without_l" else w * l
+    return num / den
+
+
+def _merge_passes_pin(mut):
+    """The split-K pin: for several partitionings (empty ranges included) the merge of the
+    partition states equals the one-pass oracle row."""
+    from oracle import oracle
+    rng = np.random.default_rng(11)
+    B, D, L = 4, 8, 23
+    tables = np.array([[2, 0, 5, 1, 3, 4]], np.int32)
+    q = rng.standard_normal((1, 2, D)).astype(np.float32)
+    k = rng.standard_normal((6, 1, B, D)).astype(np.float32)
+    v = rng.standard_normal((6, 1, B, D)).astype(np.float32)
+    ref = oracle.decode(q, k, v, tables, np.array([L], np.int32), 0.7)[0, 1]
+    for cuts in ([0, L], [0, 8, 16, L], [0, 4, 4, 12, L], [0, 1, L, L]):
+        try:
+            got = _split_merge(q[0, 1], k, v, tables[0], 0, cuts, 0.7, mut)
+        except (ValueError, ZeroDivisionError):
+            return False          # a mistake that cannot even produce a row fails too
+        if not np.allclose(got, ref, rtol=0, atol=1e-12):
+            return False
+    return True
+
+
+@pytest.mark.parametrize("mut", MERGE_MUTATIONS)
+def test_planted_merge_mistakes_fail_the_split_pin(mut):
+    assert _merge_passes_pin(mut) == (mut == "none")

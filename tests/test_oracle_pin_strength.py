@@ -166,3 +166,80 @@ def _merge_passes_pin(mut):
 @pytest.mark.parametrize("mut", MERGE_MUTATIONS)
 def test_planted_merge_mistakes_fail_the_split_pin(mut):
     assert _merge_passes_pin(mut) == (mut == "none")
+
+
+# ---------------------------------------------------------------- append and copy-on-write copy
+
+RESHAPE_MUTATIONS = ["none", "block_offset_swapped", "value_not_written", "negative_slot_written"]
+COPY_MUTATIONS = ["none", "key_pool_only", "first_slot_only", "first_head_only", "pair_reversed"]
+
+
+def _reshape(key, value, kc, vc, slots, mut):
+    kc, vc = kc.copy(), vc.copy()
+    B = kc.shape[2]
+    for t, s in enumerate(slots):
+        if s < 0 and mut != "negative_slot_written":
+            continue
+        s = int(s) % (kc.shape[0] * B)
+        b, o = (s % B, s // B) if mut == "block_offset_swapped" else (s // B, s % B)
+        kc[b, :, o] = key[t]
+        if mut != "value_not_written":
+            vc[b, :, o] = value[t]
+    return kc, vc
+
+
+def _copy(kc, vc, pairs, mut):
+    kc, vc = kc.copy(), vc.copy()
+    for src, dst in pairs:
+        if mut == "pair_reversed":
+            src, dst = dst, src
+        sl = (slice(None), slice(0, 1)) if mut == "first_slot_only" else (slice(0, 1),) if mut == "first_head_only" \
+            else (slice(None),)
+        kc[(dst,) + sl] = kc[(src,) + sl]
+        if mut != "key_pool_only":
+            vc[(dst,) + sl] = vc[(src,) + sl]
+    return kc, vc
+
+
+def _reshape_passes_pins(mut):
+    from conftest import read_golden
+    from oracle import oracle
+    hdr, rows = read_golden("translation_fullstackaihub.txt")
+    B, table = hdr["block_size"], hdr["table"]
+    rng = np.random.default_rng(1)
+    key = rng.standard_normal((32, 2, 8)).astype(np.float32)
+    val = rng.standard_normal((32, 2, 8)).astype(np.float32)
+    kc = np.zeros((20, 2, B, 8), np.float32)
+    slots = np.array([oracle.physical_slot(table, B, i) for i in range(32)], np.int64)
+    slots[5] = -1                                     # a padding token
+    try:
+        k2, v2 = _reshape(key, val, kc, kc, slots, mut)
+    except IndexError:
+        return False                                  # a mistake that writes outside the pool fails too
+    for tok, blk, off, _ in rows:
+        if tok != 5 and not (np.array_equal(k2[blk, :, off], key[tok]) and np.array_equal(v2[blk, :, off], val[tok])):
+            return False
+    untouched = [b for b in range(20) if b not in table]
+    written = {(table[i // B], i % B) for i in range(32) if i != 5}
+    stray = [(b, o) for b in table for o in range(B) if (b, o) not in written and np.any(k2[b, :, o] != 0)]
+    return bool(np.all(k2[untouched] == 0) and np.all(v2[untouched] == 0)) and not stray
+
+
+def _copy_passes_pins(mut):
+    rng = np.random.default_rng(3)
+    kc = rng.standard_normal((6, 2, 16, 4)).astype(np.float32)
+    vc = rng.standard_normal((6, 2, 16, 4)).astype(np.float32)
+    k2, v2 = _copy(kc, vc, [(0, 3), (1, 5)], mut)
+    if not all(np.array_equal(k2[d], kc[s]) and np.array_equal(v2[d], vc[s]) for s, d in ((0, 3), (1, 5))):
+        return False
+    return all(np.array_equal(k2[b], kc[b]) and np.array_equal(v2[b], vc[b]) for b in (0, 1, 2, 4))
+
+
+@pytest.mark.parametrize("mut", RESHAPE_MUTATIONS)
+def test_planted_append_mistakes_fail_a_pin(mut):
+    assert _reshape_passes_pins(mut) == (mut == "none")
+
+
+@pytest.mark.parametrize("mut", COPY_MUTATIONS)
+def test_planted_copy_mistakes_fail_a_pin(mut):
+    assert _copy_passes_pins(mut) == (mut == "none")

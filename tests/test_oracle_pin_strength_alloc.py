@@ -1,4 +1,4 @@
-"""The prefix-cache and beam-search pins are strong enough: plausible mistakes
+"""The prefix-cache, beam-search and swap pins are strong enough: plausible mistakes
 planted in a subclass of the oracle allocator each fail at least one pin (CPU only).  The unmutated class
 passes them all.  Nothing here changes the real oracle or touches the library."""
 import pytest
@@ -98,8 +98,57 @@ class _ForkWithoutReference(OracleAllocator):
         self.ntokens[child] = self.ntokens[parent]
 
 
+class _SwapOutKeepsReference(OracleAllocator):
+    """Swap-out that gives the sequence host blocks but keeps its device blocks referenced."""
+    def swap_out(self, seq_id):
+        table = list(self.tables[seq_id])
+        self.ref_backup = {b: self.ref[b] for b in table}
+        pairs = super().swap_out(seq_id)
+        for b, r in self.ref_backup.items():
+            if self.ref[b] < r:
+                if b in self.free:
+                    self.free.remove(b)
+                self.ref[b] = r
+        return pairs
+
+
+class _SwapInReversed(OracleAllocator):
+    """Swap-in that hands back the host blocks in reverse table order."""
+    def swap_in(self, seq_id):
+        if seq_id in self.on_host:
+            self.tables[seq_id] = self.tables[seq_id][::-1]
+        pairs = super().swap_in(seq_id)
+        return pairs
+
+
+class _PartialSwapOut(OracleAllocator):
+    """Swap-out that moves what fits on the host instead of refusing when the host is short."""
+    def swap_out(self, seq_id):
+        if seq_id not in self.tables or seq_id in self.on_host:
+            raise ValueError("unknown or swapped-out sequence")
+        table = self.tables[seq_id]
+        pairs = []
+        for i, blk in enumerate(table):
+            if not self.host_free:
+                break
+            h = self.host_free.popleft()
+            pairs.append((blk, h))
+            self._release(blk)
+            table[i] = h
+        self.on_host.add(seq_id)
+        return pairs
+
+
 BEAM_MUTANTS = {"none": OracleAllocator, "append_before_free": _AppendBeforeFree,
                 "fork_without_reference": _ForkWithoutReference}
+
+SWAP_PINS = [pins.test_swap_out_releases_device_blocks_and_swap_in_restores_the_sequence,
+             pins.test_swapping_out_one_sharer_leaves_the_shared_blocks_to_the_other,
+             pins.test_swap_round_trip_keeps_the_attention_output,
+             pins.test_swap_out_of_blocks_changes_nothing]
+
+SWAP_MUTANTS = {"none": OracleAllocator, "swap_out_keeps_reference": _SwapOutKeepsReference,
+                "swap_in_reversed": _SwapInReversed, "partial_swap_out": _PartialSwapOut}
 
 MUTANTS = {"none": OracleAllocator, "evict_any_oldest": _EvictAnyOldest, "match_content_only": _MatchContentOnly,
            "release_to_free": _ReleaseToFree, "no_hold_on_hit": _NoHoldOnHit,
@@ -133,3 +182,12 @@ def test_planted_beam_mistakes_fail_a_pin(name, monkeypatch):
         assert failed == []
     else:
         assert failed, "mutation %s passed every beam pin" % name
+
+
+@pytest.mark.parametrize("name", sorted(SWAP_MUTANTS))
+def test_planted_swap_mistakes_fail_a_pin(name, monkeypatch):
+    failed = _failures(SWAP_MUTANTS[name], monkeypatch, SWAP_PINS)
+    if name == "none":
+        assert failed == []
+    else:
+        assert failed, "mutation %s passed every swap pin" % name

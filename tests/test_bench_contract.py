@@ -38,3 +38,22 @@ def test_bench_refuses_fewer_than_three_warmup_steps():
     import pytest
     with pytest.raises(SystemExit):
         bench.main(["--impl", "reference", "--steps", "2", "--warmup", "1"])
+
+
+def test_reference_leg_under_torchrun_prints_one_line_from_rank_zero():
+    """Launched the way the N-GPU bench is (torchrun, two ranks), the reference leg runs on
+    rank 0 only: one JSON line in all, and every rank exits 0."""
+    import socket
+    import subprocess
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--gpus", "2", "--workload", "decode-tiny-f32", "--steps", "3", "--warmup", "3"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0

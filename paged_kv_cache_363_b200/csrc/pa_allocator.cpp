@@ -49,6 +49,11 @@ struct pa_allocator {
         std::vector<int32_t> table;  // device blocks, or host blocks while swapped out
         int64_t tokens = 0;
         bool on_host = false;
+        // scratch of the batch check: tokens and last block as if the batch's earlier
+        // appends of this sequence had run (valid while epoch == the allocator's)
+        uint64_t epoch = 0;
+        int64_t pend_tokens = 0;
+        int32_t pend_last = -1;
     };
     int32_t num_blocks = 0;
     int32_t block_size = 0;
@@ -68,6 +73,14 @@ struct pa_allocator {
     // host tier for swapped-out sequences (0 blocks until pa_alloc_add_host_pool)
     int32_t num_host_blocks = 0;
     std::deque<int32_t> host_free;
+
+    // scratch of the batch check, reused across calls (a handle serves one thread at a
+    // time): per block, the batch that last changed its count and the change within it;
+    // per batch entry, its sequence
+    uint64_t epoch = 0;
+    std::vector<uint64_t> blk_epoch;
+    std::vector<int32_t> blk_dref;
+    std::vector<Seq*> batch_seq;
 
     // the sequence, if it exists and is resident on the device
     Seq* resident(int64_t seq_id)
@@ -131,43 +144,48 @@ struct pa_allocator {
     }
 
     // Blocks that appends of seq_ids[0..n) in order would take (fresh or copy-on-write),
-    // without changing anything; -1 if a sequence is unknown.
-    int64_t blocks_for_appends(const int64_t* seq_ids, int n) const
+    // without changing the allocation; -1 if a sequence is unknown or swapped out.  The
+    // batch's sequences are left in batch_seq[0..n) for the appends that follow.  No
+    // container is allocated per call: per-sequence and per-block scratch is tagged with
+    // the call's epoch, and anything older counts as untouched.
+    int64_t blocks_for_appends(const int64_t* seq_ids, int n)
     {
-        std::unordered_map<int64_t, std::pair<int64_t, int32_t>> st;  // seq -> (tokens, last block or -1)
-        std::unordered_map<int32_t, int32_t> dref;                    // reference count changes
+        ++epoch;
+        batch_seq.resize((size_t)n);
         int64_t need = 0;
         for (int k = 0; k < n; ++k) {
-            auto it = st.find(seq_ids[k]);
-            if (it == st.end()) {
-                auto q = seqs.find(seq_ids[k]);
-                if (q == seqs.end() || q->second.on_host) return -1;
-                it = st.emplace(seq_ids[k], std::make_pair(q->second.tokens,
-                                                           q->second.table.empty() ? -1 : q->second.table.back()))
-                         .first;
+            auto it = seqs.find(seq_ids[k]);
+            if (it == seqs.end() || it->second.on_host) return -1;
+            Seq& q = it->second;
+            batch_seq[(size_t)k] = &q;
+            if (q.epoch != epoch) {
+                q.epoch = epoch;
+                q.pend_tokens = q.tokens;
+                q.pend_last = q.table.empty() ? -1 : q.table.back();
             }
-            auto& [tokens, last] = it->second;
-            if (tokens % block_size == 0) {
+            if (q.pend_tokens % block_size == 0) {
                 need += 1;
-                last = -1;  // a private fresh block
-            } else if (last >= 0) {
-                auto d = dref.find(last);
-                const int32_t r = ref[(size_t)last] + (d == dref.end() ? 0 : d->second);
-                if (r > 1) {
+                q.pend_last = -1;  // a private fresh block
+            } else if (q.pend_last >= 0) {
+                const size_t b = (size_t)q.pend_last;
+                const int32_t d = blk_epoch[b] == epoch ? blk_dref[b] : 0;
+                if (ref[b] + d > 1) {
                     need += 1;
-                    dref[last] -= 1;
-                    last = -1;  // a private copy
+                    blk_epoch[b] = epoch;
+                    blk_dref[b] = d - 1;
+                    q.pend_last = -1;  // a private copy
                 }
             }
-            tokens += 1;
+            q.pend_tokens += 1;
         }
         return need;
     }
 
     // One append; the caller has checked that the blocks it may take are available.
-    int64_t append(int64_t seq_id, int32_t* src, int32_t* dst)
+    int64_t append(int64_t seq_id, int32_t* src, int32_t* dst) { return append(seqs.find(seq_id)->second, src, dst); }
+
+    int64_t append(Seq& q, int32_t* src, int32_t* dst)
     {
-        Seq& q = seqs.find(seq_id)->second;
         const int64_t i = q.tokens;
         *src = -1;
         *dst = -1;
@@ -208,6 +226,8 @@ pa_allocator* pa_alloc_create(int num_blocks, int block_size, const int32_t* fre
     a->node_key.assign((size_t)num_blocks, std::vector<int32_t>());
     a->nchild.assign((size_t)num_blocks, 0);
     a->stamp.assign((size_t)num_blocks, 0);
+    a->blk_epoch.assign((size_t)num_blocks, 0);
+    a->blk_dref.assign((size_t)num_blocks, 0);
     if (free_order) {
         std::vector<char> seen((size_t)num_blocks, 0);
         for (int i = 0; i < num_blocks; ++i) {
@@ -341,7 +361,7 @@ pa_status pa_alloc_append_slot(pa_allocator* a, int64_t seq_id, int64_t* slot_ou
         return PA_ERR_OOM;
     }
     int32_t src, dst;
-    *slot_out = a->append(seq_id, &src, &dst);
+    *slot_out = a->append(*a->batch_seq[0], &src, &dst);
     if (cow_src_out) *cow_src_out = src;
     if (cow_dst_out) *cow_dst_out = dst;
     return PA_OK;
@@ -371,7 +391,7 @@ pa_status pa_alloc_append_slots(pa_allocator* a, const int64_t* seq_ids, int n, 
     int ncow = 0;
     for (int k = 0; k < n; ++k) {
         int32_t src, dst;
-        slots_out[k] = a->append(seq_ids[k], &src, &dst);
+        slots_out[k] = a->append(*a->batch_seq[(size_t)k], &src, &dst);
         if (src >= 0) {
             cow_pairs_out[2 * ncow] = src;
             cow_pairs_out[2 * ncow + 1] = dst;

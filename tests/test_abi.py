@@ -206,7 +206,7 @@ def _replay(ops, NB, B, order, NH=0):
     return lib_a, ora
 
 
-@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("seed", range(24))
 def test_allocator_matches_oracle_on_random_scripts(seed):
     rng = np.random.default_rng(seed)
     NB, B = int(rng.integers(20, 80)), int(rng.choice([4, 16]))

@@ -81,6 +81,8 @@ struct pa_allocator {
     std::vector<uint64_t> blk_epoch;
     std::vector<int32_t> blk_dref;
     std::vector<Seq*> batch_seq;
+    std::vector<int32_t> touched;          // beam step: blocks whose count it changes
+    std::vector<const Seq*> beam_par;      // beam step: each new beam's parent
 
     // the sequence, if it exists and is resident on the device
     Seq* resident(int64_t seq_id)
@@ -432,24 +434,40 @@ pa_status pa_alloc_beam_step(pa_allocator* a, const int64_t* beam_ids, int num_b
         }
     }
     // Count the blocks the appends take, on the reference counts the forks and frees leave.
-    std::unordered_map<int32_t, int32_t> delta;
-    for (int j = 0; j < num_new; ++j)
-        for (int32_t b : a->seqs.find(beam_ids[parents[j]])->second.table) delta[b] += 1;
+    // The count changes live in the per-block scratch tagged with this call's epoch; the
+    // blocks touched are listed once each.
+    const uint64_t ep = ++a->epoch;
+    std::vector<int32_t>& touched = a->touched;
+    touched.clear();
+    auto delta = [&](int32_t b) -> int32_t& {
+        if (a->blk_epoch[(size_t)b] != ep) {
+            a->blk_epoch[(size_t)b] = ep;
+            a->blk_dref[(size_t)b] = 0;
+            touched.push_back(b);
+        }
+        return a->blk_dref[(size_t)b];
+    };
+    std::vector<const pa_allocator::Seq*>& par = a->beam_par;
+    par.resize((size_t)num_new);
+    for (int j = 0; j < num_new; ++j) {
+        par[(size_t)j] = &a->seqs.find(beam_ids[parents[j]])->second;
+        for (int32_t b : par[(size_t)j]->table) delta(b) += 1;
+    }
     for (int i = 0; i < num_beams; ++i)
-        for (int32_t b : a->seqs.find(beam_ids[i])->second.table) delta[b] -= 1;
+        for (int32_t b : a->seqs.find(beam_ids[i])->second.table) delta(b) -= 1;
     int64_t released = 0;
-    for (const auto& d : delta)
-        if (a->ref[(size_t)d.first] > 0 && a->ref[(size_t)d.first] + d.second == 0) released += 1;
+    for (int32_t b : touched)
+        if (a->ref[(size_t)b] > 0 && a->ref[(size_t)b] + a->blk_dref[(size_t)b] == 0) released += 1;
     int64_t need = 0;
     for (int j = 0; j < num_new; ++j) {
-        const pa_allocator::Seq& par = a->seqs.find(beam_ids[parents[j]])->second;
-        if (par.tokens % a->block_size == 0) {
+        const pa_allocator::Seq& p = *par[(size_t)j];
+        if (p.tokens % a->block_size == 0) {
             need += 1;
         } else {
-            const int32_t last = par.table.back();
-            if (a->ref[(size_t)last] + delta[last] > 1) {
+            const int32_t last = p.table.back();
+            if (a->ref[(size_t)last] + delta(last) > 1) {
                 need += 1;
-                delta[last] -= 1;
+                delta(last) -= 1;
             }
         }
     }
@@ -460,7 +478,7 @@ pa_status pa_alloc_beam_step(pa_allocator* a, const int64_t* beam_ids, int num_b
     // fork the chosen parents, free the old beams, install the new ones, append one slot each
     std::vector<pa_allocator::Seq> fresh((size_t)num_new);
     for (int j = 0; j < num_new; ++j) {
-        fresh[(size_t)j] = a->seqs.find(beam_ids[parents[j]])->second;
+        fresh[(size_t)j] = *par[(size_t)j];
         for (int32_t b : fresh[(size_t)j].table) a->add_ref(b);
     }
     for (int i = 0; i < num_beams; ++i) {

@@ -206,6 +206,16 @@ def _replay(ops, NB, B, order, NH=0):
     return lib_a, ora
 
 
+def test_allocator_batch_with_repeated_sequences_matches_oracle():
+    """A batch may list a sequence more than once (one append per entry, in order); the
+    pre-count must see the earlier entries' blocks, copy-on-write included."""
+    ops = [("add", 0, 5), ("fork", 0, 1), ("fork", 0, 2), ("batch", [0, 0, 1, 0, 1, 2, 2, 2, 2]),
+           ("add", 3, 4), ("fork", 3, 4), ("batch", [4, 3, 4, 3, 3, 4]), ("free", 0),
+           ("batch", [1, 2, 1, 2, 1, 2, 1, 2, 1])]
+    _replay(ops, 12, 4, list(range(12)))
+    _replay(ops + [("batch", [3] * 40)], 12, 4, list(range(12)))   # runs out: all or nothing
+
+
 @pytest.mark.parametrize("seed", range(24))
 def test_allocator_matches_oracle_on_random_scripts(seed):
     rng = np.random.default_rng(seed)

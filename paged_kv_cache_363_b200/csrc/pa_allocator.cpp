@@ -62,8 +62,20 @@ struct pa_allocator {
     std::unordered_map<int64_t, Seq> seqs;
     int64_t cow_copies = 0;
 
-    // prefix tree: key = (parent block or -1, the block's B token ids) -> block
-    std::map<std::vector<int32_t>, int32_t> tree;
+    // prefix tree: key = (parent block or -1, the block's B token ids) -> block, hashed
+    // with 64-bit FNV-1a (Fowler, Noll and Vo) over the key's words
+    struct KeyHash {
+        size_t operator()(const std::vector<int32_t>& k) const noexcept
+        {
+            uint64_t h = 14695981039346656037ull;
+            for (int32_t x : k) {
+                h ^= (uint32_t)x;
+                h *= 1099511628211ull;
+            }
+            return (size_t)h;
+        }
+    };
+    std::unordered_map<std::vector<int32_t>, int32_t, KeyHash> tree;
     std::vector<std::vector<int32_t>> node_key;  // per block: its key (empty = not in the tree)
     std::vector<int32_t> nchild;                 // per block: cached children
     std::map<uint64_t, int32_t> lru;             // unreferenced cached blocks by release stamp

@@ -79,7 +79,8 @@ struct pa_allocator {
     std::vector<std::vector<int32_t>> node_key;  // per block: its key (empty = not in the tree)
     std::vector<int32_t> nchild;                 // per block: cached children
     std::map<uint64_t, int32_t> lru;             // unreferenced cached blocks by release stamp
-    std::vector<uint64_t> stamp;                 // per block: its key in lru
+    std::map<uint64_t, int32_t> leaves;          // those of them with no cached child (the evictable ones)
+    std::vector<uint64_t> stamp;                 // per block: its key in lru (and leaves)
     uint64_t clock = 0;
 
     // host tier for swapped-out sequences (0 blocks until pa_alloc_add_host_pool)
@@ -111,13 +112,19 @@ struct pa_allocator {
         return (int64_t)q.table[(size_t)(i / block_size)] * block_size + i % block_size;
     }
 
+    // Removes an unreferenced cached leaf from the tree.  Its parent may become a leaf;
+    // an unreferenced one then joins the evictable set under its own release stamp.  (A
+    // child is only ever hung under a referenced block, so an unreferenced block's child
+    // count can only fall.)
     void evict(int32_t b)
     {
         const std::vector<int32_t>& k = node_key[(size_t)b];
-        if (k[0] >= 0) nchild[(size_t)k[0]] -= 1;
+        const int32_t p = k[0];
         tree.erase(k);
         node_key[(size_t)b].clear();
         lru.erase(stamp[(size_t)b]);
+        leaves.erase(stamp[(size_t)b]);
+        if (p >= 0 && --nchild[(size_t)p] == 0 && ref[(size_t)p] == 0) leaves.emplace(stamp[(size_t)p], p);
     }
 
     // A block with count 1: the free queue's head, else the oldest unreferenced cached
@@ -129,12 +136,7 @@ struct pa_allocator {
             b = free_q.front();
             free_q.pop_front();
         } else {
-            b = -1;
-            for (const auto& e : lru)
-                if (nchild[(size_t)e.second] == 0) {
-                    b = e.second;
-                    break;
-                }
+            b = leaves.begin()->second;  // the earliest released unreferenced leaf
             evict(b);
         }
         ref[(size_t)b] = 1;
@@ -143,7 +145,10 @@ struct pa_allocator {
 
     void add_ref(int32_t b)
     {
-        if (ref[(size_t)b]++ == 0) lru.erase(stamp[(size_t)b]);
+        if (ref[(size_t)b]++ == 0) {
+            lru.erase(stamp[(size_t)b]);
+            leaves.erase(stamp[(size_t)b]);
+        }
     }
 
     void drop_ref(int32_t b)
@@ -152,6 +157,7 @@ struct pa_allocator {
         if (cached(b)) {
             stamp[(size_t)b] = clock++;
             lru.emplace(stamp[(size_t)b], b);
+            if (nchild[(size_t)b] == 0) leaves.emplace(stamp[(size_t)b], b);
         } else {
             free_q.push_back(b);
         }

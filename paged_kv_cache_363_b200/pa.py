@@ -454,7 +454,9 @@ class Allocator:
 
     def block_table(self, seq_id):
         n = _int(0)
-        cap = self.num_blocks
+        tokens = int(lib.pa_alloc_num_tokens(self._h, int(seq_id)))
+        # a table holds ceil(tokens / B) blocks; an unknown id gets the call's own error
+        cap = max(1, -(-tokens // self.block_size)) if tokens >= 0 else 1
         out = np.empty(cap, np.int32)
         _check(lib.pa_alloc_block_table(self._h, int(seq_id), _np_ptr(out), cap, ctypes.byref(n)),
                "pa_alloc_block_table")

@@ -132,8 +132,10 @@ PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const 
  * from that plan and may be called any number of times: the last CTA of each run
  * resets the plan's work counter.  A run must use the workspace, block_tables,
  * context_lens and every size argument of its plan (the caller's promise; nothing
- * checks it), and follow it in stream order.  pa_decode is the plan followed by one
- * run.  Errors as for pa_decode.
+ * checks it), and follow it in stream order.  A run on a workspace that holds no plan
+ * reads whatever the workspace holds: undefined.  After a run that raised a device
+ * status bit (pa_device_status), plan again before the next run.  pa_decode is the
+ * plan followed by one run.  Errors as for pa_decode.
  */
 PA_API pa_status pa_decode_plan(const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
                                 int num_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,

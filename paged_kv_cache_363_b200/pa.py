@@ -180,9 +180,12 @@ PA_STATIC_WORKSPACE_BYTES = 16 * 1024 * 1024
 def pa_decode_plan(block_tables, context_lens, max_context_len, num_heads, k_cache, workspace, partition_size=0,
                    dtype=None, stream=None):
     """The work plan of a decode step into `workspace` (run it with pa_decode_run, once per layer).
-    k_cache gives the pool's shape and dtype (its data is not read)."""
+    k_cache gives the pool's shape and dtype (its data is not read); `dtype`, when given, must be
+    that dtype (the plan's choice of kernel depends on it)."""
     NB, Hkv, B, D = k_cache.shape
     S = context_lens.shape[0]
+    if dtype is not None and dtype != k_cache.dtype:
+        raise ValueError("pa_decode_plan: dtype %s differs from k_cache's %s" % (dtype, k_cache.dtype))
     st = lib.pa_decode_plan(_dev_ptr(block_tables, "block_tables"), _dev_ptr(context_lens, "context_lens"), S,
                             int(num_heads), Hkv, D, B, block_tables.shape[1], NB, int(max_context_len),
                             int(partition_size), _dev_ptr(workspace, "workspace"),

@@ -433,6 +433,35 @@ def make_batch(wl, device="cuda", values=None, fill=float("nan"), partition_size
 STEP_INPUTS = ("q", "new_k", "new_v", "slot_mapping", "cow_pairs", "block_tables", "context_lens")
 
 
+# ---------------------------------------------------------------- multi-GPU splits
+
+def sequence_shard(num_seqs, world, rank):
+    """Data-parallel split by sequence: this rank's contiguous range of a global
+    batch's sequences (shard sizes differ by at most one).  Each rank keeps its own
+    pools and allocator for its sequences; decode needs no exchange between ranks."""
+    if world < 1 or not 0 <= rank < world or num_seqs < 0:
+        raise ValueError("bad world, rank or num_seqs")
+    base, extra = divmod(num_seqs, world)
+    start = rank * base + min(rank, extra)
+    return range(start, start + base + (1 if rank < extra else 0))
+
+
+def kv_head_shard(num_heads, num_kv_heads, world, rank):
+    """Tensor-parallel split by kv head: this rank holds kv heads [k0, k1) of every
+    block (pools [num_blocks, k1 - k0, B, D]) and computes the query heads that read
+    them, [k0 * G, k1 * G) with G = num_heads / num_kv_heads.  A block table names
+    whole blocks, whatever heads they hold, so every rank runs the same allocator
+    script and holds the same tables (replicated host state, no device exchange); the
+    output stays sharded by head.  Returns (query-head range, kv-head range)."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("bad world or rank")
+    if num_kv_heads % world or num_heads % num_kv_heads:
+        raise ValueError("num_kv_heads must divide by the world size, num_heads by num_kv_heads")
+    per = num_kv_heads // world
+    g = num_heads // num_kv_heads
+    return range(rank * per * g, (rank + 1) * per * g), range(rank * per, (rank + 1) * per)
+
+
 def pack_layout(tensors, align=256):
     """Byte layout of one step's inputs packed into a single buffer.
 
@@ -564,15 +593,6 @@ class HostStepper:
         with torch.cuda.graph(g, stream=cap, capture_error_mode="relaxed"):
             self._kernels(i, mcl, cap)
         return g
-
-    def launches_per_step(self, max_context_len=None):
-        """Kernels one step launches: [copy-on-write copies], append, plan, decode, [merge]."""
-        b = self.batch
-        mcl = b.max_context_len if max_context_len is None else int(max_context_len)
-        wl = b.wl
-        part = pa.pa_decode_partition_size(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size,
-                                           mcl, b.partition_size)
-        return (1 if "cow_pairs" in self.dev_views[0] else 0) + 1 + 2 + (1 if mcl > part else 0)
 
     def drain(self):
         """Make the compute stream wait for every queued read-back."""

@@ -1,5 +1,8 @@
 """Test helpers: the oracle's side of each comparison, built only from the seeded
 generator's values and the oracle (never from anything the CUDA path produced)."""
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -72,10 +75,12 @@ def oracle_decode_side(wl, values):
                 tables_pre=tables_pre, lens_pre=lens_pre, out_pre=out_pre)
 
 
-def oracle_logical(q_rows, k_seqs, v_seqs, block_size, scale):
-    """Oracle attention of sequences given directly by their logical K/V rows
-    (each [L, Hkv, D] fp32), placed in a compact pool with an identity block table
-    (the result does not depend on placement: a pinned property of the oracle)."""
+NTHREADS = max(1, os.cpu_count() or 1)
+
+
+def _compact_pool(k_seqs, v_seqs, block_size):
+    """Sequences given by their logical K/V rows (each [L, Hkv, D] fp32) placed in a
+    compact pool, sequence after sequence, with identity block tables."""
     S = len(k_seqs)
     B = block_size
     Hkv, D = k_seqs[0].shape[1], k_seqs[0].shape[2]
@@ -95,7 +100,55 @@ def oracle_logical(q_rows, k_seqs, v_seqs, block_size, scale):
         tables[s, :nblk[s]] = np.arange(base, base + nblk[s])
         base += nblk[s]
     lens = np.array([len(k) for k in k_seqs], np.int32)
-    return oracle.decode(np.asarray(q_rows, np.float32), kp, vp, tables, lens, scale, nthreads=8)
+    return kp, vp, tables, lens
+
+
+def oracle_logical(q_rows, k_seqs, v_seqs, block_size, scale):
+    """Oracle attention of sequences given directly by their logical K/V rows
+    (each [L, Hkv, D] fp32), placed in a compact pool with an identity block table
+    (the result does not depend on placement: a pinned property of the oracle)."""
+    kp, vp, tables, lens = _compact_pool(k_seqs, v_seqs, block_size)
+    return oracle.decode(np.asarray(q_rows, np.float32), kp, vp, tables, lens, scale, nthreads=NTHREADS)
+
+
+def oracle_logical_all(q, seq_rows, block_size, scale, token_budget=200_000):
+    """oracle_logical over a whole batch, a few sequences at a time so the fp32 pools
+    stay small.  q: [S, Hq, D]; seq_rows(s) -> (K rows, V rows) of sequence s, each
+    [L_s, Hkv, D] fp32.  Returns out [S, Hq, D] float64: every row of the batch."""
+    q = np.asarray(q, np.float32)
+    S = q.shape[0]
+    out = np.zeros(q.shape, np.float64)
+    s0 = 0
+    while s0 < S:
+        ks, vs, s1, tok = [], [], s0, 0
+        while s1 < S and (s1 == s0 or tok < token_budget):
+            k, v = seq_rows(s1)
+            ks.append(np.asarray(k, np.float32))
+            vs.append(np.asarray(v, np.float32))
+            tok += len(k)
+            s1 += 1
+        out[s0:s1] = oracle_logical(q[s0:s1], ks, vs, block_size, scale)
+        s0 = s1
+    return out
+
+
+def oracle_logical_prefill(q_rows, k_seq, v_seq, block_size, scale):
+    """Oracle chunked prefill of one sequence given by its logical K/V rows
+    ([L, Hkv, D] fp32): the n = len(q_rows) queries are its last n tokens."""
+    kp, vp, tables, lens = _compact_pool([k_seq], [v_seq], block_size)
+    n = len(q_rows)
+    return oracle.prefill(np.asarray(q_rows, np.float32), kp, vp, tables, lens, np.array([0, n], np.int32), scale,
+                          nthreads=NTHREADS)
+
+
+def report_error(name, err, rows=None):
+    """Print a comparison's max-abs error and, when PA_PARITY_REPORT names a file,
+    append it there as a JSON line."""
+    print("parity %s: max-abs %.4g%s" % (name, err, "" if rows is None else " over %d rows" % rows))
+    path = os.environ.get("PA_PARITY_REPORT")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": name, "max_abs": err, "rows": rows}) + "\n")
 
 
 def max_abs(a, b):

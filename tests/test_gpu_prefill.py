@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from oracle import oracle
-from pa_testlib import TOL, max_abs
+from pa_testlib import NTHREADS, TOL, max_abs, oracle_logical_prefill, report_error
 
 pytestmark = pytest.mark.gpu
 
@@ -55,7 +55,7 @@ def _run(pa, q, k, v, tables, lens, q_start, scale):
 
 def _oracle(q, k, v, tables, lens, q_start, scale):
     return oracle.prefill(q.float().numpy(), np.nan_to_num(k.float().numpy()), np.nan_to_num(v.float().numpy()),
-                          tables, lens, q_start, scale, nthreads=8)
+                          tables, lens, q_start, scale, nthreads=NTHREADS)
 
 
 CASES = [
@@ -93,21 +93,14 @@ def test_single_token_chunks_agree_with_decode(pa):
     assert max_abs(got, out.float().cpu().numpy()) <= TOL["bf16"]
 
 
-def test_long_chunk_sampled_rows(pa):
+def test_long_chunk_every_row(pa):
     lens, nq = [2100, 1500, 4096], [640, 1500, 300]
     q, k, v, tables, L, qs = _case(9, lens, nq, 32, 8, 16)
     scale = 128 ** -0.5
     got = _run(pa, q, k, v, tables, L, qs, scale)
-    rows = np.array([0, 1, 127, 128, 639, 640, 641, 1500, 2139, 2140, 2439])
-    # the oracle on the sampled rows only: each row is its own one-row chunk at its position
-    ref = np.zeros((len(rows),) + q.shape[1:])
-    for i, r in enumerate(rows):
-        s = int(np.searchsorted(qs, r, side="right") - 1)
-        pos = int(L[s] - (qs[s + 1] - qs[s]) + (r - qs[s]))
-        ref[i] = oracle.prefill(q[r:r + 1].float().numpy(), np.nan_to_num(k.float().numpy()),
-                                np.nan_to_num(v.float().numpy()), tables[s:s + 1], np.array([pos + 1], np.int32),
-                                np.array([0, 1], np.int32), scale)[0]
-    assert max_abs(got[rows], ref) <= TOL["bf16"]
+    err = max_abs(got, _oracle(q, k, v, tables, L, qs, scale))
+    report_error("prefill long chunks (contexts 2100/1500/4096)", err, got.shape[0] * got.shape[1])
+    assert err <= TOL["bf16"], err
 
 
 def test_bad_chunk_is_flagged_and_skipped(pa):
@@ -120,6 +113,41 @@ def test_bad_chunk_is_flagged_and_skipped(pa):
     assert max_abs(got[:10], _oracle(q[:10], k, v, tables[:1], L[:1], qs[:2], 0.1)) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("bad", ["past_end", "backwards", "negative_start", "over_max_query_len"])
+def test_bad_query_rows_are_flagged_and_skipped(pa, bad):
+    """q_start is device data: a sequence whose query rows leave [0, num_query_tokens),
+    run backwards, or outnumber max_query_len is flagged and skipped whole before any
+    store, and the other sequence still matches the oracle."""
+    lens, nq = [60, 70], [10, 20]
+    q, k, v, tables, L, qs = _case(31, lens, nq, 8, 2, 16)
+    max_q = 20
+    good = 0                                   # the sequence left intact
+    qs_bad = qs.copy()
+    if bad == "past_end":
+        qs_bad[2] = qs[2] + 5                   # rows 10..34 of a 30-row q
+    elif bad == "backwards":
+        qs_bad[2] = 5                           # sequence 1 would run from row 10 back to row 5
+    elif bad == "negative_start":
+        qs_bad[0] = -5                          # sequence 0 starts before row 0
+        good = 1
+    elif bad == "over_max_query_len":
+        max_q = 15                              # sequence 1 has 20 rows
+    out = torch.full(q.shape, 7.0, dtype=torch.bfloat16, device="cuda")
+    pa.pa_prefill(out, q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(tables).cuda(), torch.from_numpy(L).cuda(),
+                  torch.from_numpy(qs_bad).cuda(), max_q, 0.1)
+    torch.cuda.synchronize()
+    assert pa.pa_device_status() == pa.PA_DEV_BAD_CONTEXT
+    got = out.float().cpu().numpy()
+    ref = _oracle(q, k, v, tables, L, qs, 0.1)
+    if good == 0:
+        assert np.all(got[10:] == 7.0)         # the bad sequence's rows are untouched
+        assert max_abs(got[:10], ref[:10]) <= TOL["bf16"]
+    else:
+        assert np.all(got[:10] == 7.0)
+        assert max_abs(got[10:], ref[10:]) <= TOL["bf16"]
+    assert pa.pa_device_status() == 0
+
+
 def test_unsupported_shapes_are_refused(pa):
     q = torch.zeros(4, 4, 64, dtype=torch.bfloat16, device="cuda")
     k = torch.zeros(4, 2, 16, 64, dtype=torch.bfloat16, device="cuda")
@@ -130,10 +158,11 @@ def test_unsupported_shapes_are_refused(pa):
     assert e.value.status == pa.PA_ERR_UNSUPPORTED
 
 
-def test_prefill_workload_full_size_sampled(pa):
+def test_prefill_workload_full_size_every_row(pa):
+    """The bench's prefill workload at full size: all 16,384 query rows of the 16
+    sequences against the oracle, sequence by sequence."""
     from paged_kv_cache_363_b200 import runner
     from paged_kv_cache_363_b200 import workloads as W
-    from pa_testlib import oracle_logical
     wl = W.make_workload(8, seed=0)
     vals = W.prefill_values(wl, "cpu")
     batch = runner.PrefillBatch(wl, "cuda", values=vals)
@@ -141,19 +170,17 @@ def test_prefill_workload_full_size_sampled(pa):
     torch.cuda.synchronize()
     assert pa.pa_device_status() == 0
     got = out.float().cpu().numpy()
-    assert np.isfinite(got).all()
     q, keys, values = vals
     koff = np.concatenate([[0], np.cumsum(wl.context_lens)])
     qs = batch.q_start_np
-    rows, ks, vs = [], [], []
-    for s in (0, 5, wl.num_seqs - 1):
-        for i in (0, 1, 511, int(wl.query_lens[s]) - 1):
-            pos = int(wl.prefix_lens[s]) + i
-            rows.append(int(qs[s]) + i)
-            ks.append(keys[koff[s]:koff[s] + pos + 1].float().numpy())
-            vs.append(values[koff[s]:koff[s] + pos + 1].float().numpy())
-    ref = oracle_logical(q[rows].float().numpy(), ks, vs, wl.block_size, wl.scale)
-    assert max_abs(got[rows], ref) <= TOL["bf16"]
+    err = 0.0
+    for s in range(wl.num_seqs):
+        L = int(wl.context_lens[s])
+        ref = oracle_logical_prefill(q[qs[s]:qs[s + 1]].float().numpy(), keys[koff[s]:koff[s] + L].float().numpy(),
+                                     values[koff[s]:koff[s] + L].float().numpy(), wl.block_size, wl.scale)
+        err = max(err, max_abs(got[qs[s]:qs[s + 1]], ref))
+    report_error("%s seed 0" % wl.name, err, got.shape[0] * got.shape[1])
+    assert err <= TOL["bf16"], err
 
 
 @pytest.mark.parametrize("scale", [0.0, -0.06, 0.3])

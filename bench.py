@@ -471,7 +471,7 @@ def plan_once_timing(batch, stream, dec_bytes, args):
     torch.cuda.synchronize(batch.device)
     return {"run_us": round(res["run"] * 1e3, 3), "run_gbs": round(dec_bytes / (res["run"] * 1e-3) / 1e9, 1),
             "plan_us": round(res["plan"] * 1e3, 3),
-            "note": "one plan per step, one run per layer; the run is the persistent decode kernel and the merge"}
+            "note": "one plan per step, one run per layer; the run is the persistent decode kernel (merge included)"}
 
 
 def e2e_leg(stepper, args, world, dev):
@@ -504,17 +504,76 @@ def e2e_leg(stepper, args, world, dev):
     return {"ms": ms, "h2d": stepper.h2d_bytes, "d2h": stepper.d2h_bytes, "host_us": 1e6 * host_s / args.steps}
 
 
-def run_prefill(args, wl, batch, dev, stream, world):
-    """Chunked prefill: TFLOP/s of pa_prefill (causal FLOPs only) against the tensor peak."""
+def make_run(name, seed, dev, overrides=None, partition=None):
+    """Workload `name` at `seed`, its seeded values on `dev`, and its batch."""
+    from paged_kv_cache_363_b200 import runner
+
+    wl = W.make_workload(W.NAME_TO_ID[name], seed=seed, **(overrides or {}))
+    if partition is not None:
+        wl.partition_size = partition
+    if isinstance(wl, W.CowWorkload):
+        values = W.cow_values(wl, dev)
+    elif isinstance(wl, W.PrefixWorkload):
+        values = W.prefix_values(wl, dev)
+    elif isinstance(wl, W.BeamWorkload):
+        values = W.beam_values(wl, dev)
+    elif isinstance(wl, W.PrefillWorkload):
+        values = W.prefill_values(wl, dev)
+    else:
+        values = W.decode_values(wl, dev)
+    return wl, values, runner.make_batch(wl, dev, values=values)
+
+
+def time_decode_steps(batch, stream, steps, warmup, dev, world):
+    """Device-resident decode steps: `warmup` untimed, then `steps` timed between a
+    barrier + synchronize on both sides, each step's decode call bracketed by its own
+    CUDA events on `stream`.  Whole-step and decode-call times are max over ranks."""
     import torch
+    import torch.distributed as dist
     from paged_kv_cache_363_b200 import pa
 
-    flops = wl.flops()
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         batch.step(stream)
     torch.cuda.synchronize(dev)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        t_start.record(stream)
+        for k in range(steps):
+            batch.append(stream)
+            ev_s[k].record(stream)
+            batch.decode(stream=stream)
+            ev_e[k].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    dec_ms = [a.elapsed_time(b) for a, b in zip(ev_s, ev_e)]
+    return {"ms_max": reduce_max(t_start.elapsed_time(t_end), dev), "dec_ms": dec_ms,
+            "dec_avg_max": reduce_max(statistics.mean(dec_ms), dev), "clocks": clk.summary(),
+            "flags": pa.pa_device_status(), "out_ok": bool(torch.isfinite(batch.out.float()).all().item())}
+
+
+def time_prefill_steps(batch, stream, steps, warmup, dev, world):
+    """pa_prefill calls: `warmup` untimed, then `steps` timed, each bracketed by CUDA
+    events on `stream`; whole-run and per-call times are max over ranks."""
+    import torch
+    import torch.distributed as dist
+    from paged_kv_cache_363_b200 import pa
+
+    for _ in range(warmup):
+        batch.step(stream)
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
     with ClockSampler(dev.index) as clk:
         t0.record(stream)
         for a, b in evs:
@@ -523,9 +582,108 @@ def run_prefill(args, wl, batch, dev, stream, world):
             b.record(stream)
         t1.record(stream)
         torch.cuda.synchronize(dev)
-    ms = reduce_max(t0.elapsed_time(t1), dev)
+    if world > 1:
+        dist.barrier()
     per = [a.elapsed_time(b) for a, b in evs]
-    avg = reduce_max(statistics.mean(per), dev)
+    return {"ms_max": reduce_max(t0.elapsed_time(t1), dev), "per_ms": per,
+            "avg_max": reduce_max(statistics.mean(per), dev), "clocks": clk.summary(),
+            "flags": pa.pa_device_status(), "out_ok": bool(torch.isfinite(batch.out.float()).all().item())}
+
+
+def bf16_peak():
+    """The measured cuBLAS bf16 burst peak (TFLOP/s), else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (cuBLAS bf16 burst)"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def decode_launches(batch):
+    """Kernels one step launches: [copy-on-write copies], append, plan, persistent
+    decode (which also merges the partitions of split sequences)."""
+    cow = 1 if getattr(batch, "cow_pairs", None) is not None and batch.cow_pairs.numel() else 0
+    return cow + 1 + 2
+
+
+def side_workload(name, args, dev, world, rank):
+    """One more workload measured in the same run as the headline: its own batch (seeded
+    per rank), `steps` device-resident steps, the decode call's (or the prefill call's)
+    roofline fraction against the measured peak."""
+    import torch
+    from paged_kv_cache_363_b200 import pa
+
+    steps = max(5, min(args.steps, 20))
+    wl, values, batch = make_run(name, rank_seed(args.seed, rank), dev)
+    del values
+    stream = torch.cuda.current_stream(dev)
+    if isinstance(wl, W.PrefillWorkload):
+        t = time_prefill_steps(batch, stream, steps, args.warmup, dev, world)
+        flops = wl.flops()
+        peak, kind = bf16_peak()
+        achieved = flops / (t["avg_max"] * 1e-3) / 1e12
+        return {"metric": "chunked prefill attention TFLOP/s (causal FLOPs)",
+                "value": round(world * flops * steps / (t["ms_max"] * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "steps": steps, "ms_per_step": round(t["ms_max"] / steps, 5),
+                "config": {"workload": wl.name, "num_seqs": wl.num_seqs, "num_heads": wl.num_heads,
+                           "num_kv_heads": wl.num_kv_heads, "query_tokens": int(wl.query_lens.sum()),
+                           "context_tokens": int(wl.context_lens.sum()), "seed": wl.seed},
+                "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel", "achieved": round(achieved, 2),
+                             "peak": peak, "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                             "algorithmic_flops_per_launch": flops, "avg_launch_us": round(t["avg_max"] * 1e3, 3)},
+                "gpu_launches": steps, "clocks": t["clocks"], "device_status": t["flags"],
+                "output_finite": t["out_ok"]}
+    part = pa.pa_decode_partition_size(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size,
+                                       batch.max_context_len, batch.partition_size)
+    dec_bytes = batch.decode_bytes()
+    step_bytes = dec_bytes + batch.append_bytes()
+    t = time_decode_steps(batch, stream, steps, args.warmup, dev, world)
+    peak, peak_kind = measured_hbm_peak()
+    achieved = dec_bytes / (t["dec_avg_max"] * 1e-3) / 1e9
+    roof = {"bound": "hbm", "kernel": "pa_decode (plan kernel + persistent decode kernel, merge included)",
+            "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "algorithmic_bytes_per_launch": dec_bytes,
+            "avg_launch_us": round(t["dec_avg_max"] * 1e3, 3),
+            "launch_us_p10_p50_p90": [round(float(np.percentile(t["dec_ms"], q)) * 1e3, 3) for q in (10, 50, 90)]}
+    if isinstance(wl, W.CowWorkload):
+        roof["note"] = ("logical bytes: the 4 streams of a prompt share its blocks, which are re-read from L2, "
+                        "so the fraction can exceed 1")
+    return {"value": round(world * step_bytes * steps / (t["ms_max"] * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "steps": steps, "ms_per_step": round(t["ms_max"] / steps, 5),
+            "seqs_per_s": round(world * wl.num_seqs * steps / (t["ms_max"] * 1e-3), 1),
+            "config": dict(workload_config(wl, part, batch), l2=l2_note(batch, dec_bytes)),
+            "roofline": roof, "gpu_launches": decode_launches(batch) * steps, "clocks": t["clocks"],
+            "device_status": t["flags"], "output_finite": t["out_ok"]}
+
+
+SIDE_WORKLOADS = ("decode-gqa-bf16", "long-splitk-bf16", "cow-sampling-bf16", "prefill-chunk-bf16")
+
+
+def side_workload_names(args):
+    """Workloads measured after the headline in the same run: by default the GQA,
+    long-context, copy-on-write and prefill workloads when the headline is the
+    Llama-7B-shaped decode at its defaults; none for other headlines or overrides."""
+    if args.workloads == "none":
+        return []
+    if args.workloads != "auto":
+        names = [n for n in args.workloads.split(",") if n]
+        for n in names:
+            if n not in W.NAME_TO_ID:
+                raise SystemExit("unknown workload %s" % n)
+        return names
+    if args.workload == "decode-mha-bf16" and profiled_config(args) and args.pool_blocks is None:
+        return list(SIDE_WORKLOADS)
+    return []
+
+
+def run_prefill(args, wl, batch, dev, stream, world):
+    """Chunked prefill: TFLOP/s of pa_prefill (causal FLOPs only) against the tensor peak."""
+    import torch
+    from paged_kv_cache_363_b200 import pa
+
+    flops = wl.flops()
+    t = time_prefill_steps(batch, stream, args.steps, args.warmup, dev, world)
+    ms, avg = t["ms_max"], t["avg_max"]
     # end to end: each step uploads its query rows from pinned memory and reads the output back
     qh = batch.q.cpu().pin_memory()
     oh = torch.empty(batch.out.shape, dtype=batch.out.dtype).pin_memory()
@@ -539,14 +697,8 @@ def run_prefill(args, wl, batch, dev, stream, world):
     e_e.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = reduce_max(e_s.elapsed_time(e_e), dev)
-    peak = None
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            peak, kind = float(json.load(f)["bf16_tflops"]), "measured (cuBLAS bf16 burst)"
-    except Exception:
-        peak, kind = 1590.0, "fallback"
+    peak, kind = bf16_peak()
     achieved = flops / (avg * 1e-3) / 1e12
-    out_ok = bool(torch.isfinite(batch.out.float()).all().item())
     line = {
         "metric": "chunked prefill attention TFLOP/s over the paged KV cache (causal FLOPs)",
         "value": round(world * flops * args.steps / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": world,
@@ -567,8 +719,8 @@ def run_prefill(args, wl, batch, dev, stream, world):
                 "h2d_bytes_per_step": qh.numel() * qh.element_size(),
                 "d2h_bytes_per_step": oh.numel() * oh.element_size(), "ms_per_step": round(e2e_ms / args.steps, 5)},
         "gpu_launches": args.steps,
-        "clocks": clk.summary(),
-        "device_status": pa.pa_device_status(), "output_finite": out_ok,
+        "clocks": t["clocks"],
+        "device_status": t["flags"], "output_finite": t["out_ok"],
     }
     return line
 
@@ -588,25 +740,11 @@ def run_gpu(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
-    from paged_kv_cache_363_b200 import runner
+    from paged_kv_cache_363_b200 import pa, runner
 
     overrides = {} if args.pool_blocks is None else {"num_blocks": args.pool_blocks}
     overrides.update(parse_overrides(args.set))
-    wl = W.make_workload(W.NAME_TO_ID[args.workload], seed=rank_seed(args.seed, rank), **overrides)
-    if args.partition is not None:
-        wl.partition_size = args.partition
-    if isinstance(wl, W.CowWorkload):
-        values = W.cow_values(wl, dev)
-    elif isinstance(wl, W.PrefixWorkload):
-        values = W.prefix_values(wl, dev)
-    elif isinstance(wl, W.BeamWorkload):
-        values = W.beam_values(wl, dev)
-    elif isinstance(wl, W.PrefillWorkload):
-        values = W.prefill_values(wl, dev)
-    else:
-        values = W.decode_values(wl, dev)
-    batch = runner.make_batch(wl, dev, values=values)
-    from paged_kv_cache_363_b200 import pa
+    wl, values, batch = make_run(args.workload, rank_seed(args.seed, rank), dev, overrides, args.partition)
     if isinstance(wl, W.PrefillWorkload):
         stream = torch.cuda.current_stream(dev)
         line = run_prefill(args, wl, batch, dev, stream, world)
@@ -617,7 +755,6 @@ def run_gpu(args):
         return 0
     part = pa.pa_decode_partition_size(wl.num_seqs, wl.num_heads, wl.num_kv_heads, wl.head_dim, wl.block_size,
                                        batch.max_context_len, batch.partition_size)
-    n_part = -(-batch.max_context_len // part)
     stream = torch.cuda.current_stream(dev)
     torch.cuda.synchronize(dev)
     if pa.pa_device_status() != 0:
@@ -625,39 +762,12 @@ def run_gpu(args):
 
     dec_bytes = batch.decode_bytes()
     step_bytes = dec_bytes + batch.append_bytes()
-    cow_launch = 1 if getattr(batch, "cow_pairs", None) is not None and batch.cow_pairs.numel() else 0
-    # [copy-on-write copies], append, plan, persistent decode, [merge of split sequences]
-    launches_per_step = cow_launch + 1 + 2 + (1 if n_part > 1 else 0)
+    launches_per_step = decode_launches(batch)
 
     # ---- device-resident timing
-    for _ in range(args.warmup):
-        batch.step(stream)
-    torch.cuda.synchronize(dev)
-    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clk:
-        t_start.record(stream)
-        for k in range(args.steps):
-            batch.append(stream)
-            ev_s[k].record(stream)
-            batch.decode(stream=stream)
-            ev_e[k].record(stream)
-        t_end.record(stream)
-        torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    ms = t_start.elapsed_time(t_end)
-    dec_ms = [a.elapsed_time(b) for a, b in zip(ev_s, ev_e)]
-    ms_max = reduce_max(ms, dev)
-    dec_avg = statistics.mean(dec_ms)
-    dec_avg_max = reduce_max(dec_avg, dev)
-    out_ok = bool(torch.isfinite(batch.out.float()).all().item())
-    flags = pa.pa_device_status()
+    t = time_decode_steps(batch, stream, args.steps, args.warmup, dev, world)
+    ms_max, dec_ms, dec_avg_max = t["ms_max"], t["dec_ms"], t["dec_avg_max"]
+    out_ok, flags = t["out_ok"], t["flags"]
 
     e2e = None
     if not args.skip_e2e:
@@ -689,7 +799,7 @@ def run_gpu(args):
                        parallelism="replicas: one batch per GPU (dp%d)" % world),
         "seqs_per_s": round(world * wl.num_seqs * args.steps / (ms_max * 1e-3), 1),
         "pct_of_peak": round(100.0 * value / peak, 2),
-        "roofline": {"bound": "hbm", "kernel": "pa_decode (plan kernel + persistent decode kernel)",
+        "roofline": {"bound": "hbm", "kernel": "pa_decode (plan kernel + persistent decode kernel, merge included)",
                      "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
                      "traffic": (profile_traffic("decode_persistent_kernel", wl.name)
@@ -700,12 +810,21 @@ def run_gpu(args):
         "plan_once": plan_once,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
+        "clocks": t["clocks"],
         "device_status": flags, "output_finite": out_ok,
     }
     if world == 1 and not args.no_cpu_baseline and isinstance(wl, W.DecodeWorkload):
         gbs, seqs_s, cores, sample, _ = oracle_leg(wl, args.cpu_budget, values)
         line["cpu_baseline"] = cpu_baseline_entry(wl, values, gbs, cores, sample, args.cpu_budget / 4)
+    # ---- the other workloads, each in its own timed region after the headline's
+    side = side_workload_names(args)
+    if side:
+        del batch, values
+        torch.cuda.empty_cache()
+        line["workloads"] = {}
+        for name in side:
+            line["workloads"][name] = side_workload(name, args, dev, world, rank)
+            torch.cuda.empty_cache()
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -731,6 +850,9 @@ def main(argv=None):
                     help="replay each buffer's kernels from a captured CUDA graph in the end-to-end leg")
     ap.add_argument("--pool-blocks", type=int, default=None,
                     help="override the pool size (profiling runs on a smaller device footprint)")
+    ap.add_argument("--workloads", default="auto",
+                    help="comma list of workloads measured after the headline in the same run (auto: GQA, long "
+                         "context, copy-on-write and prefill after the default headline; none: skip)")
     ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
                     help="override a workload field, e.g. num_kv_heads=32 or lens=uniform,128,2048")
     args = ap.parse_args(argv)

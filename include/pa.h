@@ -81,8 +81,9 @@ typedef enum { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
  * Context-partition length (tokens) that pa_decode uses for these arguments:
  * `partition_size` itself when > 0 (it must be a multiple of block_size, at most
  * 4096), else an automatic choice.  A sequence longer than one partition is
- * split into partitions whose softmax states are merged by log-sum-exp in a
- * second kernel.  Returns a negative pa_status on invalid arguments.
+ * split into partitions whose softmax states are merged by log-sum-exp (by the
+ * decode kernel's warps that have run out of partitions to attend over, at the
+ * end of the call).  Returns a negative pa_status on invalid arguments.
  */
 PA_API int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
                              int max_context_len, int partition_size);
@@ -92,7 +93,8 @@ PA_API int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_head
  * num_seqs > 0).  The workspace holds the call's work plan (the (sequence,
  * partition) pairs, longest first, and a work counter) and, when a sequence can
  * span more than one partition, per (sequence, query head, partition) the running
- * max, the softmax sum and the unnormalised head_dim-vector of the partition.
+ * max, the softmax sum and the unnormalised head_dim-vector of the partition, and
+ * two merge counters per (sequence, query head).
  */
 PA_API size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
                                 int max_context_len, int partition_size);
@@ -129,13 +131,15 @@ PA_API pa_status pa_decode(void* out, const void* q, const void* k_cache, const 
  * over the same sequences (the same block_tables, context_lens and sizes; other q,
  * out and caches per layer).  pa_decode_plan writes the work plan into the workspace
  * (the plan kernel only; no q, out or caches); pa_decode_run then runs the decode
- * from that plan and may be called any number of times: the last CTA of each run
- * resets the plan's work counter.  A run must use the workspace, block_tables,
+ * from that plan and may be called any number of times: the last CTA of each run to
+ * stop taking work (at the end of the work list, or on a wait that gave up) resets
+ * the plan's work counter.  A run must use the workspace, block_tables,
  * context_lens and every size argument of its plan (the caller's promise; nothing
  * checks it), and follow it in stream order.  A run on a workspace that holds no plan
- * reads whatever the workspace holds: undefined.  After a run that raised a device
- * status bit (pa_device_status), plan again before the next run.  pa_decode is the
- * plan followed by one run.  Errors as for pa_decode.
+ * reads whatever the workspace holds: undefined.  A run that raised a device status
+ * bit (pa_device_status) left some outputs unwritten; planning again before the next
+ * run is the safe course.  pa_decode is the plan followed by one run.  Errors as for
+ * pa_decode.
  */
 PA_API pa_status pa_decode_plan(const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
                                 int num_heads, int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
@@ -164,6 +168,8 @@ PA_API pa_status pa_decode_run(void* out, const void* q, const void* k_cache, co
  *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  *  - The first call made on a device resolves that device's array address
  *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *    After a device reset (cudaDeviceReset) the next call resolves it again, so
+ *    that call too belongs before any capture.
  *  - Arguments whose pa_decode_workspace_size() exceeds
  *    PA_STATIC_WORKSPACE_BYTES return PA_ERR_UNSUPPORTED before any device work
  *    (a larger partition_size needs less).
@@ -256,10 +262,13 @@ PA_API pa_status pa_selftest_bounded_wait(uint64_t* waited_ns, void* stream);
  * query i at position context_lens[s] - n_s + i.  Each attends causally to tokens
  * 0..its position: out[row][h] = softmax_t(scale * q[row][h] . K_t) . V_t over
  * t <= position, with query head h reading kv head h / (num_heads / num_kv_heads).
- * q_start (device, int32, S+1 entries, q_start[0] = 0, non-decreasing) and
- * context_lens are device arrays; max_query_len bounds every n_s (it sizes the grid:
- * larger n_s leave rows unwritten).  A sequence with n_s > context_lens[s] or a
- * context beyond its table raises PA_DEV_BAD_CONTEXT and is skipped.  bf16 only,
+ * q_start (device, int32, S+1 entries, non-decreasing, within [0, num_query_tokens])
+ * and context_lens are device arrays; max_query_len bounds every n_s (it sizes the
+ * grid).  The kernel checks each sequence's device data before any store: a
+ * sequence whose rows leave [0, num_query_tokens) or run backwards (q_start[s] < 0,
+ * q_start[s+1] > num_query_tokens, q_start[s+1] < q_start[s]), with
+ * n_s > max_query_len, n_s > context_lens[s], or a context beyond its table row
+ * raises PA_DEV_BAD_CONTEXT and is skipped whole (its output rows untouched).  bf16 only,
  * head_dim 128, num_heads / num_kv_heads in {1, 2, 4, 8} (else PA_ERR_UNSUPPORTED).
  * With every n_s = 1 this is pa_decode.  No workspace.  Asynchronous on stream.
  */

@@ -30,6 +30,7 @@ __device__ unsigned int g_status_word;
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 unsigned int* g_status_ptr[kMaxDevices] = {};
+unsigned long long g_status_ctx[kMaxDevices] = {};  // context id each cached address belongs to
 
 pa_status cuda_fail(const char* what, cudaError_t e)
 {
@@ -37,7 +38,8 @@ pa_status cuda_fail(const char* what, cudaError_t e)
     return PA_ERR_CUDA;
 }
 
-// Address of the status word on the current device (resolved once per device).
+// Address of the status word on the current device: resolved once per device and
+// context, and again after a device reset has re-created the context.
 pa_status status_ptr(unsigned int** out)
 {
     int dev = 0;
@@ -48,11 +50,13 @@ pa_status status_ptr(unsigned int** out)
         return PA_ERR_INVALID;
     }
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_status_ptr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (!g_status_ptr[dev] || ctx == 0 || g_status_ctx[dev] != ctx) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_status_word);
         if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress(status word)", e);
         g_status_ptr[dev] = static_cast<unsigned int*>(p);
+        g_status_ctx[dev] = current_context_id();  // current now, if it was not before the lookup
     }
     *out = g_status_ptr[dev];
     return PA_OK;
@@ -205,6 +209,7 @@ pa_status decode_call(const char* fn, int phases, void* out, const void* q, cons
     if (np > 1) {
         a.ws_acc = reinterpret_cast<float*>(ws + wl.acc);
         a.ws_ml = reinterpret_cast<float*>(ws + wl.ml);
+        a.ready = reinterpret_cast<unsigned int*>(ws + wl.ready);
     }
     unsigned int* status = nullptr;
     st = status_ptr(&status);
@@ -244,6 +249,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     int max_context_len, float scale, int partition_size, void* workspace,
                     size_t workspace_bytes, pa_dtype dtype, void* stream)
 {
+    pa::CallRange range("pa_decode");
     return decode_call("pa_decode", kDecodePlan | kDecodeRun, out, q, k_cache, v_cache, block_tables, context_lens,
                        num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
                        max_context_len, scale, partition_size, workspace, workspace_bytes, dtype, stream);
@@ -254,6 +260,7 @@ pa_status pa_decode_plan(const int32_t* block_tables, const int32_t* context_len
                          int max_context_len, int partition_size, void* workspace, size_t workspace_bytes,
                          pa_dtype dtype, void* stream)
 {
+    pa::CallRange range("pa_decode_plan");
     return decode_call("pa_decode_plan", kDecodePlan, nullptr, nullptr, nullptr, nullptr, block_tables, context_lens,
                        num_seqs, num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
                        max_context_len, 1.0f, partition_size, workspace, workspace_bytes, dtype, stream);
@@ -265,6 +272,7 @@ pa_status pa_decode_run(void* out, const void* q, const void* k_cache, const voi
                         int max_context_len, float scale, int partition_size, void* workspace,
                         size_t workspace_bytes, pa_dtype dtype, void* stream)
 {
+    pa::CallRange range("pa_decode_run");
     return decode_call("pa_decode_run", kDecodeRun, out, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
                        num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
                        max_context_len, scale, partition_size, workspace, workspace_bytes, dtype, stream);
@@ -274,6 +282,7 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache
                                const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
                                int block_size, int num_blocks, pa_dtype dtype, void* stream)
 {
+    pa::CallRange range("pa_reshape_and_cache");
     pa_status st = check_common("pa_reshape_and_cache", num_kv_heads, head_dim, block_size, num_blocks, dtype);
     if (st != PA_OK) return st;
     if (num_tokens < 0) {
@@ -371,6 +380,7 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapp
                          int num_kv_heads, int head_dim, int block_size, int num_blocks, pa_dtype dtype,
                          void* stream)
 {
+    pa::CallRange range("pa_copy_blocks");
     pa_status st = check_common("pa_copy_blocks", num_kv_heads, head_dim, block_size, num_blocks, dtype);
     if (st != PA_OK) return st;
     if (num_pairs < 0 || num_pairs > 65535) {
@@ -407,6 +417,7 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
                      int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
                      int num_query_tokens, int max_query_len, float scale, pa_dtype dtype, void* stream)
 {
+    pa::CallRange range("pa_prefill");
     pa_status st = check_common("pa_prefill", num_kv_heads, head_dim, block_size, num_blocks, dtype);
     if (st != PA_OK) return st;
     if (dtype != PA_DTYPE_BF16 || head_dim != 128) {
@@ -455,6 +466,8 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
     a.max_blocks_per_seq = max_blocks_per_seq;
     a.num_blocks = num_blocks;
     a.block_size = block_size;
+    a.num_query_tokens = num_query_tokens;
+    a.max_query_len = max_query_len;
     a.scale_log2 = scale * 1.4426950408889634f;
     const cudaError_t e =
         launch_prefill(a, group, num_query_tokens, max_query_len, static_cast<cudaStream_t>(stream));
@@ -489,6 +502,7 @@ pa_status pa_swap_blocks(void* dst_k_cache, void* dst_v_cache, const void* src_k
                          const int64_t* block_mapping, int num_pairs, int num_kv_heads, int head_dim, int block_size,
                          int num_src_blocks, int num_dst_blocks, pa_dtype dtype, void* stream)
 {
+    pa::CallRange range("pa_swap_blocks");
     pa_status st = check_common("pa_swap_blocks", num_kv_heads, head_dim, block_size, num_src_blocks, dtype);
     if (st != PA_OK) return st;
     if (num_dst_blocks <= 0) {

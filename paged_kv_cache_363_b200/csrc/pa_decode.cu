@@ -25,9 +25,10 @@
 //  * At the end of a unit each warp leaves its softmax state in shared memory and goes
 //    on with the next unit; the warp that consumed the unit's last tile merges the four
 //    states.  A sequence longer than one partition leaves (max, sum, unnormalised
-//    output) per partition in the workspace and a log-sum-exp merge kernel combines
-//    them.  Plan, persistent and merge kernels are chained with programmatic dependent
-//    launch.
+//    output) per partition in the workspace; consumer warps left without units at
+//    the tail of the grid merge those partitions by log-sum-exp as they finish, so no
+//    second kernel waits for the whole grid to drain.  The plan and persistent
+//    kernels are chained with programmatic dependent launch.
 //  * Logits are kept in base-2 units (q pre-scaled by scale*log2 e) and exponentials
 //    use exp2f, the reformulation of online softmax by Milakov & Gimelshein (2018).
 //  * Every wait is bounded: a wait that runs out raises PA_DEV_WAIT_TIMEOUT and the
@@ -66,6 +67,31 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
             fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
     });
     return fn;
+}
+
+unsigned long long current_context_id()
+{
+    using GetCurrent = CUresult (*)(CUcontext*);
+    using GetId = CUresult (*)(CUcontext, unsigned long long*);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrent>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetId>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
 }
 
 // The pool [num_blocks][kv_heads][B][D] as a 2-D bf16 tensor of rows of D elements;
@@ -241,7 +267,12 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
         fence_mbar_init();
     }
     __syncthreads();
-    pdl_wait_primary();  // the plan kernel's list and counter are visible after this
+    // A CTA of the first wave starts on its own unit while the plan kernel still runs:
+    // only its unit producer (before its second unit) and its consumers (before the
+    // merge) wait for the plan.  Every other CTA waits here; the plan kernel's list and
+    // counters are visible after the wait.
+    const bool early = (int)blockIdx.x < a.first_wave;
+    if (!early) pdl_wait_primary();
 
     auto slot = [&](int k) { return smem + P::OFF_SLOT + (k % UR) * P::SLOT_BYTES; };
     auto slot_table = [&](int k) { return reinterpret_cast<int*>(slot(k) + P::QBYTES); };
@@ -251,16 +282,43 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
         // ---------------- unit producer: takes units from the plan, fills the unit ring
         // The first unit's list entry is requested together with the pair count, not
         // after it: its index is inside the list whatever the count (the grid has at
-        // most one CTA per unit the list can hold).
-        const unsigned npairs = __ldcg(a.plan + 1);
-        const uint2 e_first = __ldcg(a.plan_list + blockIdx.x / (unsigned)a.num_kv_heads);
-        const unsigned nunits = npairs * (unsigned)a.num_kv_heads;
+        // most one CTA per unit the list can hold).  A first-wave CTA knows its first
+        // unit without the list: partition 0 of sequence b / Hkv (the plan puts that
+        // pair at list position b / Hkv).
+        unsigned nunits = 0;
+        uint2 e_first;
+        // count this CTA as started (the tail merge waits on other CTAs only once all have)
+        auto plan_ready = [&]() {
+            nunits = __ldcg(a.plan + 1) * (unsigned)a.num_kv_heads;
+            if (lane == 0 && a.ready) atomicAdd(a.plan + 7, 1u);
+        };
+        if (early) {
+            const int s0 = (int)(blockIdx.x / (unsigned)a.num_kv_heads);
+            e_first = make_uint2((unsigned)s0 << 11, (unsigned)clamped_context(a, s0, B, false));
+        } else {
+            e_first = __ldcg(a.plan_list + blockIdx.x / (unsigned)a.num_kv_heads);
+            plan_ready();
+        }
+        // This CTA takes no more units.  The last CTA to stop (at the end marker or on
+        // a wait that gave up) resets the work counter, so the plan in the workspace
+        // serves the next run as it is (one plan per decode step, one run per layer);
+        // it happens while the CTAs still finish their last units, off the kernel's
+        // critical path.  Lane 0 only.
+        auto leave = [&]() {
+            if (atomicAdd(a.plan + 4, 1u) == gridDim.x - 1) {
+                a.plan[0] = 0u;
+                a.plan[4] = 0u;
+            }
+        };
         int first = 0;
         int k = 0;
         bool ended = false;
         for (;; ++k) {
             if (k >= UR && !mbar_wait_warp(&uempty[k % UR], ((k / UR) & 1) ^ 1, abort_flag)) {
-                if (lane == 0) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+                if (lane == 0) {
+                    atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+                    leave();
+                }
                 *abort_flag = 1;
                 break;
             }
@@ -268,22 +326,19 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
             // the first unit of CTA b is unit b; later ones come from the counter
             unsigned u = blockIdx.x;
             if (k > 0) {
+                if (k == 1 && early) {
+                    pdl_wait_primary();
+                    plan_ready();
+                }
                 if (lane == 0) u = gridDim.x + atomicAdd(a.plan, 1u);
                 u = __shfl_sync(0xffffffffu, u, 0);
             }
-            if (u >= nunits) {
+            if (u >= nunits && !(k == 0 && early)) {
                 if (lane == 0) {
                     info->flags = kEndUnit;
                     mbar_arrive(&utab[k % UR]);
                     mbar_arrive(&ufull[k % UR]);
-                    // This CTA takes no more units.  The last CTA to get here resets the
-                    // work counter, so the plan in the workspace serves the next run as it
-                    // is (one plan per decode step, one run per layer); it happens while the
-                    // CTAs still finish their last units, off the kernel's critical path.
-                    if (atomicAdd(a.plan + 4, 1u) == gridDim.x - 1) {
-                        a.plan[0] = 0u;
-                        a.plan[4] = 0u;
-                    }
+                    leave();
                 }
                 ended = true;
                 break;
@@ -294,7 +349,7 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
             const int part = (int)(e.x & 2047u);
             const int L = (int)e.y;
             const int nblk_seq = (L + B - 1) / B;
-            const int pb = (int)a.plan[2];
+            const int pb = (k == 0 && early) ? a.partition_blocks : (int)a.plan[2];  // equal when early
             const int b0 = part * pb;
             const int nb = max(0, min(pb, nblk_seq - b0));
             int* tab = slot_table(k);
@@ -421,10 +476,18 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
                     ok = false;
                     break;
                 }
-                finish_unit_warp<T, D, G, NCW>(a, mg_m, mg_l, mg_acc, info->s, info->kvh, info->part,
-                                               (info->flags & kSplitUnit) != 0, first % NCW, lane);
+                const bool split = (info->flags & kSplitUnit) != 0;
+                finish_unit_warp<T, D, G, NCW>(a, mg_m, mg_l, mg_acc, info->s, info->kvh, info->part, split,
+                                               first % NCW, lane);
                 __syncwarp();
                 if (lane == 0) {
+                    // the partition's state (all lanes' stores, ordered by the warp barrier)
+                    // is published to the tail merge with a release count, once the plan
+                    // kernel (which zeroes the counts) is done: a first-wave unit may end first
+                    if (split) {
+                        if (early && k == 0) pdl_wait_primary();
+                        red_release_add(a.ready + (size_t)info->s * a.num_kv_heads + info->kvh, 1u);
+                    }
                     mbar_arrive(mg_free);
                     mbar_arrive(&uempty[k % UR]);
                 }
@@ -433,6 +496,11 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
         if (!ok) {
             if (lane == 0) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
             *abort_flag = 1;
+        }
+        // no more units for this CTA: merge finished split sequences meanwhile
+        if (a.ready) {
+            if (early) pdl_wait_primary();  // the plan's split list and counters
+            tail_merge_warp<T, D, G>(a, B, ok, lane, gridDim.x * (unsigned)NCW);
         }
     }
 }
@@ -490,6 +558,14 @@ cudaError_t launch_persistent(const DecodeArgs& a, cudaStream_t stream)
     const unsigned grid = (unsigned)(units < ctas ? units : ctas);
     DecodeArgs args = a;
     args.num_ctas = (int)grid;
+    // The first wave: with the partition fixed, CTA b < first_wave starts on kv head
+    // b % Hkv of partition 0 of sequence b / Hkv without waiting for the plan.  The plan
+    // grows an automatic partition only when the tokens of all sequences exceed
+    // 4 x partition x CTAs, which the bound num_seqs x max_context_len rules out here.
+    const bool fixed_partition =
+        !a.adaptive || (int64_t)a.num_seqs * a.max_context_len <= 4LL * a.partition_blocks * BS * (int64_t)grid;
+    const int64_t pairs0 = (int64_t)a.num_seqs * a.num_kv_heads;
+    args.first_wave = fixed_partition ? (int)(pairs0 < (int64_t)grid ? pairs0 : (int64_t)grid) : 0;
 
     if (a.phases & kDecodePlan) {
         // one CTA; fewer threads for small batches keep its barriers short
@@ -499,10 +575,8 @@ cudaError_t launch_persistent(const DecodeArgs& a, cudaStream_t stream)
         if (e != cudaSuccess) return e;
     }
     if (!(a.phases & kDecodeRun)) return cudaSuccess;
-    e = launch_pdl(decode_persistent_kernel<Cons, BS>, dim3(grid), dim3(P::THREADS), (size_t)P::SMEM, stream, args,
-                   tk, tv);
-    if (e != cudaSuccess || a.num_partitions <= 1) return e;
-    return launch_merge<typename Cons::T, P::D>(args, BS, stream);
+    return launch_pdl(decode_persistent_kernel<Cons, BS>, dim3(grid), dim3(P::THREADS), (size_t)P::SMEM, stream,
+                      args, tk, tv);
 }
 
 template <typename T, int D, int B>

@@ -7,10 +7,21 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "pa.h"
 
 namespace pa {
+
+// A profiler range (NVTX, header-only v3) around one C-ABI call, so a profiler can
+// pick out pa_decode, pa_prefill and the companions by name.  With no profiler
+// attached the push and pop are calls into the NVTX no-op stubs.
+struct CallRange {
+    explicit CallRange(const char* name) { nvtxRangePushA(name); }
+    ~CallRange() { nvtxRangePop(); }
+    CallRange(const CallRange&) = delete;
+    CallRange& operator=(const CallRange&) = delete;
+};
 
 // Largest context partition (tokens) and largest number of partitions per sequence.
 constexpr int kMaxPartitionTokens = 4096;
@@ -25,12 +36,16 @@ struct DecodeArgs {
     const int32_t* context_lens;
     unsigned int* plan;        // [0] work counter, [1] (sequence, partition) pairs, [2] blocks per
                                // partition, [3] sequences split into several partitions, [4] CTAs
-                               // that finished the current run
+                               // that stopped taking units in the current run, [5] merge-row
+                               // counter, [6] consumer warps done with merging, [7] CTAs started
     uint2* plan_list;          // [S * NP] longest first: {sequence << 11 | partition, context length}
     uint2* split_list;         // [S] the sequences split into several partitions (plan[3] of them):
                                // {sequence, context length}
     float* ws_acc;             // [S][Hq][NP][D] unnormalised partition outputs (NP > 1)
     float* ws_ml;              // [S][Hq][NP][2] (running max in log2 units, softmax sum)
+    unsigned int* ready;       // (NP > 1) [S][Hkv] partitions finished of each (sequence, kv head),
+                               // then [S][Hkv] of its query-head rows merged; both back to 0 after
+                               // the merge, so a plan serves several runs
     unsigned int* status;      // device status word (PA_DEV_* bits)
     int num_seqs;
     int num_heads;
@@ -41,6 +56,8 @@ struct DecodeArgs {
     int partition_blocks;      // blocks per context partition (the smallest the plan may use)
     int adaptive;              // non-zero: the plan may use a multiple of partition_blocks
     int num_ctas;              // CTAs of the persistent kernel
+    int first_wave;            // units the CTAs start on without waiting for the plan: CTA b < first_wave
+                               // takes kv head b % Hkv of partition 0 of sequence b / Hkv (0: none)
     int num_partitions;        // NP = ceil(max_context_len / smallest partition tokens)
     float scale_log2;          // scale * log2(e): logits are kept in base-2 units
     int phases;                // host side: kDecodePlan and/or kDecodeRun
@@ -57,6 +74,7 @@ struct DecodeWorkspace {
     size_t splits;     // 8 * S bytes
     size_t acc;        // 4 * S * Hq * NP * D bytes (0 bytes when NP == 1)
     size_t ml;         // 8 * S * Hq * NP bytes (0 bytes when NP == 1)
+    size_t ready;      // 8 * S * Hq bytes: two counters per (sequence, kv head) (0 bytes when NP == 1)
     size_t total;
 };
 
@@ -70,13 +88,14 @@ inline DecodeWorkspace decode_workspace(size_t S, size_t Hq, size_t D, size_t NP
     w.splits = up(w.list + 8 * S * NP);
     w.acc = up(w.splits + 8 * S);
     w.ml = up(w.acc + (split ? 4 * S * Hq * NP * D : 0));
-    w.total = up(w.ml + (split ? 8 * S * Hq * NP : 0));
+    w.ready = up(w.ml + (split ? 8 * S * Hq * NP : 0));
+    w.total = up(w.ready + (split ? 8 * S * Hq : 0));
     return w;
 }
 
-// One call: the plan kernel, the persistent kernel (tensor cores for bf16 with a group
-// of 2, 4 or 8 query heads per kv head, CUDA cores otherwise) and, when a sequence may
-// span several partitions, the log-sum-exp merge kernel.
+// One call: the plan kernel and the persistent kernel (tensor cores for bf16 with a
+// group of 2, 4 or 8 query heads per kv head, CUDA cores otherwise), which also merges
+// the partitions of split sequences.
 cudaError_t launch_decode(const DecodeArgs& a, pa_dtype dtype, int head_dim, int block_size, int group,
                           cudaStream_t stream);
 bool decode_uses_tensor_cores(pa_dtype dtype, int head_dim, int group);
@@ -86,6 +105,13 @@ bool decode_uses_tensor_cores(pa_dtype dtype, int head_dim, int group);
 // elements, boxes of 64 columns x `box_rows` rows, 128-byte swizzle.
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
 cudaError_t tensor_map(CUtensorMap* out, const void* pool, uint64_t rows, int D, int box_rows);
+
+// Process-unique id of the CUDA context current on this thread (cuCtxGetId), or 0
+// when none is current or the driver lacks the call.  Device addresses of the
+// library's own __device__ variables are cached per device under this id: a device
+// reset re-creates the context (and may reload the module elsewhere), which changes
+// the id, so the address is looked up again.
+unsigned long long current_context_id();
 
 struct ReshapeArgs {
     const void* key;
@@ -130,6 +156,8 @@ struct PrefillArgs {
     int max_blocks_per_seq;
     int num_blocks;
     int block_size;
+    int num_query_tokens;      // rows of q and out: every sequence's rows must lie in [0, this)
+    int max_query_len;         // the launch covers this many rows per sequence
     float scale_log2;
 };
 

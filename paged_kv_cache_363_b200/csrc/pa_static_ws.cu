@@ -12,7 +12,8 @@
 // PA_STATIC_WORKSPACE_BYTES of it until the process exits.  In host code the
 // array's name is only a host-side handle, not a device address, so this file
 // resolves the address once per device (cudaGetSymbolAddress, with that device
-// current) on the first call made on the device, and passes that address on.
+// current) on the first call made on the device, and passes that address on; a
+// device reset makes the next call resolve it again.
 // Nothing else here allocates.
 #include <cuda_runtime.h>
 
@@ -33,8 +34,11 @@ static __device__ __align__(256) unsigned char g_static_workspace[PA_STATIC_WORK
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_ws_ptr[kMaxDevices] = {};
+unsigned long long g_ws_ctx[kMaxDevices] = {};  // context id each cached address belongs to
 
-// Device address of the array on the current device (resolved at the first call).
+// Device address of the array on the current device: resolved at the first call on
+// the device, and again at the first call after a device reset (cudaDeviceReset
+// ends the context; the next one may load the library's module at another address).
 pa_status static_workspace(void** out)
 {
     int dev = 0;
@@ -48,7 +52,8 @@ pa_status static_workspace(void** out)
         return PA_ERR_INVALID;
     }
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_ws_ptr[dev]) {
+    const unsigned long long ctx = pa::current_context_id();
+    if (!g_ws_ptr[dev] || ctx == 0 || g_ws_ctx[dev] != ctx) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_static_workspace);
         if (e != cudaSuccess || !p) {
@@ -56,6 +61,7 @@ pa_status static_workspace(void** out)
             return PA_ERR_CUDA;
         }
         g_ws_ptr[dev] = p;
+        g_ws_ctx[dev] = pa::current_context_id();
     }
     *out = g_ws_ptr[dev];
     return PA_OK;
@@ -71,6 +77,7 @@ pa_status pa_decode_static_workspace(void* out, const void* q, const void* k_cac
                                      int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
                                      int partition_size, pa_dtype dtype, void* stream)
 {
+    pa::CallRange range("pa_decode_static_workspace");
     const size_t need = pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, block_size,
                                                  max_context_len, partition_size);
     if (need > (size_t)PA_STATIC_WORKSPACE_BYTES) {

@@ -471,7 +471,7 @@ def plan_once_timing(batch, stream, dec_bytes, args):
     torch.cuda.synchronize(batch.device)
     return {"run_us": round(res["run"] * 1e3, 3), "run_gbs": round(dec_bytes / (res["run"] * 1e-3) / 1e9, 1),
             "plan_us": round(res["plan"] * 1e3, 3),
-            "note": "one plan per step, one run per layer; the run is the persistent decode kernel (merge included)"}
+            "note": "one plan per step, one run per layer; the run is the persistent decode kernel and the merge"}
 
 
 def e2e_leg(stepper, args, world, dev):
@@ -599,11 +599,11 @@ def bf16_peak():
         return 1590.0, "fallback"
 
 
-def decode_launches(batch):
+def decode_launches(batch, n_part):
     """Kernels one step launches: [copy-on-write copies], append, plan, persistent
-    decode (which also merges the partitions of split sequences)."""
+    decode, [merge of split sequences]."""
     cow = 1 if getattr(batch, "cow_pairs", None) is not None and batch.cow_pairs.numel() else 0
-    return cow + 1 + 2
+    return cow + 1 + 2 + (1 if n_part > 1 else 0)
 
 
 def side_workload(name, args, dev, world, rank):
@@ -640,7 +640,7 @@ def side_workload(name, args, dev, world, rank):
     t = time_decode_steps(batch, stream, steps, args.warmup, dev, world)
     peak, peak_kind = measured_hbm_peak()
     achieved = dec_bytes / (t["dec_avg_max"] * 1e-3) / 1e9
-    roof = {"bound": "hbm", "kernel": "pa_decode (plan kernel + persistent decode kernel, merge included)",
+    roof = {"bound": "hbm", "kernel": "pa_decode (plan kernel + persistent decode kernel + merge)",
             "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "algorithmic_bytes_per_launch": dec_bytes,
             "avg_launch_us": round(t["dec_avg_max"] * 1e3, 3),
@@ -652,7 +652,8 @@ def side_workload(name, args, dev, world, rank):
             "steps": steps, "ms_per_step": round(t["ms_max"] / steps, 5),
             "seqs_per_s": round(world * wl.num_seqs * steps / (t["ms_max"] * 1e-3), 1),
             "config": dict(workload_config(wl, part, batch), l2=l2_note(batch, dec_bytes)),
-            "roofline": roof, "gpu_launches": decode_launches(batch) * steps, "clocks": t["clocks"],
+            "roofline": roof, "gpu_launches": decode_launches(batch, -(-batch.max_context_len // part)) * steps,
+            "clocks": t["clocks"],
             "device_status": t["flags"], "output_finite": t["out_ok"]}
 
 
@@ -762,7 +763,7 @@ def run_gpu(args):
 
     dec_bytes = batch.decode_bytes()
     step_bytes = dec_bytes + batch.append_bytes()
-    launches_per_step = decode_launches(batch)
+    launches_per_step = decode_launches(batch, -(-batch.max_context_len // part))
 
     # ---- device-resident timing
     t = time_decode_steps(batch, stream, args.steps, args.warmup, dev, world)
@@ -799,7 +800,7 @@ def run_gpu(args):
                        parallelism="replicas: one batch per GPU (dp%d)" % world),
         "seqs_per_s": round(world * wl.num_seqs * args.steps / (ms_max * 1e-3), 1),
         "pct_of_peak": round(100.0 * value / peak, 2),
-        "roofline": {"bound": "hbm", "kernel": "pa_decode (plan kernel + persistent decode kernel, merge included)",
+        "roofline": {"bound": "hbm", "kernel": "pa_decode (plan kernel + persistent decode kernel + merge)",
                      "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
                      "traffic": (profile_traffic("decode_persistent_kernel", wl.name)

@@ -81,9 +81,8 @@ typedef enum { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
  * Context-partition length (tokens) that pa_decode uses for these arguments:
  * `partition_size` itself when > 0 (it must be a multiple of block_size, at most
  * 4096), else an automatic choice.  A sequence longer than one partition is
- * split into partitions whose softmax states are merged by log-sum-exp (by the
- * decode kernel's warps that have run out of partitions to attend over, at the
- * end of the call).  Returns a negative pa_status on invalid arguments.
+ * split into partitions whose softmax states are merged by log-sum-exp in a
+ * second kernel.  Returns a negative pa_status on invalid arguments.
  */
 PA_API int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
                              int max_context_len, int partition_size);
@@ -93,8 +92,7 @@ PA_API int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_head
  * num_seqs > 0).  The workspace holds the call's work plan (the (sequence,
  * partition) pairs, longest first, and a work counter) and, when a sequence can
  * span more than one partition, per (sequence, query head, partition) the running
- * max, the softmax sum and the unnormalised head_dim-vector of the partition, and
- * two merge counters per (sequence, query head).
+ * max, the softmax sum and the unnormalised head_dim-vector of the partition.
  */
 PA_API size_t pa_decode_workspace_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
                                 int max_context_len, int partition_size);

@@ -209,7 +209,6 @@ pa_status decode_call(const char* fn, int phases, void* out, const void* q, cons
     if (np > 1) {
         a.ws_acc = reinterpret_cast<float*>(ws + wl.acc);
         a.ws_ml = reinterpret_cast<float*>(ws + wl.ml);
-        a.ready = reinterpret_cast<unsigned int*>(ws + wl.ready);
     }
     unsigned int* status = nullptr;
     st = status_ptr(&status);

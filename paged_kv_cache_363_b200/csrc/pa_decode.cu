@@ -25,10 +25,12 @@
 //  * At the end of a unit each warp leaves its softmax state in shared memory and goes
 //    on with the next unit; the warp that consumed the unit's last tile merges the four
 //    states.  A sequence longer than one partition leaves (max, sum, unnormalised
-//    output) per partition in the workspace; consumer warps left without units at
-//    the tail of the grid merge those partitions by log-sum-exp as they finish, so no
-//    second kernel waits for the whole grid to drain.  The plan and persistent
-//    kernels are chained with programmatic dependent launch.
+//    output) per partition in the workspace and a log-sum-exp merge kernel combines
+//    them.  Plan, persistent and merge kernels are chained with programmatic dependent
+//    launch.
+//  * The first wave of CTAs does not wait for the plan: when the partition length is
+//    fixed, CTA b starts on partition 0 of sequence b / Hkv (kv head b % Hkv), which
+//    the plan lists at position b / Hkv, while the plan kernel still runs.
 //  * Logits are kept in base-2 units (q pre-scaled by scale*log2 e) and exponentials
 //    use exp2f, the reformulation of online softmax by Milakov & Gimelshein (2018).
 //  * Every wait is bounded: a wait that runs out raises PA_DEV_WAIT_TIMEOUT and the
@@ -268,9 +270,8 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
     }
     __syncthreads();
     // A CTA of the first wave starts on its own unit while the plan kernel still runs:
-    // only its unit producer (before its second unit) and its consumers (before the
-    // merge) wait for the plan.  Every other CTA waits here; the plan kernel's list and
-    // counters are visible after the wait.
+    // only its unit producer waits for the plan, before its second unit.  Every other
+    // CTA waits here; the plan kernel's list and counters are visible after the wait.
     const bool early = (int)blockIdx.x < a.first_wave;
     if (!early) pdl_wait_primary();
 
@@ -287,11 +288,7 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
         // pair at list position b / Hkv).
         unsigned nunits = 0;
         uint2 e_first;
-        // count this CTA as started (the tail merge waits on other CTAs only once all have)
-        auto plan_ready = [&]() {
-            nunits = __ldcg(a.plan + 1) * (unsigned)a.num_kv_heads;
-            if (lane == 0 && a.ready) atomicAdd(a.plan + 7, 1u);
-        };
+        auto plan_ready = [&]() { nunits = __ldcg(a.plan + 1) * (unsigned)a.num_kv_heads; };
         if (early) {
             const int s0 = (int)(blockIdx.x / (unsigned)a.num_kv_heads);
             e_first = make_uint2((unsigned)s0 << 11, (unsigned)clamped_context(a, s0, B, false));
@@ -481,13 +478,6 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
                                                first % NCW, lane);
                 __syncwarp();
                 if (lane == 0) {
-                    // the partition's state (all lanes' stores, ordered by the warp barrier)
-                    // is published to the tail merge with a release count, once the plan
-                    // kernel (which zeroes the counts) is done: a first-wave unit may end first
-                    if (split) {
-                        if (early && k == 0) pdl_wait_primary();
-                        red_release_add(a.ready + (size_t)info->s * a.num_kv_heads + info->kvh, 1u);
-                    }
                     mbar_arrive(mg_free);
                     mbar_arrive(&uempty[k % UR]);
                 }
@@ -496,11 +486,6 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
         if (!ok) {
             if (lane == 0) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
             *abort_flag = 1;
-        }
-        // no more units for this CTA: merge finished split sequences meanwhile
-        if (a.ready) {
-            if (early) pdl_wait_primary();  // the plan's split list and counters
-            tail_merge_warp<T, D, G>(a, B, ok, lane, gridDim.x * (unsigned)NCW);
         }
     }
 }
@@ -575,8 +560,10 @@ cudaError_t launch_persistent(const DecodeArgs& a, cudaStream_t stream)
         if (e != cudaSuccess) return e;
     }
     if (!(a.phases & kDecodeRun)) return cudaSuccess;
-    return launch_pdl(decode_persistent_kernel<Cons, BS>, dim3(grid), dim3(P::THREADS), (size_t)P::SMEM, stream,
-                      args, tk, tv);
+    e = launch_pdl(decode_persistent_kernel<Cons, BS>, dim3(grid), dim3(P::THREADS), (size_t)P::SMEM, stream, args,
+                   tk, tv);
+    if (e != cudaSuccess || a.num_partitions <= 1) return e;
+    return launch_merge<typename Cons::T, P::D>(args, BS, stream);
 }
 
 template <typename T, int D, int B>

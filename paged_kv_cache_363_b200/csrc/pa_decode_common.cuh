@@ -1,7 +1,7 @@
 // Pieces of the paged decode path shared by its two consumers (CUDA cores and
 // tensor cores): vector loads, the longest-first work plan, the per-partition
 // epilogue that merges the consumer warps' softmax states, and the log-sum-exp
-// merge of a sequence's context partitions at the tail of the grid.
+// merge of a sequence's context partitions.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -152,11 +152,6 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeArgs a, i
         if (np > 1) {
             atomicAdd(&bucket[pb], np - 1);
             a.split_list[atomicAdd(&s_nsplit, 1)] = make_uint2((unsigned)s, (unsigned)L);
-            // the sequence's merge counters start at zero (every run leaves them there too)
-            for (int k = 0; k < a.num_kv_heads; ++k) {
-                a.ready[(size_t)s * a.num_kv_heads + k] = 0u;
-                a.ready[((size_t)a.num_seqs + s) * a.num_kv_heads + k] = 0u;
-            }
         }
         atomicAdd(&bucket[last], 1);
     }
@@ -180,9 +175,6 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeArgs a, i
         if (lane == 0) {
             a.plan[0] = 0u;                 // work counter
             a.plan[4] = 0u;                 // CTAs that stopped taking units (the last one resets both)
-            a.plan[5] = 0u;                 // merge-row counter
-            a.plan[6] = 0u;                 // consumer warps done merging (the last one resets 5, 6, 7)
-            a.plan[7] = 0u;                 // CTAs started
             a.plan[1] = (unsigned)running;  // number of (sequence, partition) pairs
             a.plan[3] = (unsigned)s_nsplit; // sequences that need the merge
         }
@@ -273,126 +265,112 @@ __device__ __forceinline__ void finish_unit_warp(const DecodeArgs& a, const floa
     }
 }
 
-// Log-sum-exp merge of one (sequence, query head) row of a split sequence:
-// M = max_p m_p, out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p over its np
-// partitions, written to out.  Run by one warp; a lane owns D/32 consecutive columns.
-// The partitions go in chunks of 8 whose column loads are all in flight together,
-// and chunk 0's loads are issued before the maxima are reduced.  The sums run in
-// partition order, so a row's bits do not depend on the warp that merges it.  The
-// partition states are read from L2 (another CTA wrote them).
+// Log-sum-exp merge of the partitions of the split sequences the plan listed:
+// M = max_p m_p, out = sum_p 2^(m_p - M) acc_p / sum_p 2^(m_p - M) l_p, per
+// (sequence, query head) row.  `nwr` warps share a row (1, 2 or 4; a CTA of four
+// warps holds 4 / nwr rows at a time, CTAs striding over the rows).  A lane owns
+// D/32 consecutive columns.  The partitions go in chunks of 8, chunk c to warp
+// c % nwr of the row, whose eight column loads are all in flight together.  The
+// warps' sums are added in warp order, so a row's bits do not depend on the CTA that
+// merges it.
+//
+// The kernel is latency-bound, so its loads are arranged to wait on as little as
+// possible.  The plan lists each split sequence together with its context length,
+// and the first chunk's columns are requested together with the partition maxima.
+// A row then costs two dependent round trips to memory: the list entry, then the
+// partition states.
 template <typename T, int D>
-__device__ __forceinline__ void merge_split_row(const DecodeArgs& a, int s, int h, int np, int lane)
+__global__ void __launch_bounds__(128, 8) decode_merge_kernel(const DecodeArgs a, int block_size, int nwr)
 {
     constexpr int EPL = D / 32;
     constexpr int CH = 8;
-    const size_t row0 = ((size_t)s * a.num_heads + h) * a.num_partitions;
-    const float2* ml = reinterpret_cast<const float2*>(a.ws_ml) + row0;
-    const float* acc = a.ws_acc + row0 * D + lane * EPL;
-    float x[CH][EPL];
-    auto load_chunk = [&](int c) {
+    __shared__ __align__(16) float s_num[4][D];
+    __shared__ float s_den[4];
+    pdl_wait_primary();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int rpc = 4 / nwr;  // rows per CTA at a time
+    const int slot = warp / nwr, sub = warp % nwr;
+    const int H = a.num_heads;
+    const unsigned* plan = a.plan;
+    const int P = (int)__ldg(plan + 2) * block_size;
+    const int rows = (int)__ldg(plan + 3) * H;
+    // the first row's list entry, requested with the counts above (the index stays
+    // inside the list, which has a slot per sequence, whatever the count turns out to be)
+    uint2 e = __ldg(a.split_list + min((int)blockIdx.x * rpc + slot, a.num_seqs * H - 1) / H);
+    for (int r0 = blockIdx.x * rpc; r0 < rows; r0 += gridDim.x * rpc) {
+        const int r = r0 + slot;
+        float num[EPL];
 #pragma unroll
-        for (int u = 0; u < CH; ++u) {
-            // partitions past np repeat the last one; their weight is 0
-            const float* src = acc + (size_t)min(c * CH + u, np - 1) * D;
-            if constexpr (EPL == 4) {
-                const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
-                x[u][0] = v.x; x[u][1] = v.y; x[u][2] = v.z; x[u][3] = v.w;
-            } else {
-                const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
-                x[u][0] = v.x; x[u][1] = v.y;
-            }
-        }
-    };
-    load_chunk(0);
-    float M = -INFINITY;
-    for (int p = lane; p < np; p += 32) M = fmaxf(M, __ldcg(&ml[p].x));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float num[EPL];
-#pragma unroll
-    for (int k = 0; k < EPL; ++k) num[k] = 0.f;
-    float den = 0.f;
-    for (int c = 0; c * CH < np; ++c) {
-        if (c > 0) load_chunk(c);
-        // lane u < 8 holds the weight of partition c * 8 + u
-        const int pw = c * CH + (lane & (CH - 1));
-        float w = 0.f;
-        if (lane < CH && pw < np) {
-            const float2 v = __ldcg(ml + pw);
-            w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
-            den = fmaf(w, v.y, den);
-        }
-#pragma unroll
-        for (int u = 0; u < CH; ++u) {
-            const float wu = __shfl_sync(0xffffffffu, w, u);
-#pragma unroll
-            for (int k = 0; k < EPL; ++k) num[k] = fmaf(wu, x[u][k], num[k]);
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    T* o = static_cast<T*>(a.out) + ((size_t)s * a.num_heads + h) * D + lane * EPL;
-#pragma unroll
-    for (int k = 0; k < EPL; ++k) o[k] = from_f32<T>(num[k] * inv);
-}
-
-// The merge of the split sequences' partitions, run by the persistent kernel's
-// consumer warps once they have no more units (the tail of the grid, where CTAs would
-// otherwise idle), instead of a separate kernel after the whole grid has drained.
-// Rows (split sequence, query head) are claimed from a counter in list order; a row
-// waits until all partitions of its (sequence, kv head) are finished (a release count
-// kept by the warps that wrote the partition states), merges them and writes out.
-//
-// A warp waits on other CTAs only when every CTA of the grid has started: then every
-// unit not yet finished belongs to a running CTA, which never waits on another, so
-// each wait ends.  A warp that sees the grid not yet fully started merges nothing
-// (the CTAs still to start will, the last of them certainly).  The last consumer warp
-// of the grid to finish resets the counters, so a plan serves the next run as is.
-// `ok` is false when this warp gave up earlier: it then only counts itself out.
-template <typename T, int D, int G>
-__device__ __forceinline__ void tail_merge_warp(const DecodeArgs& a, int block_size, bool ok, int lane,
-                                                unsigned total_warps)
-{
-    const unsigned H = (unsigned)a.num_heads;
-    const unsigned Hkv = (unsigned)a.num_kv_heads;
-    unsigned go = 0;
-    if (lane == 0 && ok) go = ld_acquire(a.plan + 7) >= gridDim.x ? 1u : 0u;
-    go = __shfl_sync(0xffffffffu, go, 0);
-    if (go) {
-        const unsigned nrows = __ldcg(a.plan + 3) * H;
-        const int P = (int)__ldcg(a.plan + 2) * block_size;
-        for (;;) {
-            unsigned r = 0;
-            if (lane == 0) r = atomicAdd(a.plan + 5, 1u);
-            r = __shfl_sync(0xffffffffu, r, 0);
-            if (r >= nrows) break;
-            const uint2 e = __ldcg(a.split_list + r / H);
-            const int s = (int)e.x, h = (int)(r % H), L = (int)e.y;
+        for (int k = 0; k < EPL; ++k) num[k] = 0.f;
+        float den = 0.f;
+        if (r < rows) {
+            if (r0 != (int)blockIdx.x * rpc) e = __ldg(a.split_list + r / H);
+            const int L = (int)e.y;
             const int np = (L + P - 1) / P;
-            const size_t key = (size_t)s * Hkv + (unsigned)h / G;
-            unsigned done = 1;
-            if (lane == 0) done = wait_count_bounded(a.ready + key, (unsigned)np) ? 1u : 0u;
-            done = __shfl_sync(0xffffffffu, done, 0);
-            if (!done) {
-                if (lane == 0) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
-                break;
-            }
-            merge_split_row<T, D>(a, s, h, np, lane);
-            if (lane == 0) {
-                // the kv head's last row merged: its counters go back to zero for the next run
-                unsigned int* merged = a.ready + (size_t)a.num_seqs * Hkv + key;
-                if (atomicAdd(merged, 1u) == (unsigned)G - 1) {
-                    a.ready[key] = 0u;
-                    *merged = 0u;
+            const size_t row0 = ((size_t)e.x * H + r % H) * a.num_partitions;
+            const float2* ml = reinterpret_cast<const float2*>(a.ws_ml) + row0;
+            const float* acc = a.ws_acc + row0 * D + lane * EPL;
+            float x[CH][EPL];
+            auto load_chunk = [&](int c) {
+#pragma unroll
+                for (int u = 0; u < CH; ++u) {
+                    // partitions past np repeat the last one; their weight is 0
+                    const float* src = acc + (size_t)min(c * CH + u, np - 1) * D;
+                    if constexpr (EPL == 4) {
+                        const float4 v = __ldg(reinterpret_cast<const float4*>(src));
+                        x[u][0] = v.x; x[u][1] = v.y; x[u][2] = v.z; x[u][3] = v.w;
+                    } else {
+                        const float2 v = __ldg(reinterpret_cast<const float2*>(src));
+                        x[u][0] = v.x; x[u][1] = v.y;
+                    }
+                }
+            };
+            int c = sub;
+            if (c * CH < np) load_chunk(c);
+            float M = -INFINITY;
+            for (int p = lane; p < np; p += 32) M = fmaxf(M, __ldg(&ml[p].x));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+            for (; c * CH < np; c += nwr) {
+                if (c != sub) load_chunk(c);
+                // lane u < 8 holds the weight of partition c * 8 + u
+                const int pw = c * CH + (lane & (CH - 1));
+                float w = 0.f;
+                if (lane < CH && pw < np) {
+                    const float2 v = __ldg(ml + pw);
+                    w = v.x == -INFINITY ? 0.f : exp2f(v.x - M);
+                    den = fmaf(w, v.y, den);
+                }
+#pragma unroll
+                for (int u = 0; u < CH; ++u) {
+                    const float wu = __shfl_sync(0xffffffffu, w, u);
+#pragma unroll
+                    for (int k = 0; k < EPL; ++k) num[k] = fmaf(wu, x[u][k], num[k]);
                 }
             }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
         }
-    }
-    if (lane == 0 && atomicAdd(a.plan + 6, 1u) == total_warps - 1) {
-        a.plan[5] = 0u;
-        a.plan[6] = 0u;
-        a.plan[7] = 0u;
+        if (nwr > 1) {
+#pragma unroll
+            for (int k = 0; k < EPL; ++k) s_num[warp][lane * EPL + k] = num[k];
+            if (lane == 0) s_den[warp] = den;
+            __syncthreads();
+            if (sub == 0) {
+                for (int j = 1; j < nwr; ++j) {
+#pragma unroll
+                    for (int k = 0; k < EPL; ++k) num[k] += s_num[warp + j][lane * EPL + k];
+                    den += s_den[warp + j];
+                }
+            }
+            __syncthreads();
+        }
+        if (r < rows && sub == 0) {
+            const float inv = den > 0.f ? 1.f / den : 0.f;
+            T* o = static_cast<T*>(a.out) + ((size_t)e.x * H + r % H) * D + lane * EPL;
+#pragma unroll
+            for (int k = 0; k < EPL; ++k) o[k] = from_f32<T>(num[k] * inv);
+        }
     }
 }
 
@@ -414,6 +392,20 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename T, int D>
+cudaError_t launch_merge(const DecodeArgs& a, int block_size, cudaStream_t stream)
+{
+    // one warp per row while a row has at most one chunk of 8 partitions, two for two
+    // chunks, else four; up to eight CTAs per SM, striding over the rows of the split sequences
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int nwr = a.num_partitions <= 8 ? 1 : (a.num_partitions <= 16 ? 2 : 4);
+    const long rpc = 4 / nwr;
+    const long ctas = ((long)a.num_seqs * a.num_heads + rpc - 1) / rpc;
+    const unsigned grid = (unsigned)(ctas < 8L * sms ? ctas : 8L * sms);
+    return launch_pdl(decode_merge_kernel<T, D>, dim3(grid), dim3(128), 0, stream, a, block_size, nwr);
 }
 
 }  // namespace

@@ -36,16 +36,12 @@ struct DecodeArgs {
     const int32_t* context_lens;
     unsigned int* plan;        // [0] work counter, [1] (sequence, partition) pairs, [2] blocks per
                                // partition, [3] sequences split into several partitions, [4] CTAs
-                               // that stopped taking units in the current run, [5] merge-row
-                               // counter, [6] consumer warps done with merging, [7] CTAs started
+                               // that stopped taking units in the current run
     uint2* plan_list;          // [S * NP] longest first: {sequence << 11 | partition, context length}
     uint2* split_list;         // [S] the sequences split into several partitions (plan[3] of them):
                                // {sequence, context length}
     float* ws_acc;             // [S][Hq][NP][D] unnormalised partition outputs (NP > 1)
     float* ws_ml;              // [S][Hq][NP][2] (running max in log2 units, softmax sum)
-    unsigned int* ready;       // (NP > 1) [S][Hkv] partitions finished of each (sequence, kv head),
-                               // then [S][Hkv] of its query-head rows merged; both back to 0 after
-                               // the merge, so a plan serves several runs
     unsigned int* status;      // device status word (PA_DEV_* bits)
     int num_seqs;
     int num_heads;
@@ -74,7 +70,6 @@ struct DecodeWorkspace {
     size_t splits;     // 8 * S bytes
     size_t acc;        // 4 * S * Hq * NP * D bytes (0 bytes when NP == 1)
     size_t ml;         // 8 * S * Hq * NP bytes (0 bytes when NP == 1)
-    size_t ready;      // 8 * S * Hq bytes: two counters per (sequence, kv head) (0 bytes when NP == 1)
     size_t total;
 };
 
@@ -88,14 +83,13 @@ inline DecodeWorkspace decode_workspace(size_t S, size_t Hq, size_t D, size_t NP
     w.splits = up(w.list + 8 * S * NP);
     w.acc = up(w.splits + 8 * S);
     w.ml = up(w.acc + (split ? 4 * S * Hq * NP * D : 0));
-    w.ready = up(w.ml + (split ? 8 * S * Hq * NP : 0));
-    w.total = up(w.ready + (split ? 8 * S * Hq : 0));
+    w.total = up(w.ml + (split ? 8 * S * Hq * NP : 0));
     return w;
 }
 
-// One call: the plan kernel and the persistent kernel (tensor cores for bf16 with a
-// group of 2, 4 or 8 query heads per kv head, CUDA cores otherwise), which also merges
-// the partitions of split sequences.
+// One call: the plan kernel, the persistent kernel (tensor cores for bf16 with a group
+// of 2, 4 or 8 query heads per kv head, CUDA cores otherwise) and, when a sequence may
+// span several partitions, the log-sum-exp merge kernel.
 cudaError_t launch_decode(const DecodeArgs& a, pa_dtype dtype, int head_dim, int block_size, int group,
                           cudaStream_t stream);
 bool decode_uses_tensor_cores(pa_dtype dtype, int head_dim, int group);

@@ -13,18 +13,17 @@
 // CTA loads serves all G heads.  It walks the keys in tiles of 64 tokens:
 //   - warp 4 stages Q once and each K and V tile by TMA, one 16-row box per (16-token
 //     run of a physical block, 64 columns), 128-byte swizzle, K in three stages and V
-//     in two, K two tiles ahead of V; lane i looks up and issues box i of the tile;
-//   - warp 5 (one thread) issues S = Q K^T (M=128, N=64, K=128: 8 MMAs) into one of
-//     two S buffers in tensor memory, and O += P V (N=128, K=64: 4 MMAs, A = P from
-//     tensor memory, B operand MN-major) once P is ready, in the order QK(0), QK(1),
-//     PV(0), QK(2), PV(1), ...: the next tile's S is computed while the softmax works
-//     on this one;
+//     in two; lane i looks up and issues box i of the tile;
+//   - warp 5 (one thread) issues S = Q K^T (M=128, N=64, K=128: 8 MMAs) into tensor
+//     memory, and O += P V (N=128, K=64: 4 MMAs, A = P from tensor memory, B operand
+//     MN-major) once P is ready; the next
+//     tile's S is issued as soon as the softmax has read this one, so it overlaps the
+//     softmax;
 //   - warps 0-3 (a thread per row) read S from tensor memory, mask (causal and past
 //     the context), keep the running max in base-2 units, rescale O in tensor memory
 //     only when the max grows by more than 8 (2^8: exact up to rounding, fewer
-//     rescales), write P as bf16 over the first half of the tile's own S buffer (it
-//     has been read), and at the end normalise O and store it.  An S buffer takes the
-//     S of tile j + 2 only after the P.V of tile j has read its P.
+//     rescales), write P as bf16 into tensor memory (two buffers, so the next tile's
+//     P is written while this tile's P.V runs), and at the end normalise O and store it.
 // Two CTAs share an SM (113 KB of shared memory and 256 tensor-memory columns each),
 // so one CTA's softmax overlaps the other's matrix multiplies.
 // Every wait is bounded; on expiry the CTA raises PA_DEV_WAIT_TIMEOUT, drains its own
@@ -52,7 +51,7 @@ constexpr int kQHalf = kM * 128;   // bytes of a 64-column half of the Q tile (1
 constexpr int kKVHalf = kN * 128;  // bytes of a 64-column half of a K or V tile (8 KB)
 constexpr int kBox = 16;           // rows per TMA box of K/V (one 16-token run of a block)
 constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 256;  // S buffers 0..63 and 64..127 (P aliased in each), O: 128..255 (two CTAs fill the 512)
+constexpr uint32_t kTmemCols = 256;  // S: 0..63, P: 64..95 and 96..127, O: 128..255 (two CTAs fill the 512)
 constexpr uint32_t kLazyRescale = 8; // base-2 units
 
 // Tiles, from a 1024-byte aligned base: Q (32 KB), K in three stages and V in two
@@ -67,8 +66,8 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + 2 * kQHalf;
 constexpr int OFF_V = OFF_K + KST * 2 * kKVHalf;
 constexpr int kTiles = OFF_V + VST * 2 * kKVHalf;
-// barriers: q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], s_full[2], p_full, o_done[2], drain
-constexpr int NBAR = 17;
+// barriers: q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full, s_free, p_full, o_done[2], drain
+constexpr int NBAR = 1 + 2 * KST + 2 * VST + 6;
 constexpr int kMisc = 160;          // barriers, TMEM base, abort flag
 constexpr int kSmem = 113 * 1024;
 static_assert(kTiles + 1023 <= kSmem, "tiles fit with any base alignment");
@@ -123,14 +122,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     unsigned char* misc = slack >= (uint32_t)kMisc ? smem_raw : smem + kTiles;
     uint64_t* bars = reinterpret_cast<uint64_t*>(misc);
     uint64_t* q_full = bars + 0;
-    uint64_t* k_full = bars + 1;    // [KST]
-    uint64_t* k_empty = bars + 4;   // [KST]
-    uint64_t* v_full = bars + 7;    // [VST]
-    uint64_t* v_empty = bars + 9;   // [VST]
-    uint64_t* s_full = bars + 11;   // [2]: S of the tiles using S buffer 0 / 1
-    uint64_t* p_full = bars + 13;
-    uint64_t* o_done = bars + 14;   // [2]: P.V of the tiles using P buffer 0 / 1
-    uint64_t* drain = bars + 16;
+    uint64_t* k_full = q_full + 1;        // [KST]
+    uint64_t* k_empty = k_full + KST;     // [KST]
+    uint64_t* v_full = k_empty + KST;     // [VST]
+    uint64_t* v_empty = v_full + VST;     // [VST]
+    uint64_t* s_full = v_empty + VST;
+    uint64_t* s_free = s_full + 1;
+    uint64_t* p_full = s_free + 1;
+    uint64_t* o_done = p_full + 1;        // [2]: P.V of the tiles using P buffer 0 / 1
+    uint64_t* drain = o_done + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + NBAR * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + NBAR * 8 + 8);
     const int warp = threadIdx.x >> 5;
@@ -146,8 +146,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_init(&v_full[i], 1);
             mbar_init(&v_empty[i], 1);
         }
-        mbar_init(&s_full[0], 1);
-        mbar_init(&s_full[1], 1);
+        mbar_init(s_full, 1);
+        mbar_init(s_free, 4);
         mbar_init(p_full, 4);
         mbar_init(&o_done[0], 1);
         mbar_init(&o_done[1], 1);
@@ -160,7 +160,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tmem_s = tmem;       // + 64 * buffer; P of a tile overwrites its S buffer's first 32 columns
+    const uint32_t tmem_s = tmem;
+    const uint32_t tmem_p = tmem + 64;  // + 32 * buffer
     const uint32_t tmem_o = tmem + 128;
 
     if (warp == 4) {
@@ -174,11 +175,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tma_load_3d(smem_u32(smem + OFF_Q + h * kQHalf), &tmap_q, h * 64, kvh * G, q0 + t_lo, q_full, pol);
         }
         const int32_t* table = a.block_tables + (size_t)s * a.max_blocks_per_seq;
-        // K runs two tiles ahead of V: K tile j + 2 is issued (its stage freed by the S of
-        // tile j - 1) before V tile j waits for its stage (freed by the P.V of tile j - 2,
-        // which comes later in the tensor-pipe order), so a V stage that is still busy
-        // never holds back the K loads the next S needs.
-        auto issue = [&](int j, bool is_k) -> bool {
+        bool ok = true;
+        for (int j = 0; j < ntiles && ok; ++j) {
             const int tok0 = j * kN;
             const int nbox = min(kN / kBox, (L - tok0 + kBox - 1) / kBox);
             const int tok = tok0 + lane * kBox;
@@ -192,77 +190,76 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             const int row = (phys * a.num_kv_heads + kvh) * a.block_size + tok % a.block_size;
             const uint32_t tx = (uint32_t)nbox * kBox * 128 * 2;  // both halves of the boxes
-            const int nst = is_k ? KST : VST;
-            const int st = j % nst;
-            uint64_t* full_bar = is_k ? &k_full[st] : &v_full[st];
-            uint64_t* empty_bar = is_k ? &k_empty[st] : &v_empty[st];
-            bool good = true;
+            // K tile j into K stage j % KST, free once S of tile j - KST has run
+            const int ks = j % KST;
             if (lane == 0) {
-                if (j >= nst && !mbar_wait_bounded(empty_bar, ((j / nst) & 1) ^ 1, abort_flag)) good = false;
-                if (good) mbar_arrive_expect_tx(full_bar, tx);
+                if (j >= KST && !mbar_wait_bounded(&k_empty[ks], ((j / KST) & 1) ^ 1, abort_flag)) ok = false;
+                if (ok) mbar_arrive_expect_tx(&k_full[ks], tx);
             }
-            good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
-            if (!good) return false;
-            const int off = is_k ? OFF_K + st * 2 * kKVHalf : OFF_V + st * 2 * kKVHalf;
-            const CUtensorMap* map = is_k ? &tmap_k : &tmap_v;
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
             if (lane < nbox)
                 for (int h = 0; h < 2; ++h)
-                    tma_load_2d(smem_u32(smem + off + h * kKVHalf + lane * kBox * 128), map, h * 64, row, full_bar,
-                                pol);
-            return true;
-        };
-        int nk = 0, nv = 0;  // K and V tiles issued
-        bool ok = issue(0, true);
-        nk += ok;
-        if (ok && ntiles > 1) nk += (ok = issue(1, true));
-        for (int j = 0; j < ntiles && ok; ++j) {
-            if (j + 2 < ntiles) nk += (ok = issue(j + 2, true));
-            if (ok) nv += (ok = issue(j, false));
+                    tma_load_2d(smem_u32(smem + OFF_K + ks * 2 * kKVHalf + h * kKVHalf + lane * kBox * 128), &tmap_k,
+                                h * 64, row, &k_full[ks], pol);
+            // V tile j into V stage j % VST, free once P.V of tile j - VST has run
+            const int vs = j % VST;
+            if (lane == 0) {
+                if (j >= VST && !mbar_wait_bounded(&v_empty[vs], ((j / VST) & 1) ^ 1, abort_flag)) ok = false;
+                if (ok) mbar_arrive_expect_tx(&v_full[vs], tx);
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            if (lane < nbox)
+                for (int h = 0; h < 2; ++h)
+                    tma_load_2d(smem_u32(smem + OFF_V + vs * 2 * kKVHalf + h * kKVHalf + lane * kBox * 128), &tmap_v,
+                                h * 64, row, &v_full[vs], pol);
         }
         if (lane == 0) {
             if (!ok) {
                 atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
                 *abort_flag = 1;
             }
-            // no copy may still be landing in shared memory at exit: the last fills issued
+            // no copy may still be landing in shared memory at exit
             volatile int never = 0;
             if (!mbar_wait_bounded(q_full, 0, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
-            for (int j = max(0, nk - KST); j < nk; ++j)
+            for (int j = max(0, ntiles - KST); j < ntiles; ++j)
                 if (!mbar_wait_bounded(&k_full[j % KST], (j / KST) & 1, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
-            for (int j = max(0, nv - VST); j < nv; ++j)
+            for (int j = max(0, ntiles - VST); j < ntiles; ++j)
                 if (!mbar_wait_bounded(&v_full[j % VST], (j / VST) & 1, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
         }
     } else if (warp == 5) {
         // ---------------- MMA issuer
-        // Tensor-pipe order: QK(0), QK(1), PV(0), QK(2), PV(1), ...: S of tile j + 1 is
-        // computed while the softmax works on tile j.  S(j) goes to S buffer j & 1 and the
-        // softmax writes P(j) over it; QK(j + 2) reuses the buffer only once PV(j), which
-        // reads that P, has completed.
         if (lane == 0) {
             constexpr uint32_t idesc_qk = umma_idesc_bf16(kM, kN, false);
             constexpr uint32_t idesc_pv = umma_idesc_bf16(kM, kD, true);
             const uint32_t sq = smem_u32(smem + OFF_Q), sk = smem_u32(smem + OFF_K), sv = smem_u32(smem + OFF_V);
+            bool ok = mbar_wait_bounded(q_full, 0, abort_flag) && mbar_wait_bounded(&k_full[0], 0, abort_flag);
             auto issue_qk = [&](int j) {
                 const uint32_t kb = sk + (j % KST) * 2 * kKVHalf;
 #pragma unroll
                 for (int k = 0; k < kD / 16; ++k) {
                     const uint32_t kk = (k & 3) * 32;
-                    umma_bf16_ss(tmem_s + (j & 1) * 64, umma_desc_sw128(sq + (k >> 2) * kQHalf + kk, 16, 1024),
+                    umma_bf16_ss(tmem_s, umma_desc_sw128(sq + (k >> 2) * kQHalf + kk, 16, 1024),
                                  umma_desc_sw128(kb + (k >> 2) * kKVHalf + kk, 16, 1024), idesc_qk, k > 0 ? 1u : 0u);
                 }
-                umma_commit(&s_full[j & 1]);
+                umma_commit(s_full);
                 umma_commit(&k_empty[j % KST]);
             };
-            bool ok = mbar_wait_bounded(q_full, 0, abort_flag);
-            for (int j = 0; j < 2 && j < ntiles && ok; ++j) {
-                if (!mbar_wait_bounded(&k_full[j % KST], (j / KST) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
+            if (ok) {
                 tc_fence_after_sync();
-                issue_qk(j);
+                issue_qk(0);
             }
             for (int j = 0; j < ntiles && ok; ++j) {
+                if (j + 1 < ntiles) {
+                    if (!mbar_wait_bounded(&k_full[(j + 1) % KST], ((j + 1) / KST) & 1, abort_flag) ||
+                        !mbar_wait_bounded(s_free, j & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    issue_qk(j + 1);
+                }
                 if (!mbar_wait_bounded(p_full, j & 1, abort_flag) ||
                     !mbar_wait_bounded(&v_full[j % VST], (j / VST) & 1, abort_flag)) {
                     ok = false;
@@ -272,21 +269,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const uint32_t vb = sv + (j % VST) * 2 * kKVHalf;
 #pragma unroll
                 for (int k = 0; k < kN / 16; ++k) {
-                    umma_bf16_ts(tmem_o, tmem_s + (j & 1) * 64 + k * 8,
+                    umma_bf16_ts(tmem_o, tmem_p + (j & 1) * 32 + k * 8,
                                  umma_desc_sw128(vb + k * 16 * 128, kKVHalf, 1024), idesc_pv,
                                  (j > 0 || k > 0) ? 1u : 0u);
                 }
                 umma_commit(&o_done[j & 1]);
                 umma_commit(&v_empty[j % VST]);
-                if (j + 2 < ntiles) {
-                    if (!mbar_wait_bounded(&k_full[(j + 2) % KST], ((j + 2) / KST) & 1, abort_flag) ||
-                        !mbar_wait_bounded(&o_done[j & 1], (j >> 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after_sync();
-                    issue_qk(j + 2);
-                }
             }
             if (!ok) {
                 atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
@@ -310,17 +298,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < ntiles; ++j) {
-            if (!mbar_wait_warp(&s_full[j & 1], (j >> 1) & 1, abort_flag)) {
+            if (!mbar_wait_warp(s_full, j & 1, abort_flag)) {
                 ok = false;
                 break;
             }
             tc_fence_after_sync();
-            const uint32_t tmem_sj = tmem_s + (j & 1) * 64;
             constexpr int NC = kN / 32;  // 32-column chunks of the S row
             uint32_t sr[NC][32];
 #pragma unroll
-            for (int c = 0; c < NC; ++c) tmem_ld32(tmem_sj + lane_base + c * 32, sr[c]);
+            for (int c = 0; c < NC; ++c) tmem_ld32(tmem_s + lane_base + c * 32, sr[c]);
             tmem_wait_ld();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_free);
             const int kv0 = j * kN;
             // Work on the raw logits: the scale and the max subtraction fold into one FMA
             // below.  Keys past a row's limit become the value that scales to -inf; only
@@ -374,10 +364,13 @@ __global__ void __launch_bounds__(kThreads, 2)
             const bool rescale = m_used != -INFINITY && m_new > m_used + (float)kLazyRescale;
             // the whole warp takes the O round trip when any of its rows needs it
             const bool rescale_warp = __any_sync(0xffffffffu, rescale) != 0;
-            // P(j) goes over S(j) in S buffer j & 1, whose previous P was read by the P.V of
-            // tile j - 2, complete before S(j) was computed.  O is stable for a rescale once
-            // the P.V of tile j - 1 has finished (each buffer has its own barrier, whose
-            // next phase is never more than one ahead of the wait).
+            // P buffer j & 1 is free once the P.V of tile j - 2 has finished; O is stable
+            // for a rescale once the P.V of tile j - 1 has (each buffer has its own
+            // barrier, whose next phase is never more than one ahead of the wait)
+            if (j >= 2 && !mbar_wait_warp(&o_done[j & 1], ((j - 2) >> 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
             if (rescale_warp && j >= 1 && !mbar_wait_warp(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag)) {
                 ok = false;
                 break;
@@ -439,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
             }
             const float rowsum = (rs0 + rs1) + (rs2 + rs3);
-            tmem_st32(tmem_sj + lane_base, w);
+            tmem_st32(tmem_p + (j & 1) * 32 + lane_base, w);
             tmem_wait_st();
             l += rowsum;
             // keys past the context in this tile: zero their V rows (0-weights must meet finite values)

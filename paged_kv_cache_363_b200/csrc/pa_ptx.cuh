@@ -1,7 +1,6 @@
 // Inline-PTX helpers for sm_100a: mbarriers, 1-D bulk global->shared copies (the
-// TMA engine's untiled form; no tensor map, one CTA's own copy), bounded waits,
-// release/acquire counters in global memory, and programmatic-dependent-launch
-// controls.
+// TMA engine's untiled form; no tensor map, one CTA's own copy), bounded waits, and
+// programmatic-dependent-launch controls.
 #pragma once
 
 #include <cstdint>
@@ -82,34 +81,6 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, v
 {
     const bool ok = mbar_wait_bounded(bar, parity, abort);
     return __all_sync(0xffffffffu, ok) != 0;
-}
-
-// Release increment of a counter in global memory (device scope): every store this
-// thread made, or observed through a barrier, before it is visible to a thread that
-// reads the new count with an acquire load.
-__device__ __forceinline__ void red_release_add(unsigned int* p, unsigned int v)
-{
-    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ unsigned int ld_acquire(const unsigned int* p)
-{
-    unsigned int v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Waits until the counter at p reaches `target` (acquire).  Returns false if it did
-// not within kWaitTimeoutNs.
-__device__ __forceinline__ bool wait_count_bounded(const unsigned int* p, unsigned int target)
-{
-    if (ld_acquire(p) >= target) return true;
-    const unsigned long long t0 = globaltimer_ns();
-    while (true) {
-        __nanosleep(64);
-        if (ld_acquire(p) >= target) return true;
-        if (globaltimer_ns() - t0 > kWaitTimeoutNs) return false;
-    }
 }
 
 // 1-D bulk copy global -> shared, completion signalled on `bar` as tx bytes.

@@ -110,13 +110,11 @@ def test_partition_and_workspace_sizes():
     up = lambda x: (x + 255) // 256 * 256
     # one partition: only the work plan (32-byte header, one 8-byte entry and an 8-byte split slot per sequence)
     assert pa.pa_decode_workspace_size(4, 4, 4, 64, 16, 100, 512) == up(up(32 + 8 * 4) + 8 * 4)
-    # plan (S * NP entries, S split slots), then S * Hq * NP * D floats, S * Hq * NP (max, sum) pairs
-    # and two merge counters per (sequence, head)
+    # plan (S * NP entries, S split slots), then S * Hq * NP * D floats and S * Hq * NP (max, sum) pairs
     S, Hq, Hkv, D, NP = 8, 32, 8, 128, 64
     acc = up(up(32 + 8 * S * NP) + 8 * S)
     ml = up(acc + 4 * S * Hq * NP * D)
-    ready = up(ml + 8 * S * Hq * NP)
-    assert pa.pa_decode_workspace_size(S, Hq, Hkv, D, 32, 32768, 512) == up(ready + 8 * S * Hq)
+    assert pa.pa_decode_workspace_size(S, Hq, Hkv, D, 32, 32768, 512) == up(ml + 8 * S * Hq * NP)
     assert pa.pa_decode_workspace_size(0, 32, 8, 128, 32, 32768, 512) == 0
 
 

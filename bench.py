@@ -630,6 +630,8 @@ def side_workload(name, args, dev, world, rank):
                            "context_tokens": int(wl.context_lens.sum()), "seed": wl.seed},
                 "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel", "achieved": round(achieved, 2),
                              "peak": peak, "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                             "traffic": (profile_traffic("prefill_tc_kernel", wl.name, PREFILL_SOURCES)
+                                         if wl.seed == 0 else None),
                              "algorithmic_flops_per_launch": flops, "avg_launch_us": round(t["avg_max"] * 1e3, 3)},
                 "gpu_launches": steps, "clocks": t["clocks"], "device_status": t["flags"],
                 "output_finite": t["out_ok"]}
@@ -642,8 +644,9 @@ def side_workload(name, args, dev, world, rank):
     achieved = dec_bytes / (t["dec_avg_max"] * 1e-3) / 1e9
     roof = {"bound": "hbm", "kernel": "pa_decode (plan kernel + persistent decode kernel + merge)",
             "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "algorithmic_bytes_per_launch": dec_bytes,
-            "avg_launch_us": round(t["dec_avg_max"] * 1e3, 3),
+            "frac": round(achieved / peak, 4),
+            "traffic": profile_traffic("decode_persistent_kernel", wl.name) if wl.seed == 0 else None,
+            "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_us": round(t["dec_avg_max"] * 1e3, 3),
             "launch_us_p10_p50_p90": [round(float(np.percentile(t["dec_ms"], q)) * 1e3, 3) for q in (10, 50, 90)]}
     if isinstance(wl, W.CowWorkload):
         roof["note"] = ("logical bytes: the 4 streams of a prompt share its blocks, which are re-read from L2, "

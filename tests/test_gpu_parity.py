@@ -426,3 +426,55 @@ def test_plan_once_then_run_per_layer(pa, runner, wid, part):
 
 def bits_t(t):
     return t.view(torch.int32) if t.dtype == torch.float32 else t.view(torch.int16)
+
+
+@pytest.mark.parametrize("G", [1, 4])
+def test_adaptive_partition_grows_without_first_wave(pa, G):
+    """A batch of 96 sequences of 12-16k tokens (1.36M tokens, more than four 1024-token
+    partitions per CTA): the automatic partition grows in the plan kernel.  No CTA may
+    then start before the plan (the first wave needs a partition length the host can
+    fix), so this runs the path in which every CTA waits for the plan.  Every row matches
+    the oracle, and a second run from the same plan gives the same bits."""
+    S, Hkv, D, B = 96, 2, 128, 16
+    Hq = Hkv * G
+    rng = np.random.default_rng(40 + G)
+    lens = rng.integers(12000, 16385, size=S).astype(np.int32)
+    nblk = (lens + B - 1) // B
+    NB = int(nblk.sum()) + 7
+    perm = rng.permutation(NB).astype(np.int32)
+    tables = np.full((S, int(nblk.max())), -1, np.int32)
+    pos = 0
+    for s in range(S):
+        tables[s, :nblk[s]] = perm[pos:pos + nblk[s]]
+        pos += nblk[s]
+    g = torch.Generator(device="cuda").manual_seed(G)
+    k = torch.randn((NB, Hkv, B, D), generator=g, device="cuda").to(torch.bfloat16)
+    v = torch.randn((NB, Hkv, B, D), generator=g, device="cuda").to(torch.bfloat16)
+    q = torch.randn((S, Hq, D), generator=g, device="cuda").to(torch.bfloat16)
+    t_d = torch.from_numpy(tables).cuda()
+    l_d = torch.from_numpy(lens).cuda()
+    maxL = int(lens.max())
+    ws = torch.zeros(pa.pa_decode_workspace_size(S, Hq, Hkv, D, B, maxL, 0) + 16, dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(q)
+    pa.pa_decode(out, q, k, v, t_d, l_d, maxL, D ** -0.5, 0, ws)
+    torch.cuda.synchronize()
+    _status_clean(pa)
+    # the plan's partition (blocks per partition, third word of the work plan) grew past the smallest
+    pb = int(ws[8:12].cpu().view(torch.int32).item())
+    assert pb * B > pa.pa_decode_partition_size(S, Hq, Hkv, D, B, maxL, 0)
+    again = torch.empty_like(q)
+    pa.pa_decode_run(again, q, k, v, t_d, l_d, maxL, D ** -0.5, ws, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(bits_t(again), bits_t(out))
+    kc, vc = k.float().cpu().numpy(), v.float().cpu().numpy()
+
+    def rows(s):
+        blk = tables[s, :nblk[s]]
+        kk = kc[blk].transpose(0, 2, 1, 3).reshape(-1, Hkv, D)[:lens[s]]
+        vv = vc[blk].transpose(0, 2, 1, 3).reshape(-1, Hkv, D)[:lens[s]]
+        return kk, vv
+
+    ref = oracle_logical_all(q.float().cpu().numpy(), rows, B, D ** -0.5)
+    err = max_abs(out.float().cpu().numpy(), ref)
+    report_error("adaptive partition, G=%d (96 x 12-16k tokens)" % G, err, S * Hq)
+    assert err <= TOL["bf16"], err

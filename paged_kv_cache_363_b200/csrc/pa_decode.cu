@@ -350,7 +350,11 @@ __global__ void __launch_bounds__(Persist<Cons, BS>::THREADS, 2)
             const int b0 = part * pb;
             const int nb = max(0, min(pb, nblk_seq - b0));
             int* tab = slot_table(k);
-            for (int i = lane; i < nb; i += 32)
+            // A first-wave unit reads its table slice (partition 0: the row's first pb
+            // entries, all inside the row) in the same trip to memory as its context
+            // length, not after it; entries past the context are loaded but never used.
+            const int nload = (k == 0 && early) ? min(pb, a.max_blocks_per_seq) : nb;
+            for (int i = lane; i < nload; i += 32)
                 tab[i] = __ldg(a.block_tables + (size_t)s * a.max_blocks_per_seq + b0 + i);
             if (lane == 0) {
                 info->s = s;

@@ -7,9 +7,6 @@ copies (when the step has any), the slot-mapped append of every sequence's new
 token, and paged decode attention over the block tables.  Inputs sit in HBM when
 the timed region starts; the KV bytes a step reads (about 1.2 GB for the default
 workload) are far larger than the 126 MB L2, so no flush is needed between steps.
-The append and the decode call of each step are replayed from CUDA graphs captured
-once (the same kernels and arguments, without launch gaps); the line also reports
-the same steps launched kernel by kernel ("plain_launch").
 
 The metric is throughput in GB/s of algorithmic bytes: the K and V rows of every
 context token, q and the output, block tables and lengths, plus the appended rows.
@@ -527,32 +524,7 @@ def make_run(name, seed, dev, overrides=None, partition=None):
     return wl, values, runner.make_batch(wl, dev, values=values)
 
 
-def decode_step_calls(batch, stream, dev, graph):
-    """The two calls of a device-resident step, (append, decode), each a callable that
-    launches on `stream`.  With graph=True each is captured once as a CUDA graph and
-    replayed: the same kernels with the same arguments, without the launch gaps between
-    dependent kernels that plain launches leave."""
-    import torch
-
-    if not graph:
-        return (lambda: batch.append(stream)), (lambda: batch.decode(stream=stream))
-    batch.workspace_for(batch.partition_size)  # sized before capture: nothing allocates inside
-    torch.cuda.synchronize(dev)
-    cap = torch.cuda.Stream(dev)
-    g_app, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_app, stream=cap, capture_error_mode="relaxed"):
-        batch.append(cap)
-    with torch.cuda.graph(g_dec, stream=cap, capture_error_mode="relaxed"):
-        batch.decode(stream=cap)
-    torch.cuda.synchronize(dev)
-
-    def replay(g):
-        with torch.cuda.stream(stream):
-            g.replay()
-    return (lambda: replay(g_app)), (lambda: replay(g_dec))
-
-
-def time_decode_steps(batch, stream, steps, warmup, dev, world, graph=True):
+def time_decode_steps(batch, stream, steps, warmup, dev, world):
     """Device-resident decode steps: `warmup` untimed, then `steps` timed between a
     barrier + synchronize on both sides, each step's decode call bracketed by its own
     CUDA events on `stream`.  Whole-step and decode-call times are max over ranks."""
@@ -560,10 +532,8 @@ def time_decode_steps(batch, stream, steps, warmup, dev, world, graph=True):
     import torch.distributed as dist
     from paged_kv_cache_363_b200 import pa
 
-    append, decode = decode_step_calls(batch, stream, dev, graph)
     for _ in range(warmup):
-        append()
-        decode()
+        batch.step(stream)
     torch.cuda.synchronize(dev)
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
@@ -575,9 +545,9 @@ def time_decode_steps(batch, stream, steps, warmup, dev, world, graph=True):
     with ClockSampler(dev.index) as clk:
         t_start.record(stream)
         for k in range(steps):
-            append()
+            batch.append(stream)
             ev_s[k].record(stream)
-            decode()
+            batch.decode(stream=stream)
             ev_e[k].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize(dev)
@@ -798,13 +768,10 @@ def run_gpu(args):
     step_bytes = dec_bytes + batch.append_bytes()
     launches_per_step = decode_launches(batch, -(-batch.max_context_len // part))
 
-    # ---- device-resident timing: each step's append and decode call replayed from CUDA
-    # graphs; the same steps with plain launches are reported beside it
+    # ---- device-resident timing
     t = time_decode_steps(batch, stream, args.steps, args.warmup, dev, world)
     ms_max, dec_ms, dec_avg_max = t["ms_max"], t["dec_ms"], t["dec_avg_max"]
     out_ok, flags = t["out_ok"], t["flags"]
-    tp = time_decode_steps(batch, stream, args.steps, args.warmup, dev, world, graph=False)
-    out_ok, flags = out_ok and tp["out_ok"], flags | tp["flags"]
 
     e2e = None
     if not args.skip_e2e:
@@ -843,11 +810,6 @@ def run_gpu(args):
                                  if profiled_config(args) else None),
                      "algorithmic_bytes_per_launch": dec_bytes, "avg_launch_us": round(dec_avg_max * 1e3, 3),
                      "launch_us_p10_p50_p90": [round(float(np.percentile(dec_ms, q)) * 1e3, 3) for q in (10, 50, 90)]},
-        "launch": "each step's append and decode call replayed from a CUDA graph (plain_launch: the same steps "
-                  "launched one kernel at a time)",
-        "plain_launch": {"value": round(world * step_bytes * args.steps / (tp["ms_max"] * 1e-3) / 1e9, 2),
-                         "ms_per_step": round(tp["ms_max"] / args.steps, 5),
-                         "decode_us": round(tp["dec_avg_max"] * 1e3, 3)},
         "companions": companions,
         "plan_once": plan_once,
         "e2e": e2e,

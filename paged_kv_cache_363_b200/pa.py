@@ -368,10 +368,12 @@ class Allocator:
         if not h:
             raise PAError(PA_ERR_INVALID, "pa_alloc_create")
         self._h = ctypes.c_void_p(h)
+        # held here: at interpreter exit the module's globals may already be gone when __del__ runs
+        self._destroy = lib.pa_alloc_destroy
 
     def close(self):
         if getattr(self, "_h", None):
-            lib.pa_alloc_destroy(self._h)
+            self._destroy(self._h)
             self._h = None
 
     def __del__(self):

@@ -268,13 +268,34 @@ PA_API pa_status pa_selftest_bounded_wait(uint64_t* waited_ns, void* stream);
  * n_s > max_query_len, n_s > context_lens[s], or a context beyond its table row
  * raises PA_DEV_BAD_CONTEXT and is skipped whole (its output rows untouched).  bf16 only,
  * head_dim 128, num_heads / num_kv_heads in {1, 2, 4, 8} (else PA_ERR_UNSUPPORTED).
- * With every n_s = 1 this is pa_decode.  No workspace.  Asynchronous on stream.
+ * With every n_s = 1 this is pa_decode.  No workspace: the grid has one CTA per work
+ * item (pa_prefill_ws below is the faster form).  Asynchronous on stream.
  */
 PA_API pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* block_tables, const int32_t* context_lens, const int32_t* q_start,
                             int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
                             int max_blocks_per_seq, int num_blocks, int num_query_tokens, int max_query_len,
                             float scale, pa_dtype dtype, void* stream);
+
+/* Bytes of device workspace pa_prefill_ws needs (a fixed size). */
+PA_API size_t pa_prefill_workspace_size(void);
+
+/*
+ * pa_prefill with a workspace: the same computation, arguments and checks, run by a
+ * grid of one CTA per SM that hands out the (sequence, kv head, query-tile pair) work
+ * items from a counter in the workspace, longest first, so that a CTA which finishes
+ * early takes more and each CTA's next item starts while its last one ends.
+ *   workspace  device scratch of at least pa_prefill_workspace_size() bytes, 16-byte
+ *              aligned; no initial contents are needed (the call zeroes its counter on
+ *              `stream` first).  Calls that share a workspace must be ordered on one
+ *              stream.
+ * A null or short workspace returns PA_ERR_INVALID.  Asynchronous on stream.
+ */
+PA_API pa_status pa_prefill_ws(void* out, const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* block_tables, const int32_t* context_lens, const int32_t* q_start,
+                               int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                               int max_blocks_per_seq, int num_blocks, int num_query_tokens, int max_query_len,
+                               float scale, void* workspace, size_t workspace_bytes, pa_dtype dtype, void* stream);
 
 /*
  * Whole-block copies from one pool to another ([FSAH] "Engineering Limitations":

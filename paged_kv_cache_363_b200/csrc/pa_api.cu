@@ -411,12 +411,14 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapp
     return PA_OK;
 }
 
-pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+static pa_status prefill_impl(const char* name, void* out, const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_tables,
                      const int32_t* context_lens, const int32_t* q_start, int num_seqs, int num_heads,
                      int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
-                     int num_query_tokens, int max_query_len, float scale, pa_dtype dtype, void* stream)
+                     int num_query_tokens, int max_query_len, float scale, pa_dtype dtype, void* stream,
+                              void* workspace, size_t workspace_bytes)
 {
-    pa::CallRange range("pa_prefill");
+    pa::CallRange range(name);
     pa_status st = check_common("pa_prefill", num_kv_heads, head_dim, block_size, num_blocks, dtype);
     if (st != PA_OK) return st;
     if (dtype != PA_DTYPE_BF16 || head_dim != 128) {
@@ -433,6 +435,10 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
     if (group != 1 && group != 2 && group != 4 && group != 8) {
         set_error("pa_prefill: num_heads / num_kv_heads must be 1, 2, 4 or 8");
         return PA_ERR_UNSUPPORTED;
+    }
+    if (workspace && (workspace_bytes < pa_prefill_workspace_size() || !aligned(workspace, 16))) {
+        set_error("pa_prefill_ws: workspace smaller than pa_prefill_workspace_size() or not 16-byte aligned");
+        return PA_ERR_INVALID;
     }
     if (num_seqs == 0 || num_query_tokens == 0) return PA_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !q_start) {
@@ -459,6 +465,7 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
     a.context_lens = context_lens;
     a.q_start = q_start;
     a.status = status;
+    a.sched = static_cast<unsigned int*>(workspace);
     a.num_seqs = num_seqs;
     a.num_heads = num_heads;
     a.num_kv_heads = num_kv_heads;
@@ -468,10 +475,42 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
     a.num_query_tokens = num_query_tokens;
     a.max_query_len = max_query_len;
     a.scale_log2 = scale * 1.4426950408889634f;
+    if (workspace) {
+        // the item counter starts at zero on every call, in stream order
+        const cudaError_t z = cudaMemsetAsync(workspace, 0, sizeof(unsigned int), static_cast<cudaStream_t>(stream));
+        if (z != cudaSuccess) return cuda_fail("pa_prefill_ws counter reset", z);
+    }
     const cudaError_t e =
         launch_prefill(a, group, num_query_tokens, max_query_len, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail("pa_prefill launch", e);
     return PA_OK;
+}
+
+size_t pa_prefill_workspace_size(void) { return 256; }
+
+pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                     const int32_t* context_lens, const int32_t* q_start, int num_seqs, int num_heads,
+                     int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, int num_blocks,
+                     int num_query_tokens, int max_query_len, float scale, pa_dtype dtype, void* stream)
+{
+    return prefill_impl("pa_prefill", out, q, k_cache, v_cache, block_tables, context_lens, q_start, num_seqs,
+                        num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                        num_query_tokens, max_query_len, scale, dtype, stream, nullptr, 0);
+}
+
+pa_status pa_prefill_ws(void* out, const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* block_tables, const int32_t* context_lens, const int32_t* q_start,
+                        int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                        int max_blocks_per_seq, int num_blocks, int num_query_tokens, int max_query_len, float scale,
+                        void* workspace, size_t workspace_bytes, pa_dtype dtype, void* stream)
+{
+    if (!workspace) {
+        set_error("pa_prefill_ws: null workspace");
+        return PA_ERR_INVALID;
+    }
+    return prefill_impl("pa_prefill_ws", out, q, k_cache, v_cache, block_tables, context_lens, q_start, num_seqs,
+                        num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                        num_query_tokens, max_query_len, scale, dtype, stream, workspace, workspace_bytes);
 }
 
 // Address a kernel can use for p: device memory as is, pinned (page-locked) host

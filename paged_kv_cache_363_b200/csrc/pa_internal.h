@@ -144,6 +144,7 @@ struct PrefillArgs {
     const int32_t* context_lens;
     const int32_t* q_start;    // [S + 1] query rows of each sequence
     unsigned int* status;
+    unsigned int* sched;       // item counter (zero at launch) for a grid of one CTA per SM; null: one item per CTA
     int num_seqs;
     int num_heads;
     int num_kv_heads;

@@ -8,13 +8,17 @@
 // section 3: the prompt's blocks are assigned when it is processed; "PagedAttention
 // Paper Breakdown", section 2: token t lives at slot T[t / B] * B + t % B).
 //
-// A CTA owns one (sequence, kv head) and two query tiles A and B of 128 rows each.  A
-// tile's rows are T query tokens x G query heads of the kv head's group (T = 128 / G),
-// so every K/V byte the CTA loads serves both tiles and all G heads.  It walks the keys
-// in tiles of 128 tokens:
-//   - warp 16 stages both Q tiles once and each K and V tile by TMA, one 16-row box per
-//     (16-token run of a physical block, 64 columns), 128-byte swizzle, K and V in two
-//     32 KB stages each; lane i looks up and issues box i of the tile;
+// A work item is one (sequence, kv head) and two query tiles A and B of 128 rows each.
+// A tile's rows are T query tokens x G query heads of the kv head's group (T = 128 / G),
+// so every K/V byte loaded serves both tiles and all G heads.  With a workspace
+// (pa_prefill_ws) one CTA per SM claims items from a counter, last query tokens first,
+// and starts an item's Q load and first S while its previous item ends; without one
+// (pa_prefill) CTA b runs item b alone.  An item walks the keys in tiles of 128 tokens:
+//   - warp 16 claims the items and passes them, with their geometry, through a ring of
+//     two shared-memory slots; it stages both Q tiles once per item and each K and V
+//     tile by TMA, one 16-row box per (16-token run of a physical block, 64 columns),
+//     128-byte swizzle, K and V in two 32 KB stages each (the rings run on across
+//     items); lane i looks up and issues box i of the tile;
 //   - warp 17 (one thread) issues, per query tile, S = Q K^T (M=128, N=128, K=128:
 //     8 MMAs) into tensor memory and O += P V (N=128, K=128: 8 MMAs, A = P from tensor
 //     memory, B operand MN-major).  The order is fixed, P.V_A(j), S_A(j+1), P.V_B(j),
@@ -29,7 +33,8 @@
 //     significant bits, more than P's 8).  P goes as bf16 over the first 64 columns of
 //     S; at the end the halves add up their row sums and store O.
 // One CTA per SM: 197 KB of shared memory, all 512 tensor-memory columns (per query
-// tile S 128 + O 128).
+// tile S 128 + O 128).  A tile's O is taken by its next item only after the softmax has
+// read it out, and its S only after the previous P.V.
 // Every wait is bounded; on expiry the CTA raises PA_DEV_WAIT_TIMEOUT, drains its own
 // copies and MMAs, frees its tensor memory and returns.
 #include <cuda.h>
@@ -38,6 +43,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -71,11 +77,14 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + kQT * 2 * kQHalf;
 constexpr int OFF_V = OFF_K + KST * 2 * kKVHalf;
 constexpr int kTiles = OFF_V + VST * 2 * kKVHalf;
-// barriers: q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], per query tile
-// {s_full, p_full, o_done}, drain
-constexpr int NBAR = 1 + 2 * KST + 2 * VST + kQT * 3 + 1;
+constexpr int IR = 2;  // item ring: the item in work and the next
+// barriers: q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], per query tile
+// {s_full, p_full, o_done, o_free}, drain, it_full[IR], it_empty[IR]
+constexpr int NBAR = 2 + 2 * KST + 2 * VST + kQT * 4 + 1 + 2 * IR;
 constexpr int kXch = 2 * kQT * 2 * 128 * 4;  // partial row maxima (and sums), [tile parity][qt][half][row]
-constexpr int kMisc = NBAR * 8 + 16 + kXch;
+// after the barriers: TMEM address and abort flag (16 bytes), the item slots, the exchange buffer
+constexpr int kSlotInts = 16;
+constexpr int kMisc = NBAR * 8 + 16 + 4 * IR * kSlotInts + kXch;
 constexpr int kSmem = (kTiles + 1023 + kMisc + 15) / 16 * 16;
 static_assert(kSmem <= 227 * 1024, "one CTA per SM");
 
@@ -128,49 +137,87 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+// One work item: query tokens [t_lo0, t_lo0 + 2T) of sequence s (two query tiles of T tokens x G heads) for
+// kv head kvh.  Items are numbered with the last query tokens of every (sequence, kv head) first, since those
+// see the most keys.  With a counter (a.sched) a grid of one CTA per SM claims them in that order, so a CTA
+// that finishes early takes more; without one, CTA b takes item b alone.  The producer warp claims the items
+// and hands them to the MMA thread and the softmax warps through a ring of IR slots in shared memory.
+struct Item {
+    int s, kvh, pair, q0, n, L, t_lo0, nqt, nA, nB, ntiles;
+    bool bad;
+};
+
+// An item's geometry in its ring slot (after the item and ring-position words), written by the producer so
+// that the MMA thread and the softmax warps read it from shared memory instead of global memory.
+__device__ __forceinline__ void put_item(int* p, const Item& it)
+{
+    p[2] = it.s; p[3] = it.kvh; p[4] = it.pair; p[5] = it.q0; p[6] = it.n; p[7] = it.L; p[8] = it.t_lo0;
+    p[9] = it.nqt; p[10] = it.nA; p[11] = it.nB; p[12] = it.ntiles;
+}
+__device__ __forceinline__ void get_item(const volatile int* p, Item& it)
+{
+    it.s = p[2]; it.kvh = p[3]; it.pair = p[4]; it.q0 = p[5]; it.n = p[6]; it.L = p[7]; it.t_lo0 = p[8];
+    it.nqt = p[9]; it.nA = p[10]; it.nB = p[11]; it.ntiles = p[12]; it.bad = false;
+}
+
+template <int G>
+__device__ __forceinline__ bool item_geom(const PrefillArgs& a, int npairs, int item, Item& it)
+{
+    constexpr int T = kM / G;
+    const int per = a.num_seqs * a.num_kv_heads;
+    it.pair = npairs - 1 - item / per;
+    const int rem = item % per;
+    it.s = rem / a.num_kv_heads;
+    it.kvh = rem % a.num_kv_heads;
+    it.q0 = __ldg(a.q_start + it.s);
+    const int q1 = __ldg(a.q_start + it.s + 1);
+    it.n = q1 - it.q0;
+    it.L = __ldg(a.context_lens + it.s);
+    const int Lcap = a.max_blocks_per_seq * a.block_size;
+    it.bad = it.q0 < 0 || q1 > a.num_query_tokens || it.n < 0 || it.n > a.max_query_len || it.L < it.n ||
+             it.L > Lcap;
+    it.t_lo0 = it.pair * kQT * T;
+    if (it.bad || it.t_lo0 >= it.n) return false;
+    it.nqt = it.t_lo0 + T < it.n ? 2 : 1;
+    it.nA = (it.L - it.n + min(it.n, it.t_lo0 + T) - 1) / kN + 1;
+    it.nB = it.nqt > 1 ? (it.L - it.n + min(it.n, it.t_lo0 + 2 * T) - 1) / kN + 1 : 0;
+    it.ntiles = it.nqt > 1 ? it.nB : it.nA;
+    return true;
+}
+
 template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ PrefillArgs a, const __grid_constant__ CUtensorMap tmap_q,
-                      const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v)
+                      const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                      int npairs)
 {
     constexpr int T = kM / G;
-    const int pair = (int)gridDim.x - 1 - (int)blockIdx.x;
-    const int kvh = blockIdx.y;
-    const int s = blockIdx.z;
-    const int q0 = __ldg(a.q_start + s);
-    const int q1 = __ldg(a.q_start + s + 1);
-    const int n = q1 - q0;
-    int L = __ldg(a.context_lens + s);
-    const int Lcap = a.max_blocks_per_seq * a.block_size;
-    if (q0 < 0 || q1 > a.num_query_tokens || n < 0 || n > a.max_query_len || L < n || L > Lcap) {
-        if (threadIdx.x == 0 && pair == 0 && kvh == 0) atomicOr(a.status, PA_DEV_BAD_CONTEXT);
-        return;
-    }
-    const int t_lo0 = pair * kQT * T;
-    if (t_lo0 >= n) return;
-    const int nqt = t_lo0 + T < n ? 2 : 1;
-    const int nA = (L - n + min(n, t_lo0 + T) - 1) / kN + 1;
-    const int nB = nqt > 1 ? (L - n + min(n, t_lo0 + 2 * T) - 1) / kN + 1 : 0;
-    const int ntiles = nqt > 1 ? nB : nA;
+    const int nitems = npairs * a.num_seqs * a.num_kv_heads;
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTiles);
     uint64_t* q_full = bars;
-    uint64_t* k_full = q_full + 1;
+    uint64_t* q_empty = q_full + 1;
+    uint64_t* k_full = q_empty + 1;
     uint64_t* k_empty = k_full + KST;
     uint64_t* v_full = k_empty + KST;
     uint64_t* v_empty = v_full + VST;
     uint64_t* qbars = v_empty + VST;
-    uint64_t* drain = qbars + kQT * 3;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1) + 2;
-    float* xch = reinterpret_cast<float*>(drain + 3);
+    uint64_t* drain = qbars + kQT * 4;
+    uint64_t* it_full = drain + 1;    // item slot written (producer)
+    uint64_t* it_empty = it_full + IR;  // item slot read (MMA thread and the 16 softmax warps)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(it_empty + IR);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(it_empty + IR) + 2;
+    // [IR][kSlotInts]: the item (-1: the end), the ring position of its first K/V tile, its geometry
+    int* item_slot = reinterpret_cast<int*>(it_empty + IR) + 4;
+    float* xch = reinterpret_cast<float*>(item_slot + IR * kSlotInts);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
         for (int i = 0; i < KST; ++i) {
             mbar_init(&k_full[i], 1);
             mbar_init(&k_empty[i], 1);
@@ -180,11 +227,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&v_empty[i], 1);
         }
         for (int qt = 0; qt < kQT; ++qt) {
-            mbar_init(&qbars[3 * qt + 0], 1);
-            mbar_init(&qbars[3 * qt + 1], 8);
-            mbar_init(&qbars[3 * qt + 2], 1);
+            mbar_init(&qbars[4 * qt + 0], 1);  // s_full: S = Q.K^T in tensor memory
+            mbar_init(&qbars[4 * qt + 1], 8);  // p_full: P written by the tile's 8 softmax warps
+            mbar_init(&qbars[4 * qt + 2], 1);  // o_done: P.V finished
+            mbar_init(&qbars[4 * qt + 3], 8);  // o_free: the item's output read out of tensor memory
         }
         mbar_init(drain, 1);
+        for (int i = 0; i < IR; ++i) {
+            mbar_init(&it_full[i], 1);
+            mbar_init(&it_empty[i], 1 + 16);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -196,69 +248,112 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kProdWarp) {
         const uint64_t pol = policy_evict_normal();
-        if (lane == 0) {
-            mbar_arrive_expect_tx(q_full, nqt * 2 * kQHalf);
-            for (int qt = 0; qt < nqt; ++qt)
-                for (int h = 0; h < 2; ++h)
-                    tma_load_3d(smem_u32(smem + OFF_Q + qt * 2 * kQHalf + h * kQHalf), &tmap_q, h * 64, kvh * G,
-                                q0 + t_lo0 + qt * T, q_full, pol);
-        }
-        const int32_t* table = a.block_tables + (size_t)s * a.max_blocks_per_seq;
-        auto lookup = [&](int j) -> int {
-            const int tok = j * kN + lane * kBox;
-            return (j < ntiles && lane < kNBox && tok < L) ? __ldg(table + tok / a.block_size) : 0;
-        };
-        int next = lookup(0);
         bool ok = true;
-        int nk = 0, nv = 0;
-        for (int j = 0; j < ntiles && ok; ++j) {
-            int phys = next;
-            next = lookup(j + 1);
-            const int tok0 = j * kN;
-            const int nbox = min(kNBox, (L - tok0 + kBox - 1) / kBox);
-            const int tok = tok0 + lane * kBox;
-            if (lane < nbox && (unsigned)phys >= (unsigned)a.num_blocks) {
-                atomicOr(a.status, PA_DEV_BAD_BLOCK);
-                phys = 0;
-            }
-            const int row = (phys * a.num_kv_heads + kvh) * a.block_size + tok % a.block_size;
-            const uint32_t tx = (uint32_t)nbox * kBox * 128 * 2;
-            const int ks = j % KST;
+        int gt = 0;          // K/V tiles of this CTA's items so far: the rings' position
+        int nk = 0, nv = 0;  // K and V tile copies issued (they differ only after a failed wait)
+        int nit = 0;         // items whose Q was loaded
+        int claimed = 0;     // claims made (static grid: one)
+        for (;;) {
+            // claim the next item with work (lane 0), skipping empty items and flagging bad sequences
+            int item = nitems;
+            Item it;
             if (lane == 0) {
-                if (j >= KST && !mbar_wait_bounded(&k_empty[ks], ((j / KST) & 1) ^ 1, abort_flag)) ok = false;
-                if (ok) mbar_arrive_expect_tx(&k_full[ks], tx);
+                for (;;) {
+                    item = a.sched ? (int)atomicAdd(a.sched, 1u) : (claimed == 0 ? (int)blockIdx.x : nitems);
+                    ++claimed;
+                    if (item >= nitems) break;
+                    if (item_geom<G>(a, npairs, item, it)) break;
+                    if (it.bad && it.pair == 0 && it.kvh == 0) atomicOr(a.status, PA_DEV_BAD_CONTEXT);
+                }
+                // hand it out (or the end, as -1) once every reader is done with the slot's last item
+                if (nit >= IR && !mbar_wait_bounded(&it_empty[nit % IR], ((nit / IR) & 1) ^ 1, abort_flag))
+                    ok = false;
+                if (ok) {
+                    int* sp = item_slot + (nit % IR) * kSlotInts;
+                    sp[0] = item < nitems ? item : -1;
+                    sp[1] = gt;
+                    if (item < nitems) put_item(sp, it);
+                    mbar_arrive(&it_full[nit % IR]);
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            item = __shfl_sync(0xffffffffu, item, 0);
+            if (!ok || item >= nitems) break;
+            __syncwarp();  // lane 0's slot writes are visible to the warp
+            get_item(item_slot + (nit % IR) * kSlotInts, it);
+            // Q of this item goes over the last one's once every Q.K^T that read it has finished
+            if (lane == 0) {
+                if (nit > 0 && !mbar_wait_bounded(q_empty, (nit - 1) & 1, abort_flag)) ok = false;
+                if (ok) {
+                    mbar_arrive_expect_tx(q_full, it.nqt * 2 * kQHalf);
+                    for (int qt = 0; qt < it.nqt; ++qt)
+                        for (int h = 0; h < 2; ++h)
+                            tma_load_3d(smem_u32(smem + OFF_Q + qt * 2 * kQHalf + h * kQHalf), &tmap_q, h * 64,
+                                        it.kvh * G, it.q0 + it.t_lo0 + qt * T, q_full, pol);
+                }
             }
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (!ok) break;
-            if (lane < nbox)
-                for (int h = 0; h < 2; ++h)
-                    tma_load_2d(smem_u32(smem + OFF_K + ks * 2 * kKVHalf + h * kKVHalf + lane * kBox * 128), &tmap_k,
-                                h * 64, row, &k_full[ks], pol);
-            ++nk;
-            const int vs = j % VST;
-            if (lane == 0) {
-                if (j >= VST && !mbar_wait_bounded(&v_empty[vs], ((j / VST) & 1) ^ 1, abort_flag)) ok = false;
-                if (ok) mbar_arrive_expect_tx(&v_full[vs], tx);
+            ++nit;
+            const int32_t* table = a.block_tables + (size_t)it.s * a.max_blocks_per_seq;
+            auto lookup = [&](int j) -> int {
+                const int tok = j * kN + lane * kBox;
+                return (j < it.ntiles && lane < kNBox && tok < it.L) ? __ldg(table + tok / a.block_size) : 0;
+            };
+            int next = lookup(0);
+            for (int j = 0; j < it.ntiles; ++j) {
+                int phys = next;
+                next = lookup(j + 1);
+                const int g = gt + j;
+                const int tok0 = j * kN;
+                const int nbox = min(kNBox, (it.L - tok0 + kBox - 1) / kBox);
+                const int tok = tok0 + lane * kBox;
+                if (lane < nbox && (unsigned)phys >= (unsigned)a.num_blocks) {
+                    atomicOr(a.status, PA_DEV_BAD_BLOCK);
+                    phys = 0;
+                }
+                const int row = (phys * a.num_kv_heads + it.kvh) * a.block_size + tok % a.block_size;
+                const uint32_t tx = (uint32_t)nbox * kBox * 128 * 2;
+                const int ks = g % KST;
+                if (lane == 0) {
+                    if (g >= KST && !mbar_wait_bounded(&k_empty[ks], ((g / KST) & 1) ^ 1, abort_flag)) ok = false;
+                    if (ok) mbar_arrive_expect_tx(&k_full[ks], tx);
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
+                if (lane < nbox)
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_2d(smem_u32(smem + OFF_K + ks * 2 * kKVHalf + h * kKVHalf + lane * kBox * 128),
+                                    &tmap_k, h * 64, row, &k_full[ks], pol);
+                ++nk;
+                const int vs = g % VST;
+                if (lane == 0) {
+                    if (g >= VST && !mbar_wait_bounded(&v_empty[vs], ((g / VST) & 1) ^ 1, abort_flag)) ok = false;
+                    if (ok) mbar_arrive_expect_tx(&v_full[vs], tx);
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
+                if (lane < nbox)
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_2d(smem_u32(smem + OFF_V + vs * 2 * kKVHalf + h * kKVHalf + lane * kBox * 128),
+                                    &tmap_v, h * 64, row, &v_full[vs], pol);
+                ++nv;
             }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) break;
-            if (lane < nbox)
-                for (int h = 0; h < 2; ++h)
-                    tma_load_2d(smem_u32(smem + OFF_V + vs * 2 * kKVHalf + h * kKVHalf + lane * kBox * 128), &tmap_v,
-                                h * 64, row, &v_full[vs], pol);
-            ++nv;
+            gt += it.ntiles;
         }
         if (lane == 0) {
             if (!ok) {
                 atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
                 *abort_flag = 1;
             }
+            // nothing may still be landing in shared memory when the CTA exits
             volatile int never = 0;
-            if (!mbar_wait_bounded(q_full, 0, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
-            for (int j = max(0, nk - KST); j < nk; ++j)
-                if (!mbar_wait_bounded(&k_full[j % KST], (j / KST) & 1, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
-            for (int j = max(0, nv - VST); j < nv; ++j)
-                if (!mbar_wait_bounded(&v_full[j % VST], (j / VST) & 1, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+            if (nit > 0 && !mbar_wait_bounded(q_full, (nit - 1) & 1, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+            // a copy older than the last ring's worth had its stage released, so it has landed
+            for (int g = max(0, nk - KST); g < nk; ++g)
+                if (!mbar_wait_bounded(&k_full[g % KST], (g / KST) & 1, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
+            for (int g = max(0, nv - VST); g < nv; ++g)
+                if (!mbar_wait_bounded(&v_full[g % VST], (g / VST) & 1, &never)) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
         }
     } else if (warp == kMmaWarp) {
         // MMA issuer, in a fixed order that staggers the two query tiles: P.V_A(j), S_A(j+1),
@@ -268,63 +363,106 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idesc_qk = umma_idesc_bf16(kM, kN, false);
             constexpr uint32_t idesc_pv = umma_idesc_bf16(kM, kD, true);
             const uint32_t sq = smem_u32(smem + OFF_Q), sk = smem_u32(smem + OFF_K), sv = smem_u32(smem + OFF_V);
-            auto issue_qk = [&](int qt, int j) {
+            auto issue_qk = [&](int qt, int g) {
                 const uint32_t qb = sq + qt * 2 * kQHalf;
-                const uint32_t kb = sk + (j % KST) * 2 * kKVHalf;
+                const uint32_t kb = sk + (g % KST) * 2 * kKVHalf;
 #pragma unroll
                 for (int k = 0; k < kD / 16; ++k) {
                     const uint32_t kk = (k & 3) * 32;
                     umma_bf16_ss(tmem + qt * 256, umma_desc_sw128(qb + (k >> 2) * kQHalf + kk, 16, 1024),
                                  umma_desc_sw128(kb + (k >> 2) * kKVHalf + kk, 16, 1024), idesc_qk, k > 0 ? 1u : 0u);
                 }
-                umma_commit(&qbars[3 * qt + 0]);
+                umma_commit(&qbars[4 * qt + 0]);
             };
-            auto issue_pv = [&](int qt, int j) {
+            auto issue_pv = [&](int qt, int g, bool first) {
                 const uint32_t ts = tmem + qt * 256;
-                const uint32_t vb = sv + (j % VST) * 2 * kKVHalf;
+                const uint32_t vb = sv + (g % VST) * 2 * kKVHalf;
 #pragma unroll
                 for (int k = 0; k < kN / 16; ++k) {
                     umma_bf16_ts(ts + 128, ts + k * 8, umma_desc_sw128(vb + k * 16 * 128, kKVHalf, 1024), idesc_pv,
-                                 (j > 0 || k > 0) ? 1u : 0u);
+                                 (!first || k > 0) ? 1u : 0u);
                 }
-                umma_commit(&qbars[3 * qt + 2]);
+                umma_commit(&qbars[4 * qt + 2]);
             };
-            const int need[kQT] = {nA, nB};
-            bool ok = mbar_wait_bounded(q_full, 0, abort_flag) && mbar_wait_bounded(&k_full[0], 0, abort_flag);
-            if (ok) {
-                tc_fence_after_sync();
-                issue_qk(0, 0);
-                if (nB > 0) issue_qk(1, 0);
-                umma_commit(&k_empty[0]);
-            }
-            for (int j = 0; j < ntiles && ok; ++j) {
-                const bool k_next = j + 1 < ntiles;
-                if (!mbar_wait_bounded(&v_full[j % VST], (j / VST) & 1, abort_flag)) {
+            bool ok = true;
+            int gt = 0, nit = 0;
+            // per query-tile slot (scalars, so that nothing goes to local memory): tiles so far (S, P and P.V
+            // phases) and items so far (o_free phases)
+            int cntA = 0, cntB = 0, nitA = 0, nitB = 0;
+            for (;;) {
+                if (!mbar_wait_bounded(&it_full[nit % IR], (nit / IR) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                for (int qt = 0; qt < kQT && ok; ++qt) {
-                    if (j >= need[qt]) continue;
-                    if (!mbar_wait_bounded(&qbars[3 * qt + 1], j & 1, abort_flag)) {  // P(j) written
+                const volatile int* sp = item_slot + (nit % IR) * kSlotInts;
+                const int item = sp[0];
+                mbar_arrive(&it_empty[nit % IR]);
+                if (item < 0) break;
+                Item it;
+                get_item(sp, it);
+                const int nA = it.nA, nB = it.nB;
+                ok = mbar_wait_bounded(q_full, nit & 1, abort_flag) &&
+                     mbar_wait_bounded(&k_full[gt % KST], (gt / KST) & 1, abort_flag);
+#pragma unroll
+                for (int qt = 0; qt < kQT; ++qt) {
+                    if (!ok || qt >= it.nqt) continue;
+                    const int cnt = qt == 0 ? cntA : cntB;
+                    // S goes over the columns the slot's last P was read from
+                    if (cnt > 0 && !mbar_wait_bounded(&qbars[4 * qt + 2], (cnt - 1) & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
-                    issue_pv(qt, j);
-                    if (j + 1 < need[qt]) {
-                        // S(j+1) goes over the columns P(j) is read from: after P.V(j) has finished
-                        if (!mbar_wait_bounded(&k_full[(j + 1) % KST], ((j + 1) / KST) & 1, abort_flag) ||
-                            !mbar_wait_bounded(&qbars[3 * qt + 2], j & 1, abort_flag)) {
+                    issue_qk(qt, gt);
+                }
+                if (!ok) break;
+                umma_commit(&k_empty[gt % KST]);
+                if (it.ntiles == 1) umma_commit(q_empty);
+                for (int j = 0; j < it.ntiles && ok; ++j) {
+                    const int g = gt + j;
+                    if (!mbar_wait_bounded(&v_full[g % VST], (g / VST) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int qt = 0; qt < kQT; ++qt) {
+                        const int need = qt == 0 ? nA : nB;
+                        const int cnt = qt == 0 ? cntA : cntB;
+                        const int nitq = qt == 0 ? nitA : nitB;
+                        if (!ok || j >= need) continue;
+                        if (!mbar_wait_bounded(&qbars[4 * qt + 1], (cnt + j) & 1, abort_flag) ||  // P(j) written
+                            (j == 0 && nitq > 0 &&
+                             !mbar_wait_bounded(&qbars[4 * qt + 3], (nitq - 1) & 1, abort_flag))) {  // O read out
                             ok = false;
                             break;
                         }
                         tc_fence_after_sync();
-                        issue_qk(qt, j + 1);
+                        issue_pv(qt, g, j == 0);
+                        if (j + 1 < need) {
+                            // S(j+1) goes over the columns P(j) is read from: after P.V(j) has finished
+                            if (!mbar_wait_bounded(&k_full[(g + 1) % KST], ((g + 1) / KST) & 1, abort_flag) ||
+                                !mbar_wait_bounded(&qbars[4 * qt + 2], (cnt + j) & 1, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after_sync();
+                            issue_qk(qt, g + 1);
+                        }
                     }
+                    if (!ok) break;
+                    umma_commit(&v_empty[g % VST]);
+                    if (j + 1 < it.ntiles) umma_commit(&k_empty[(g + 1) % KST]);
+                    if (j + 2 == it.ntiles) umma_commit(q_empty);  // the item's last Q.K^T went out in this step
                 }
+                cntA += nA;
+                ++nitA;
+                if (it.nqt > 1) {
+                    cntB += nB;
+                    ++nitB;
+                }
+                gt += it.ntiles;
+                ++nit;
                 if (!ok) break;
-                umma_commit(&v_empty[j % VST]);
-                if (k_next) umma_commit(&k_empty[(j + 1) % KST]);
             }
             if (!ok) {
                 atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
@@ -341,161 +479,192 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int half = (warp >> 2) & 1;
         const int r = threadIdx.x & 127;
         const int t256 = threadIdx.x & 255;
-        const int t_lo = t_lo0 + qt * T;
-        const int ntq = qt == 0 ? nA : nB;
-        uint64_t* s_full = &qbars[3 * qt + 0];
-        uint64_t* p_full = &qbars[3 * qt + 1];
-        uint64_t* o_done = &qbars[3 * qt + 2];
+        uint64_t* s_full = &qbars[4 * qt + 0];
+        uint64_t* p_full = &qbars[4 * qt + 1];
+        uint64_t* o_done = &qbars[4 * qt + 2];
+        uint64_t* o_free = &qbars[4 * qt + 3];
         const int pair_bar = 1 + qt * 4 + (warp & 3);
         const uint32_t tmem_s = tmem + qt * 256;
         const uint32_t tmem_o = tmem_s + 128;
         const int t_local = r / G;
         const int g = r % G;
-        const int tq = t_lo + t_local;
-        const bool valid_row = t_local < T && tq < n;
-        const int lim = valid_row ? (L - n + tq) : -1;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const float sl = a.scale_log2;
-        float m_used = -INFINITY, l = 0.f;
-        bool ok = true;
+        const float masked = sl >= 0.f ? -INFINITY : INFINITY;
         constexpr int NC = 2;  // 32-key chunks per half
+        bool ok = true;
+        int cnt = 0;  // tiles of this slot so far
+        int xc = 0;   // exchanges with the other half so far (the buffer alternates)
         auto xslot = [&](int par, int h) -> float* { return xch + ((par * kQT + qt) * 2 + h) * 128 + r; };
-        for (int j = 0; j < ntq; ++j) {
-            // a failed wait is carried to the pair barrier below, where both warps leave together
-            const bool ok_s = ok && mbar_wait_warp(s_full, j & 1, abort_flag);
-            tc_fence_after_sync();
-            uint32_t sr[NC][32];
-#pragma unroll
-            for (int c = 0; c < NC; ++c) tmem_ld32(tmem_s + lane_base + half * 64 + c * 32, sr[c]);
-            tmem_wait_ld();
-            const int kv0 = j * kN + half * 64;
-            const float masked = sl >= 0.f ? -INFINITY : INFINITY;
-            const bool mask_tile = __any_sync(0xffffffffu, kv0 + 63 > lim);
-            if (mask_tile) {
-#pragma unroll
-                for (int c = 0; c < NC; ++c)
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (kv0 + c * 32 + e > lim) sr[c][e] = __float_as_uint(masked);
+        for (int k = 0;; ++k) {
+            const bool got = ok && mbar_wait_warp(&it_full[k % IR], (k / IR) & 1, abort_flag);
+            const volatile int* slot_k = item_slot + (k % IR) * kSlotInts;  // held until this item is done
+            const int item = got ? slot_k[0] : -1;
+            __syncwarp();
+            // the two warps of a row pair leave together: a warp whose wait failed stops its partner too
+            if (!pair_sync_and(pair_bar, got && item >= 0)) {
+                if (!got || item >= 0) ok = false;
+                break;
             }
-            float m0 = masked, m1 = masked, m2 = masked, m3 = masked, m4 = masked, m5 = masked, m6 = masked,
-                  m7 = masked;
-            if (sl >= 0.f) {
-#pragma unroll
-                for (int c = 0; c < NC; ++c)
-#pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        m0 = fmaxf(m0, __uint_as_float(sr[c][e + 0]));
-                        m1 = fmaxf(m1, __uint_as_float(sr[c][e + 1]));
-                        m2 = fmaxf(m2, __uint_as_float(sr[c][e + 2]));
-                        m3 = fmaxf(m3, __uint_as_float(sr[c][e + 3]));
-                        m4 = fmaxf(m4, __uint_as_float(sr[c][e + 4]));
-                        m5 = fmaxf(m5, __uint_as_float(sr[c][e + 5]));
-                        m6 = fmaxf(m6, __uint_as_float(sr[c][e + 6]));
-                        m7 = fmaxf(m7, __uint_as_float(sr[c][e + 7]));
-                    }
-                m0 = fmaxf(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)), fmaxf(fmaxf(m4, m5), fmaxf(m6, m7)));
-            } else {
-#pragma unroll
-                for (int c = 0; c < NC; ++c)
-#pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        m0 = fminf(m0, __uint_as_float(sr[c][e + 0]));
-                        m1 = fminf(m1, __uint_as_float(sr[c][e + 1]));
-                        m2 = fminf(m2, __uint_as_float(sr[c][e + 2]));
-                        m3 = fminf(m3, __uint_as_float(sr[c][e + 3]));
-                        m4 = fminf(m4, __uint_as_float(sr[c][e + 4]));
-                        m5 = fminf(m5, __uint_as_float(sr[c][e + 5]));
-                        m6 = fminf(m6, __uint_as_float(sr[c][e + 6]));
-                        m7 = fminf(m7, __uint_as_float(sr[c][e + 7]));
-                    }
-                m0 = fminf(fminf(fminf(m0, m1), fminf(m2, m3)), fminf(fminf(m4, m5), fminf(m6, m7)));
+            int ntq, lim, jz;  // tiles of this slot, this row's last key, the key tile past the context (or -1)
+            {
+                Item it;
+                get_item(slot_k, it);
+                ntq = qt == 0 ? it.nA : it.nB;
+                const int tq = it.t_lo0 + qt * T + t_local;
+                lim = (t_local < T && tq < it.n) ? (it.L - it.n + tq) : -1;
+                jz = (it.L % kN != 0 && (it.L - 1) / kN < ntq) ? (it.L - 1) / kN : -1;
             }
-            // swap the partial maxima; the barrier also orders this half's S reads before the other half's P
-            // stores over S's first 64 columns
-            *xslot(j & 1, half) = m0;
-            tc_fence_before_sync();
-            if (!pair_sync_and(pair_bar, ok_s)) {
+            if (ntq == 0) {
+                if (lane == 0) mbar_arrive(&it_empty[k % IR]);
+                continue;
+            }
+            float m_used = -INFINITY, l = 0.f;
+            for (int j = 0; j < ntq; ++j) {
+                // a failed wait is carried to the pair barrier below, where both warps leave together
+                const bool ok_s = ok && mbar_wait_warp(s_full, (cnt + j) & 1, abort_flag);
+                tc_fence_after_sync();
+                uint32_t sr[NC][32];
+#pragma unroll
+                for (int c = 0; c < NC; ++c) tmem_ld32(tmem_s + lane_base + half * 64 + c * 32, sr[c]);
+                tmem_wait_ld();
+                const int kv0 = j * kN + half * 64;
+                const bool mask_tile = __any_sync(0xffffffffu, kv0 + 63 > lim);
+                if (mask_tile) {
+#pragma unroll
+                    for (int c = 0; c < NC; ++c)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (kv0 + c * 32 + e > lim) sr[c][e] = __float_as_uint(masked);
+                }
+                float m0 = masked, m1 = masked, m2 = masked, m3 = masked, m4 = masked, m5 = masked, m6 = masked,
+                      m7 = masked;
+                if (sl >= 0.f) {
+#pragma unroll
+                    for (int c = 0; c < NC; ++c)
+#pragma unroll
+                        for (int e = 0; e < 32; e += 8) {
+                            m0 = fmaxf(m0, __uint_as_float(sr[c][e + 0]));
+                            m1 = fmaxf(m1, __uint_as_float(sr[c][e + 1]));
+                            m2 = fmaxf(m2, __uint_as_float(sr[c][e + 2]));
+                            m3 = fmaxf(m3, __uint_as_float(sr[c][e + 3]));
+                            m4 = fmaxf(m4, __uint_as_float(sr[c][e + 4]));
+                            m5 = fmaxf(m5, __uint_as_float(sr[c][e + 5]));
+                            m6 = fmaxf(m6, __uint_as_float(sr[c][e + 6]));
+                            m7 = fmaxf(m7, __uint_as_float(sr[c][e + 7]));
+                        }
+                    m0 = fmaxf(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)), fmaxf(fmaxf(m4, m5), fmaxf(m6, m7)));
+                } else {
+#pragma unroll
+                    for (int c = 0; c < NC; ++c)
+#pragma unroll
+                        for (int e = 0; e < 32; e += 8) {
+                            m0 = fminf(m0, __uint_as_float(sr[c][e + 0]));
+                            m1 = fminf(m1, __uint_as_float(sr[c][e + 1]));
+                            m2 = fminf(m2, __uint_as_float(sr[c][e + 2]));
+                            m3 = fminf(m3, __uint_as_float(sr[c][e + 3]));
+                            m4 = fminf(m4, __uint_as_float(sr[c][e + 4]));
+                            m5 = fminf(m5, __uint_as_float(sr[c][e + 5]));
+                            m6 = fminf(m6, __uint_as_float(sr[c][e + 6]));
+                            m7 = fminf(m7, __uint_as_float(sr[c][e + 7]));
+                        }
+                    m0 = fminf(fminf(fminf(m0, m1), fminf(m2, m3)), fminf(fminf(m4, m5), fminf(m6, m7)));
+                }
+                // swap the partial maxima; the barrier also orders this half's S reads before the other half's
+                // P stores over S's first 64 columns
+                *xslot(xc & 1, half) = m0;
+                tc_fence_before_sync();
+                const bool pair_ok = pair_sync_and(pair_bar, ok_s);
+                ++xc;
+                if (!pair_ok) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const float other = *xslot((xc - 1) & 1, half ^ 1);
+                const float mraw = sl >= 0.f ? fmaxf(m0, other) : fminf(m0, other);
+                const float mx = mraw == masked ? -INFINITY : mraw * sl;
+                const float m_new = fmaxf(m_used, mx);
+                const bool rescale = m_used != -INFINITY && m_new > m_used + (float)kLazyRescale;
+                const bool rescale_warp = __any_sync(0xffffffffu, rescale) != 0;
+                const float alpha = rescale ? fast_exp2(m_used - m_new) : 1.f;
+                if (rescale || m_used == -INFINITY) m_used = m_new;
+                const float mref = m_used == -INFINITY ? 0.f : m_used;
+                float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
+#pragma unroll
+                for (int c = 0; c < NC; ++c) {
+#pragma unroll
+                    for (int e2 = 0; e2 < 16; ++e2) {
+                        const float2 pp = exp2_pair(fmaf(__uint_as_float(sr[c][2 * e2]), sl, -mref),
+                                                    fmaf(__uint_as_float(sr[c][2 * e2 + 1]), sl, -mref));
+                        float p0 = pp.x, p1 = pp.y;
+                        if (mask_tile) {
+                            const int kv = kv0 + c * 32 + 2 * e2;
+                            p0 = kv <= lim ? p0 : 0.f;
+                            p1 = kv + 1 <= lim ? p1 : 0.f;
+                        }
+                        if (e2 & 1) {
+                            rs2 += p0;
+                            rs3 += p1;
+                        } else {
+                            rs0 += p0;
+                            rs1 += p1;
+                        }
+                        sr[c][e2] = pack_bf16(p0, p1);
+                    }
+                    tmem_st16(tmem_s + lane_base + half * 32 + c * 16, sr[c]);
+                }
+                if (rescale_warp) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tmem_o + lane_base + half * 64 + c * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(tmem_o + lane_base + half * 64 + c * 32, o);
+                    }
+                }
+                tmem_wait_st();
+                l = l * alpha + ((rs0 + rs1) + (rs2 + rs3));
+                if (j == jz) {
+                    // rows past the context: their P is 0, and 0 must not meet a NaN left in the pool
+                    const int gv = slot_k[1] + j;
+                    const bool v_ok = mbar_wait_warp(&v_full[gv % VST], (gv / VST) & 1, abort_flag);
+                    if (!v_ok) ok = false;
+                    const int first = max(0, slot_k[7] - j * kN);
+                    const int chunks = v_ok ? (kN - first) * 16 : 0;
+                    for (int i = t256; i < chunks; i += 256) {
+                        const int row = first + (i >> 4);
+                        const int h = (i >> 3) & 1;
+                        *reinterpret_cast<uint4*>(smem + OFF_V + (gv % VST) * 2 * kKVHalf + h * kKVHalf + row * 128 +
+                                                  (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+                    }
+                }
+                fence_async_smem();
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(p_full);
+            }
+            // both warps of the pair always get here, with the same number of exchanges behind them
+            const bool ok_o = ok && mbar_wait_warp(o_done, (cnt + ntq - 1) & 1, abort_flag);
+            if (lane == 0) mbar_arrive(&it_empty[k % IR]);
+            *xslot(xc & 1, half) = l;
+            const bool all_ok = pair_sync_and(pair_bar, ok_o);
+            ++xc;
+            if (!all_ok) {
                 ok = false;
                 break;
             }
             tc_fence_after_sync();
-            const float other = *xslot(j & 1, half ^ 1);
-            const float mraw = sl >= 0.f ? fmaxf(m0, other) : fminf(m0, other);
-            const float mx = mraw == masked ? -INFINITY : mraw * sl;
-            const float m_new = fmaxf(m_used, mx);
-            const bool rescale = m_used != -INFINITY && m_new > m_used + (float)kLazyRescale;
-            const bool rescale_warp = __any_sync(0xffffffffu, rescale) != 0;
-            const float alpha = rescale ? fast_exp2(m_used - m_new) : 1.f;
-            if (rescale || m_used == -INFINITY) m_used = m_new;
-            const float mref = m_used == -INFINITY ? 0.f : m_used;
-            float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
-#pragma unroll
-            for (int c = 0; c < NC; ++c) {
-#pragma unroll
-                for (int e2 = 0; e2 < 16; ++e2) {
-                    const float2 pp = exp2_pair(fmaf(__uint_as_float(sr[c][2 * e2]), sl, -mref),
-                                                fmaf(__uint_as_float(sr[c][2 * e2 + 1]), sl, -mref));
-                    float p0 = pp.x, p1 = pp.y;
-                    if (mask_tile) {
-                        const int kv = kv0 + c * 32 + 2 * e2;
-                        p0 = kv <= lim ? p0 : 0.f;
-                        p1 = kv + 1 <= lim ? p1 : 0.f;
-                    }
-                    if (e2 & 1) {
-                        rs2 += p0;
-                        rs3 += p1;
-                    } else {
-                        rs0 += p0;
-                        rs1 += p1;
-                    }
-                    sr[c][e2] = pack_bf16(p0, p1);
-                }
-                tmem_st16(tmem_s + lane_base + half * 32 + c * 16, sr[c]);
-            }
-            if (rescale_warp) {
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(tmem_o + lane_base + half * 64 + c * 32, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    tmem_st32(tmem_o + lane_base + half * 64 + c * 32, o);
-                }
-            }
-            tmem_wait_st();
-            l = l * alpha + ((rs0 + rs1) + (rs2 + rs3));
-            if (j * kN + kN > L) {
-                // V rows past the context: their P is 0, and 0 must not meet a NaN left in the pool
-                const bool v_ok = mbar_wait_warp(&v_full[j % VST], (j / VST) & 1, abort_flag);
-                if (!v_ok) ok = false;
-                const int first = max(0, L - j * kN);
-                const int chunks = v_ok ? (kN - first) * 16 : 0;
-                for (int i = t256; i < chunks; i += 256) {
-                    const int row = first + (i >> 4);
-                    const int h = (i >> 3) & 1;
-                    *reinterpret_cast<uint4*>(smem + OFF_V + (j % VST) * 2 * kKVHalf + h * kKVHalf + row * 128 +
-                                              (i & 7) * 16) = make_uint4(0, 0, 0, 0);
-                }
-            }
-            fence_async_smem();
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
-        }
-        if (ntq > 0) {
-            // the row sum is split between the halves as well; both warps of the pair always get here
-            *xslot(ntq & 1, half) = l;
-            if (!pair_sync_and(pair_bar, ok)) ok = false;
-            if (ok) l += *xslot(ntq & 1, half ^ 1);
-        }
-        if (ntq == 0) {
-        } else if (ok && mbar_wait_warp(o_done, (ntq - 1) & 1, abort_flag)) {
-            tc_fence_after_sync();
+            l += *xslot((xc - 1) & 1, half ^ 1);
             const float inv = l > 0.f ? 1.f / l : 0.f;
+            Item it;
+            get_item(slot_k, it);
+            const int tq = it.t_lo0 + qt * T + t_local;
+            const bool valid_row = t_local < T && tq < it.n;
             __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) +
-                                 ((size_t)(q0 + tq) * a.num_heads + (size_t)kvh * G + g) * kD + half * 64;
+                                 ((size_t)(it.q0 + tq) * a.num_heads + (size_t)it.kvh * G + g) * kD + half * 64;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t o[32];
@@ -513,8 +682,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-        } else {
-            ok = false;
+            // O may now take the slot's next item
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(o_free);
+            cnt += ntq;
         }
         if (!ok) {
             if (lane == 0) atomicOr(a.status, PA_DEV_WAIT_TIMEOUT);
@@ -567,9 +739,17 @@ cudaError_t launch_g(const PrefillArgs& a, int num_query_tokens, int max_query_l
         attr_done[dev & 63].store(true);
     }
     constexpr int T = kM / G;
-    const dim3 grid((unsigned)((max_query_len + kQT * T - 1) / (kQT * T)), (unsigned)a.num_kv_heads,
-                    (unsigned)a.num_seqs);
-    prefill_tc_kernel<G><<<grid, kThreads, kSmem, stream>>>(a, tq, tk, tv);
+    static std::atomic<int> sm_count[64] = {};
+    int sms = sm_count[dev & 63].load();
+    if (sms == 0) {
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        sm_count[dev & 63].store(sms);
+    }
+    const int npairs = (max_query_len + kQT * T - 1) / (kQT * T);
+    const long long nitems = (long long)npairs * a.num_seqs * a.num_kv_heads;
+    if (nitems > INT32_MAX) return cudaErrorInvalidValue;
+    const int grid = a.sched ? (int)std::min<long long>(nitems, sms) : (int)nitems;
+    prefill_tc_kernel<G><<<grid, kThreads, kSmem, stream>>>(a, tq, tk, tv, npairs);
     return cudaGetLastError();
 }
 

@@ -42,6 +42,8 @@ SIGNATURES = [
     ("pa_decode_static_workspace", _int, [_vp, _vp, _vp, _vp, _vp, _vp] + [_int] * 8 + [_f32, _int, _int, _vp]),
     ("pa_reshape_and_cache", _int, [_vp, _vp, _vp, _vp, _vp] + [_int] * 6 + [_vp]),
     ("pa_prefill", _int, [_vp] * 7 + [_int] * 9 + [_f32, _int, _vp]),
+    ("pa_prefill_workspace_size", _sz, []),
+    ("pa_prefill_ws", _int, [_vp] * 7 + [_int] * 9 + [_f32, _vp, _sz, _int, _vp]),
     ("pa_copy_blocks", _int, [_vp, _vp, _vp] + [_int] * 6 + [_vp]),
     ("pa_check_block_mapping", _int, [_vp, _int, _int]),
     ("pa_check_slot_mapping", _int, [_vp, _int, _int, _int]),
@@ -274,9 +276,15 @@ def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None
     _check(st, "pa_reshape_and_cache")
 
 
-def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, q_start, max_query_len, scale, stream=None):
+def pa_prefill_workspace_size():
+    return int(lib.pa_prefill_workspace_size())
+
+
+def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, q_start, max_query_len, scale, stream=None,
+               workspace=None):
     """out[Nq,Hq,D] <- causal attention of the packed query rows q[Nq,Hq,D] (rows q_start[s]..q_start[s+1]-1
-    are the last tokens of sequence s) over k/v_cache[NB,Hkv,B,D] through block_tables."""
+    are the last tokens of sequence s) over k/v_cache[NB,Hkv,B,D] through block_tables.  With a device
+    `workspace` (at least pa_prefill_workspace_size() bytes) this calls pa_prefill_ws."""
     import torch
     Nq, Hq, D = q.shape
     NB, Hkv, B, D2 = k_cache.shape
@@ -290,11 +298,16 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, q_start, ma
     dt = _dtype_code(q)
     if any(_dtype_code(t) != dt for t in (out, k_cache, v_cache)):
         raise TypeError("q, out and the caches must share a dtype")
-    st = lib.pa_prefill(_dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
-                        _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables"),
-                        _dev_ptr(context_lens, "context_lens"), _dev_ptr(q_start, "q_start"), S, Hq, Hkv, D, B,
-                        block_tables.shape[1], NB, Nq, int(max_query_len), float(scale), dt, _stream(stream))
-    _check(st, "pa_prefill")
+    args = (_dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+            _dev_ptr(block_tables, "block_tables"), _dev_ptr(context_lens, "context_lens"),
+            _dev_ptr(q_start, "q_start"), S, Hq, Hkv, D, B, block_tables.shape[1], NB, Nq, int(max_query_len),
+            float(scale))
+    if workspace is None:
+        _check(lib.pa_prefill(*args, dt, _stream(stream)), "pa_prefill")
+    else:
+        nbytes = workspace.numel() * workspace.element_size()
+        _check(lib.pa_prefill_ws(*args, _dev_ptr(workspace, "workspace"), nbytes, dt, _stream(stream)),
+               "pa_prefill_ws")
 
 
 def pa_swap_blocks(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache, block_mapping, stream=None):

@@ -380,7 +380,7 @@ class BeamBatch:
 
 class PrefillBatch:
     """Chunked prefill: every sequence's prefix and chunk placed by the allocator and
-    written with pa_reshape_and_cache; the step is one pa_prefill over all chunks."""
+    written with pa_reshape_and_cache; the step is one pa_prefill_ws over all chunks."""
 
     def __init__(self, wl, device="cuda", values=None, fill=float("nan"), partition_size=None):
         self.wl = wl
@@ -407,10 +407,11 @@ class PrefillBatch:
         self.max_query_len = int(wl.query_lens.max()) if S else 0
         self.q = q.to(self.device).contiguous()
         self.out = torch.empty_like(self.q)
+        self.workspace = torch.empty(pa.pa_prefill_workspace_size(), dtype=torch.uint8, device=self.device)
 
     def step(self, stream=None):
         pa.pa_prefill(self.out, self.q, self.k_cache, self.v_cache, self.block_tables, self.context_lens,
-                      self.q_start, self.max_query_len, self.wl.scale, stream=stream)
+                      self.q_start, self.max_query_len, self.wl.scale, stream=stream, workspace=self.workspace)
         return self.out
 
 

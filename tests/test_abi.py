@@ -55,6 +55,13 @@ def test_host_validation_rejects_before_any_device_work():
     assert "workspace" in L.pa_last_error_string().decode()
     # zero sequences is a no-op
     assert L.pa_decode(None, None, None, None, None, None, 0, 4, 4, 128, 16, 4, 8, 0, 1.0, 0, None, 0, 1, None) == pa.PA_OK
+    # prefill with a workspace: a null or short one is refused before anything else
+    assert L.pa_prefill_workspace_size() >= 16
+    assert L.pa_prefill_ws(p, p, p, p, p, p, p, 1, 4, 4, 128, 16, 4, 8, 16, 16, 1.0, None, 256, 1, None) == \
+        pa.PA_ERR_INVALID
+    assert L.pa_prefill_ws(p, p, p, p, p, p, p, 1, 4, 4, 128, 16, 4, 8, 16, 16, 1.0, p, 8, 1, None) == \
+        pa.PA_ERR_INVALID
+    assert "workspace" in L.pa_last_error_string().decode()
     # companions
     assert L.pa_reshape_and_cache(p, p, p, p, p, 4, 4, 100, 16, 8, 1, None) == pa.PA_ERR_UNSUPPORTED
     assert L.pa_reshape_and_cache(p, p, p, p, None, 4, 4, 128, 16, 8, 1, None) == pa.PA_ERR_INVALID

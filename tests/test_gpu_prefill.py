@@ -45,11 +45,21 @@ def _case(seed, lens, nq, Hq, Hkv, B, D=128):
     return q, k, v, tables, np.array(lens, np.int32), q_start
 
 
-def _run(pa, q, k, v, tables, lens, q_start, scale):
+def _run(pa, q, k, v, tables, lens, q_start, scale, ws=True, calls=1):
+    """pa_prefill_ws (one CTA per SM taking items from a counter) or, with ws=False, pa_prefill (one item per
+    CTA); `calls` > 1 repeats the call on the same workspace and checks that every call gives the same bits."""
     out = torch.full(q.shape, 7.0, dtype=torch.bfloat16, device="cuda")
-    pa.pa_prefill(out, q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda(),
-                  torch.from_numpy(q_start).cuda(), int(np.max(np.diff(q_start))), scale)
-    torch.cuda.synchronize()
+    workspace = torch.empty(pa.pa_prefill_workspace_size(), dtype=torch.uint8, device="cuda") if ws else None
+    first = None
+    for _ in range(calls):
+        pa.pa_prefill(out, q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(tables).cuda(),
+                      torch.from_numpy(lens).cuda(), torch.from_numpy(q_start).cuda(), int(np.max(np.diff(q_start))),
+                      scale, workspace=workspace)
+        torch.cuda.synchronize()
+        if first is None:
+            first = out.clone()
+        else:
+            assert torch.equal(out, first), "a repeated call on the same workspace changed the output"
     return out.float().cpu().numpy()
 
 
@@ -75,9 +85,11 @@ def test_prefill_matches_oracle(pa, G, B, case):
     Hkv = 2
     q, k, v, tables, L, qs = _case(100 * G + B + case, lens, nq, Hkv * G, Hkv, B)
     scale = 128 ** -0.5
-    got = _run(pa, q, k, v, tables, L, qs, scale)
+    got = _run(pa, q, k, v, tables, L, qs, scale, calls=2)
     assert np.isfinite(got).all()
     assert max_abs(got, _oracle(q, k, v, tables, L, qs, scale)) <= TOL["bf16"]
+    # the grid of one item per CTA computes each item the same way: the same bits
+    assert np.array_equal(_run(pa, q, k, v, tables, L, qs, scale, ws=False), got)
     assert pa.pa_device_status() == 0
 
 
@@ -113,8 +125,9 @@ def test_bad_chunk_is_flagged_and_skipped(pa):
     assert max_abs(got[:10], _oracle(q[:10], k, v, tables[:1], L[:1], qs[:2], 0.1)) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("ws", [True, False])
 @pytest.mark.parametrize("bad", ["past_end", "backwards", "negative_start", "over_max_query_len"])
-def test_bad_query_rows_are_flagged_and_skipped(pa, bad):
+def test_bad_query_rows_are_flagged_and_skipped(pa, bad, ws):
     """q_start is device data: a sequence whose query rows leave [0, num_query_tokens),
     run backwards, or outnumber max_query_len is flagged and skipped whole before any
     store, and the other sequence still matches the oracle."""
@@ -133,8 +146,9 @@ def test_bad_query_rows_are_flagged_and_skipped(pa, bad):
     elif bad == "over_max_query_len":
         max_q = 15                              # sequence 1 has 20 rows
     out = torch.full(q.shape, 7.0, dtype=torch.bfloat16, device="cuda")
+    workspace = torch.empty(pa.pa_prefill_workspace_size(), dtype=torch.uint8, device="cuda") if ws else None
     pa.pa_prefill(out, q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(tables).cuda(), torch.from_numpy(L).cuda(),
-                  torch.from_numpy(qs_bad).cuda(), max_q, 0.1)
+                  torch.from_numpy(qs_bad).cuda(), max_q, 0.1, workspace=workspace)
     torch.cuda.synchronize()
     assert pa.pa_device_status() == pa.PA_DEV_BAD_CONTEXT
     got = out.float().cpu().numpy()

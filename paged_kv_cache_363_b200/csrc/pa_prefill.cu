@@ -11,9 +11,11 @@
 // A work item is one (sequence, kv head) and two query tiles A and B of 128 rows each.
 // A tile's rows are T query tokens x G query heads of the kv head's group (T = 128 / G),
 // so every K/V byte loaded serves both tiles and all G heads.  With a workspace
-// (pa_prefill_ws) one CTA per SM claims items from a counter, last query tokens first,
-// and starts an item's Q load and first S while its previous item ends; without one
-// (pa_prefill) CTA b runs item b alone.  An item walks the keys in tiles of 128 tokens:
+// (pa_prefill_ws) one CTA per SM claims items from a counter, and starts an item's Q
+// load and first S while its previous item ends; without one (pa_prefill) CTA b runs
+// item b alone.  Items go in chunks of 16 (sequence, kv head) groups, the last query
+// tokens of the chunk's groups first, so the CTAs that run together share a few
+// groups' K/V in L2.  An item walks the keys in tiles of 128 tokens:
 //   - warp 16 claims the items and passes them, with their geometry, through a ring of
 //     two shared-memory slots; it stages both Q tiles once per item and each K and V
 //     tile by TMA, one 16-row box per (16-token run of a physical block, 64 columns),
@@ -78,6 +80,7 @@ constexpr int OFF_K = OFF_Q + kQT * 2 * kQHalf;
 constexpr int OFF_V = OFF_K + KST * 2 * kKVHalf;
 constexpr int kTiles = OFF_V + VST * 2 * kKVHalf;
 constexpr int IR = 2;  // item ring: the item in work and the next
+constexpr int kChunkGroups = 16;  // (sequence, kv head) groups whose items are interleaved
 // barriers: q_full, q_empty, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], per query tile
 // {s_full, p_full, o_done, o_free}, drain, it_full[IR], it_empty[IR]
 constexpr int NBAR = 2 + 2 * KST + 2 * VST + kQT * 4 + 1 + 2 * IR;
@@ -164,11 +167,16 @@ template <int G>
 __device__ __forceinline__ bool item_geom(const PrefillArgs& a, int npairs, int item, Item& it)
 {
     constexpr int T = kM / G;
-    const int per = a.num_seqs * a.num_kv_heads;
-    it.pair = npairs - 1 - item / per;
-    const int rem = item % per;
-    it.s = rem / a.num_kv_heads;
-    it.kvh = rem % a.num_kv_heads;
+    // groups = (sequence, kv head) pairs, kChunkGroups at a time; inside a chunk the last query tokens come first,
+    // across its groups.  The CTAs that run together then share a few groups' K/V, which stays in L2.
+    const int ngroups = a.num_seqs * a.num_kv_heads;
+    const int chunk = item / (kChunkGroups * npairs);
+    const int cg = min(kChunkGroups, ngroups - chunk * kChunkGroups);  // groups in this chunk
+    const int idx = item - chunk * kChunkGroups * npairs;
+    it.pair = npairs - 1 - idx / cg;
+    const int grp = chunk * kChunkGroups + idx % cg;
+    it.s = grp / a.num_kv_heads;
+    it.kvh = grp % a.num_kv_heads;
     it.q0 = __ldg(a.q_start + it.s);
     const int q1 = __ldg(a.q_start + it.s + 1);
     it.n = q1 - it.q0;

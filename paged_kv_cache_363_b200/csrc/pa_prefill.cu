@@ -64,7 +64,7 @@ constexpr int kQHalf = kM * 128;   // bytes of a 64-column half of a Q tile (16 
 constexpr int kKVHalf = kN * 128;  // bytes of a 64-column half of a K or V tile (16 KB)
 constexpr int kBox = 16;           // rows per TMA box of K/V (one 16-token run of a block)
 constexpr int kNBox = kN / kBox;   // boxes per K/V tile
-constexpr int kQT = 2;             // query tiles per CTA, sharing every K/V tile
+constexpr int kQT = 2;             // query tiles per work item, sharing every K/V tile
 constexpr int kThreads = 576;      // 8 softmax warps per query tile (two per row), producer, MMA issuer
 constexpr int kProdWarp = 16, kMmaWarp = 17;
 constexpr uint32_t kTmemCols = 512;  // per query tile: S 0..127 (P over 0..63 once S is read), O 128..255

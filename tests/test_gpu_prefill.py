@@ -204,3 +204,31 @@ def test_any_finite_scale(pa, scale):
     got = _run(pa, q, k, v, tables, L, qs, scale)
     assert np.isfinite(got).all()
     assert max_abs(got, _oracle(q, k, v, tables, L, qs, scale)) <= TOL["bf16"]
+
+
+def test_workspace_call_replays_from_a_cuda_graph(pa):
+    """pa_prefill_ws zeroes its counter on the stream before the launch, so a captured call replays: every
+    replay of the graph gives the direct call's bits."""
+    q, k, v, tables, L, qs = _case(77, [300, 129, 1000], [300, 17, 64], 8, 2, 16)
+    want = _run(pa, q, k, v, tables, L, qs, 0.09)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    td, ld, sd = torch.from_numpy(tables).cuda(), torch.from_numpy(L).cuda(), torch.from_numpy(qs).cuda()
+    ws = torch.empty(pa.pa_prefill_workspace_size(), dtype=torch.uint8, device="cuda")
+    out = torch.full(q.shape, 7.0, dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        pa.pa_prefill(out, qd, kd, vd, td, ld, sd, int(np.max(np.diff(qs))), 0.09, stream=s, workspace=ws)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        pa.pa_prefill(out, qd, kd, vd, td, ld, sd, int(np.max(np.diff(qs))), 0.09,
+                      stream=torch.cuda.current_stream(), workspace=ws)
+    for _ in range(3):
+        out.fill_(7.0)
+        g.replay()
+        torch.cuda.synchronize()
+        assert np.array_equal(out.float().cpu().numpy(), want)
+    assert pa.pa_device_status() == 0
+    del g

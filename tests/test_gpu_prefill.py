@@ -232,3 +232,15 @@ def test_workspace_call_replays_from_a_cuda_graph(pa):
         assert np.array_equal(out.float().cpu().numpy(), want)
     assert pa.pa_device_status() == 0
     del g
+
+
+@pytest.mark.parametrize("ws", [True, False])
+def test_sequences_without_queries(pa, ws):
+    """Sequences with no query rows (n_s = 0, with or without context) have no work items; the others match the
+    oracle and no status bit is raised."""
+    lens, nq = [50, 0, 300, 40, 1], [10, 0, 0, 40, 1]
+    q, k, v, tables, L, qs = _case(91, [max(x, 1) for x in lens], nq, 4, 2, 16)
+    L = np.array(lens, np.int32)
+    got = _run(pa, q, k, v, tables, L, qs, 0.1, ws=ws)
+    assert pa.pa_device_status() == 0
+    assert max_abs(got, _oracle(q, k, v, tables, L, qs, 0.1)) <= TOL["bf16"]

@@ -141,10 +141,11 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[32
 }
 
 // One work item: query tokens [t_lo0, t_lo0 + 2T) of sequence s (two query tiles of T tokens x G heads) for
-// kv head kvh.  Items are numbered with the last query tokens of every (sequence, kv head) first, since those
-// see the most keys.  With a counter (a.sched) a grid of one CTA per SM claims them in that order, so a CTA
-// that finishes early takes more; without one, CTA b takes item b alone.  The producer warp claims the items
-// and hands them to the MMA thread and the softmax warps through a ring of IR slots in shared memory.
+// kv head kvh.  Items are numbered by chunks of kChunkGroups (sequence, kv head) groups, and inside a chunk
+// with the last query tokens (which see the most keys) first.  With a counter (a.sched) a grid of one CTA per
+// SM claims them in that order, so a CTA that finishes early takes more; without one, CTA b takes item b
+// alone.  The producer warp claims the items and hands them to the MMA thread and the softmax warps through
+// a ring of IR slots in shared memory.
 struct Item {
     int s, kvh, pair, q0, n, L, t_lo0, nqt, nA, nB, ntiles;
     bool bad;

@@ -80,9 +80,12 @@ typedef enum { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
 /*
  * Context-partition length (tokens) that pa_decode uses for these arguments:
  * `partition_size` itself when > 0 (it must be a multiple of block_size, at most
- * 4096), else an automatic choice.  A sequence longer than one partition is
- * split into partitions whose softmax states are merged by log-sum-exp in a
- * second kernel.  Returns a negative pa_status on invalid arguments.
+ * 4096), else the shortest length of the automatic choice (512), which the call may
+ * lengthen by doubling, up to 4096, from the batch's size and context lengths (the
+ * workspace sized for the shortest length serves every longer one).  A sequence
+ * longer than one partition is split into partitions whose softmax states are merged
+ * by log-sum-exp in a second kernel.  Returns a negative pa_status on invalid
+ * arguments.
  */
 PA_API int pa_decode_partition_size(int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
                              int max_context_len, int partition_size);

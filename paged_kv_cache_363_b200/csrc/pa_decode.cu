@@ -547,12 +547,19 @@ cudaError_t launch_persistent(const DecodeArgs& a, cudaStream_t stream)
     const unsigned grid = (unsigned)(units < ctas ? units : ctas);
     DecodeArgs args = a;
     args.num_ctas = (int)grid;
+    // An automatic partition starts at 1024 tokens instead of 512 when the batch has at least three
+    // (sequence, kv head) pairs per CTA, so that units twice as long still balance, and a context bound of
+    // 3072 tokens or more, so that long sequences split into half as many partitions to merge.  Plan and run
+    // calls take the same arguments, so they make the same choice.
+    if (a.adaptive && a.partition_blocks * BS == 512 && (int64_t)a.num_seqs * a.num_kv_heads >= 3LL * grid &&
+        a.max_context_len >= 3072)
+        args.partition_blocks = 1024 / BS;
     // The first wave: with the partition fixed, CTA b < first_wave starts on kv head
     // b % Hkv of partition 0 of sequence b / Hkv without waiting for the plan.  The plan
     // grows an automatic partition only when the tokens of all sequences exceed
     // 4 x partition x CTAs, which the bound num_seqs x max_context_len rules out here.
     const bool fixed_partition =
-        !a.adaptive || (int64_t)a.num_seqs * a.max_context_len <= 4LL * a.partition_blocks * BS * (int64_t)grid;
+        !a.adaptive || (int64_t)a.num_seqs * a.max_context_len <= 4LL * args.partition_blocks * BS * (int64_t)grid;
     const int64_t pairs0 = (int64_t)a.num_seqs * a.num_kv_heads;
     args.first_wave = fixed_partition ? (int)(pairs0 < (int64_t)grid ? pairs0 : (int64_t)grid) : 0;
 

@@ -547,12 +547,14 @@ cudaError_t launch_persistent(const DecodeArgs& a, cudaStream_t stream)
     const unsigned grid = (unsigned)(units < ctas ? units : ctas);
     DecodeArgs args = a;
     args.num_ctas = (int)grid;
-    // An automatic partition starts at 1024 tokens instead of 512 when the batch has at least three
-    // (sequence, kv head) pairs per CTA, so that units twice as long still balance, and a context bound of
-    // 3072 tokens or more, so that long sequences split into half as many partitions to merge.  Plan and run
-    // calls take the same arguments, so they make the same choice.
-    if (a.adaptive && a.partition_blocks * BS == 512 && (int64_t)a.num_seqs * a.num_kv_heads >= 3LL * grid &&
-        a.max_context_len >= 3072)
+    // An automatic partition starts at 1024 tokens instead of 512 when units twice as long still balance and
+    // halving the partitions saves merge work: at least three (sequence, kv head) pairs per CTA with a context
+    // bound of 3072 tokens or more (long sequences split into half as many partitions), or at least ten pairs
+    // per CTA (many sequences just over one partition).  Plan and run calls take the same arguments, so they
+    // make the same choice.
+    const int64_t pairs_all = (int64_t)a.num_seqs * a.num_kv_heads;
+    if (a.adaptive && a.partition_blocks * BS == 512 &&
+        ((pairs_all >= 3LL * grid && a.max_context_len >= 3072) || pairs_all >= 10LL * grid))
         args.partition_blocks = 1024 / BS;
     // The first wave: with the partition fixed, CTA b < first_wave starts on kv head
     // b % Hkv of partition 0 of sequence b / Hkv without waiting for the plan.  The plan

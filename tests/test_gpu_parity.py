@@ -394,12 +394,14 @@ def test_cow_small_pool_bit_exact(pa, runner):
     _status_clean(pa)
 
 
-@pytest.mark.parametrize("wid,part", [(3, 0), (2, 256), (5, 512), (1, 0)])
-def test_plan_once_then_run_per_layer(pa, runner, wid, part):
+@pytest.mark.parametrize("wid,part,full", [(3, 0, False), (3, 0, True), (2, 256, False), (5, 512, False),
+                                           (1, 0, False)])
+def test_plan_once_then_run_per_layer(pa, runner, wid, part, full):
     """One plan per step, one run per layer: each run equals a whole pa_decode of the
     same layer bit for bit (the runs reuse the plan; the last CTA of each resets its
-    work counter, or the next run would skip units)."""
-    over = {"num_seqs": 40, "num_blocks": 6000} if wid in (2, 3) else {}
+    work counter, or the next run would skip units).  The full-size GQA batch takes the
+    1024-token starting partition, which plan and run must both choose."""
+    over = {"num_seqs": 40, "num_blocks": 6000} if wid in (2, 3) and not full else {}
     wl = W.make_workload(wid, seed=2, **over)
     wl.partition_size = part
     batch = runner.DecodeBatch(wl, "cuda")
@@ -409,6 +411,11 @@ def test_plan_once_then_run_per_layer(pa, runner, wid, part):
                      dtype=torch.uint8, device="cuda")
     pa.pa_decode_plan(batch.block_tables, batch.context_lens, batch.max_context_len, wl.num_heads, batch.k_cache, ws,
                       part)
+    if full:
+        # 1024 (sequence, kv head) pairs and contexts up to 4096: the plan starts at 1024 tokens
+        torch.cuda.synchronize()
+        pb = int(ws[8:12].cpu().view(torch.int32)[0])
+        assert pb * wl.block_size == 1024, pb
     g = torch.Generator(device="cuda").manual_seed(wid)
     for layer in range(4):
         q = torch.randn(batch.q.shape, generator=g, device="cuda").to(batch.q.dtype)

@@ -31,9 +31,10 @@
 //     halves of a row swap partial maxima through shared memory at a hardware barrier
 //     over their 64 threads.  The running max is kept in base-2 units, and O is
 //     rescaled in tensor memory only when it grows by more than 8 (2^8: exact up to
-//     rounding).  Exponentials are taken two at a time in fp16 (ex2.approx.f16x2: 11
-//     significant bits, more than P's 8).  P goes as bf16 over the first 64 columns of
-//     S; at the end the halves add up their row sums and store O.
+//     rounding).  The exponent arguments are formed two at a time (fma.rn.f32x2), the
+//     exponentials in fp32 (an fp16 pair costs the transcendental unit as much as two
+//     fp32 ones and needs conversions both ways).  P goes as bf16 over the first 64
+//     columns of S; at the end the halves add up their row sums and store O.
 // One CTA per SM: 197 KB of shared memory, all 512 tensor-memory columns (per query
 // tile S 128 + O 128).  A tile's O is taken by its next item only after the softmax has
 // read it out, and its S only after the previous P.V.
@@ -42,7 +43,6 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -98,13 +98,21 @@ __device__ __forceinline__ float fast_exp2(float x)
     return y;
 }
 
-// 2^x for two arguments at once: rounded to fp16 on the way in (11 significant bits, as many as the result's)
-__device__ __forceinline__ float2 exp2_pair(float x0, float x1)
+// a pair of floats in one 64-bit register, for the f32x2 instructions
+__device__ __forceinline__ uint64_t pack2f(float lo, float hi)
 {
-    const __half2 h = __floats2half2_rn(x0, x1);
-    uint32_t y;
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(y) : "r"(*reinterpret_cast<const uint32_t*>(&h)));
-    return __half22float2(*reinterpret_cast<const __half2*>(&y));
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+// (x0, x1) = (s0, s1) * b + c, elementwise over the pairs b and c, in one instruction
+__device__ __forceinline__ void ffma2(float& x0, float& x1, uint32_t s0, uint32_t s1, uint64_t b, uint64_t c)
+{
+    asm("{\n\t.reg .b64 ra, rd;\n\tmov.b64 ra, {%2, %3};\n\t"
+        "fma.rn.f32x2 rd, ra, %4, %5;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(x0), "=f"(x1)
+        : "r"(s0), "r"(s1), "l"(b), "l"(c));
 }
 
 // A barrier over the 64 threads of the two warps that share a row quarter (hardware barrier `id`), returning the
@@ -600,13 +608,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (rescale || m_used == -INFINITY) m_used = m_new;
                 const float mref = m_used == -INFINITY ? 0.f : m_used;
                 float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
+                const uint64_t slp = pack2f(sl, sl), mrp = pack2f(-mref, -mref);
 #pragma unroll
                 for (int c = 0; c < NC; ++c) {
 #pragma unroll
                     for (int e2 = 0; e2 < 16; ++e2) {
-                        const float2 pp = exp2_pair(fmaf(__uint_as_float(sr[c][2 * e2]), sl, -mref),
-                                                    fmaf(__uint_as_float(sr[c][2 * e2 + 1]), sl, -mref));
-                        float p0 = pp.x, p1 = pp.y;
+                        float x0, x1;
+                        ffma2(x0, x1, sr[c][2 * e2], sr[c][2 * e2 + 1], slp, mrp);
+                        float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
                         if (mask_tile) {
                             const int kv = kv0 + c * 32 + 2 * e2;
                             p0 = kv <= lim ? p0 : 0.f;

@@ -413,10 +413,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const volatile int* sp = item_slot + (nit % IR) * kSlotInts;
                 const int item = sp[0];
-                mbar_arrive(&it_empty[nit % IR]);
-                if (item < 0) break;
                 Item it;
-                get_item(sp, it);
+                if (item >= 0) get_item(sp, it);
+                mbar_arrive(&it_empty[nit % IR]);  // after the slot's last read
+                if (item < 0) break;
                 const int nA = it.nA, nB = it.nB;
                 ok = mbar_wait_bounded(q_full, nit & 1, abort_flag) &&
                      mbar_wait_bounded(&k_full[gt % KST], (gt / KST) & 1, abort_flag);
@@ -664,6 +664,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(p_full);
             }
+            // the output's place, read before the slot is released (the producer may then refill it)
+            Item it;
+            get_item(slot_k, it);
+            const int tq = it.t_lo0 + qt * T + t_local;
+            const bool valid_row = t_local < T && tq < it.n;
+            __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) +
+                                 ((size_t)(it.q0 + tq) * a.num_heads + (size_t)it.kvh * G + g) * kD + half * 64;
+            __syncwarp();
             // both warps of the pair always get here, with the same number of exchanges behind them
             const bool ok_o = ok && mbar_wait_warp(o_done, (cnt + ntq - 1) & 1, abort_flag);
             if (lane == 0) mbar_arrive(&it_empty[k % IR]);
@@ -677,12 +685,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after_sync();
             l += *xslot((xc - 1) & 1, half ^ 1);
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            Item it;
-            get_item(slot_k, it);
-            const int tq = it.t_lo0 + qt * T + t_local;
-            const bool valid_row = t_local < T && tq < it.n;
-            __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) +
-                                 ((size_t)(it.q0 + tq) * a.num_heads + (size_t)it.kvh * G + g) * kD + half * 64;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t o[32];

@@ -244,3 +244,40 @@ def test_sequences_without_queries(pa, ws):
     got = _run(pa, q, k, v, tables, L, qs, 0.1, ws=ws)
     assert pa.pa_device_status() == 0
     assert max_abs(got, _oracle(q, k, v, tables, L, qs, 0.1)) <= TOL["bf16"]
+
+
+def test_many_small_items_through_the_ring(pa):
+    """4,800 items of one to four key tiles each (600 short sequences x 8 kv heads): every CTA of the
+    persistent grid takes ~32 of them, so the two-slot item ring is refilled as fast as it can be.  A reader
+    that used a slot after releasing it would put rows in the wrong place; every row is compared."""
+    rng = np.random.default_rng(31)
+    g = torch.Generator().manual_seed(31)
+    S, Hkv, G, B, D = 600, 8, 4, 16, 128
+    lens = rng.integers(1, 201, size=S).astype(np.int32)
+    nq = np.minimum(lens, rng.integers(1, 41, size=S)).astype(np.int32)
+    nblk = -(-lens // B)
+    NB = int(nblk.sum()) + 7
+    order = rng.permutation(NB).astype(np.int32)
+    tables = np.full((S, int(nblk.max())), -1, np.int32)
+    starts = np.concatenate([[0], np.cumsum(nblk)])
+    for s in range(S):
+        tables[s, :nblk[s]] = order[starts[s]:starts[s + 1]]
+    # the context's slots get random rows; every other slot of the pools stays NaN
+    tok_s = np.repeat(np.arange(S), lens)
+    tok_t = np.concatenate([np.arange(L) for L in lens])
+    blk = torch.from_numpy(tables[tok_s, tok_t // B].astype(np.int64))
+    off = torch.from_numpy((tok_t % B).astype(np.int64))
+    k = torch.full((NB, Hkv, B, D), float("nan"), dtype=torch.bfloat16)
+    v = torch.full((NB, Hkv, B, D), float("nan"), dtype=torch.bfloat16)
+    k[blk, :, off] = torch.randn(len(tok_s), Hkv, D, generator=g).to(torch.bfloat16)
+    v[blk, :, off] = torch.randn(len(tok_s), Hkv, D, generator=g).to(torch.bfloat16)
+    q_start = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    q = torch.randn(int(q_start[-1]), Hkv * G, D, generator=g).to(torch.bfloat16)
+    scale = 128 ** -0.5
+    got = _run(pa, q, k, v, tables, lens, q_start, scale, calls=3)
+    assert np.isfinite(got).all()
+    err = max_abs(got, _oracle(q, k, v, tables, lens, q_start, scale))
+    report_error("prefill, 600 short sequences (4,800 small items)", err, got.shape[0] * got.shape[1])
+    assert err <= TOL["bf16"], err
+    assert np.array_equal(_run(pa, q, k, v, tables, lens, q_start, scale, ws=False), got)
+    assert pa.pa_device_status() == 0

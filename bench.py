@@ -199,6 +199,20 @@ def l2_note(batch, logical_bytes):
             "the %.0f MB of logical bytes" % (unique / 1e6, logical_bytes / 1e6))
 
 
+def partition_used(batch, wl):
+    """Tokens per context partition that the last decode call used: the plan kernel writes
+    its choice, in blocks, to word 2 of the workspace.  The automatic choice may be longer
+    than the starting value pa_decode_partition_size reports."""
+    import torch
+    return int(batch.workspace[:4].view(torch.int32)[2].item()) * wl.block_size
+
+
+def partition_entry(batch, wl, start):
+    """The partition as requested (config's partition_size: 0 = automatic, as the reference
+    line reports it) and as run: the starting value and the plan's final choice, in tokens."""
+    return {"partition_size": wl.partition_size, "partition_start": start, "partition_used": partition_used(batch, wl)}
+
+
 def workload_config(wl, partition, batch=None):
     cfg = {"workload": wl.name, "num_heads": wl.num_heads, "num_kv_heads": wl.num_kv_heads,
            "head_dim": wl.head_dim, "block_size": wl.block_size, "num_blocks": wl.num_blocks,
@@ -654,8 +668,10 @@ def side_workload(name, args, dev, world, rank):
     return {"value": round(world * step_bytes * steps / (t["ms_max"] * 1e-3) / 1e9, 2), "unit": "GB/s",
             "steps": steps, "ms_per_step": round(t["ms_max"] / steps, 5),
             "seqs_per_s": round(world * wl.num_seqs * steps / (t["ms_max"] * 1e-3), 1),
-            "config": dict(workload_config(wl, part, batch), l2=l2_note(batch, dec_bytes)),
-            "roofline": roof, "gpu_launches": decode_launches(batch, -(-batch.max_context_len // part)) * steps,
+            "config": dict(workload_config(wl, part, batch), l2=l2_note(batch, dec_bytes),
+                           **partition_entry(batch, wl, part)),
+            "roofline": roof,
+            "gpu_launches": decode_launches(batch, -(-batch.max_context_len // partition_used(batch, wl))) * steps,
             "clocks": t["clocks"],
             "device_status": t["flags"], "output_finite": t["out_ok"]}
 
@@ -766,10 +782,9 @@ def run_gpu(args):
 
     dec_bytes = batch.decode_bytes()
     step_bytes = dec_bytes + batch.append_bytes()
-    launches_per_step = decode_launches(batch, -(-batch.max_context_len // part))
-
     # ---- device-resident timing
     t = time_decode_steps(batch, stream, args.steps, args.warmup, dev, world)
+    launches_per_step = decode_launches(batch, -(-batch.max_context_len // partition_used(batch, wl)))
     ms_max, dec_ms, dec_avg_max = t["ms_max"], t["dec_ms"], t["dec_avg_max"]
     out_ok, flags = t["out_ok"], t["flags"]
 
@@ -800,7 +815,7 @@ def run_gpu(args):
         "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
         "config": dict(workload_config(wl, part, batch), l2=l2_note(batch, dec_bytes),
-                       parallelism="replicas: one batch per GPU (dp%d)" % world),
+                       parallelism="replicas: one batch per GPU (dp%d)" % world, **partition_entry(batch, wl, part)),
         "seqs_per_s": round(world * wl.num_seqs * args.steps / (ms_max * 1e-3), 1),
         "pct_of_peak": round(100.0 * value / peak, 2),
         "roofline": {"bound": "hbm", "kernel": "pa_decode (plan kernel + persistent decode kernel + merge)",
